@@ -1,0 +1,228 @@
+/*
+ * km.h -- C ABI of the B200 (sm_100a) exact Lloyd K-Means library (libkm.so).
+ *
+ * The method is the one described in "Flash-KMeans: Fast and Memory-Efficient
+ * Exact K-Means":
+ *   - §2.1 FlashAssign: the nearest-centroid assignment computed by fusing the
+ *     distance tile ||x||^2 - 2 x.c + ||c||^2 with an online per-row argmin,
+ *     so no N x K distance matrix is ever written to device memory;
+ *   - §2.2 Sort-Inverse Update: the centroid update formed by sorting the
+ *     assignment vector (an explicit inverse map from cluster to points) and
+ *     reducing contiguous same-cluster segments on chip, instead of scattering
+ *     every point into its cluster with atomics;
+ *   - §2.3 Chunked Stream Overlap: points held in host memory are streamed in
+ *     chunks, with copies overlapping compute.
+ * §2 states that the mathematics of standard Lloyd K-Means is unchanged, so
+ * every entry point computes exact Lloyd iterations (up to floating-point
+ * rounding of the stated precisions).
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  - Pointers are DEVICE pointers owned by the caller unless a parameter says
+ *    "host".  The library never allocates or frees device memory: all scratch
+ *    comes from the caller's `workspace` (size from km_workspace_size).
+ *    Workspace base must be 256-byte aligned (cudaMalloc/torch allocations are).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Unless stated,
+ *    work is enqueued asynchronously and the call returns without waiting.
+ *  - Layouts are row-major and contiguous.  B >= 1 independent problems are
+ *    stacked: instance b owns X + b*N*D, C + b*K*D, idx + b*N, counts + b*K.
+ *  - dtype: KM_BF16 (X and centroid operands in bfloat16; the distance dot
+ *    products run on the tensor cores with float32 accumulation) or KM_F32
+ *    (float32 inputs; dot products use a three-term TF32 split, hi*hi + hi*lo
+ *    + lo*hi, on the tensor cores, which keeps float32-level accuracy).
+ *  - Centroid outputs are float32.  Assignments are int32 in [0, K).
+ *  - Ties: the lowest centroid index wins an exact tie.  A cluster with no
+ *    member keeps its previous centroid (the pages fix neither rule; these are
+ *    the plain readings).
+ *  - Supported shapes: D % 8 == 0; bf16: 8 <= D <= 256; f32: 8 <= D <= 64;
+ *    1 <= K <= min(N, 1 << 20); N < 2^31.  Others return KM_ERR_UNSUPPORTED
+ *    or KM_ERR_INVALID_ARG before anything is launched.
+ *  - Inputs containing NaN or Inf give unspecified (but memory-safe) results.
+ *  - Every wait inside a kernel is bounded in time; a wait that runs out sets
+ *    a status word in the workspace and the kernel returns early.  Read it with
+ *    km_workspace_status().  Entry points that synchronise (km_fit_host,
+ *    km_workspace_status) report it as KM_ERR_TIMEOUT.
+ *  - Errors: a non-zero km_status; km_last_error() gives a message for the
+ *    calling thread.
+ *  - Calls on distinct workspaces may run concurrently; calls sharing one
+ *    workspace must be ordered (same stream or synchronised).
+ */
+#ifndef KM_H_
+#define KM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KM_VERSION 1
+
+typedef enum km_status {
+  KM_OK = 0,
+  KM_ERR_INVALID_ARG = 1, /* null required pointer, bad size, misaligned pointer */
+  KM_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve (shape, device) */
+  KM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  KM_ERR_WORKSPACE = 4,   /* workspace null or smaller than km_workspace_size() */
+  KM_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out */
+} km_status;
+
+typedef enum km_dtype { KM_F32 = 0, KM_BF16 = 1 } km_dtype;
+
+typedef enum km_op {
+  KM_OP_ASSIGN = 0,  /* km_assign */
+  KM_OP_UPDATE = 1,  /* km_update */
+  KM_OP_FIT = 2,     /* km_fit */
+  KM_OP_FIT_HOST = 3, /* km_fit_host (uses chunk_rows) */
+  KM_OP_ARGSORT = 4   /* km_argsort (D and dtype ignored) */
+} km_op;
+
+/* Library version (KM_VERSION of the build). */
+int km_version(void);
+
+/* Static string for a km_status value. */
+const char* km_status_string(int status);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* km_last_error(void);
+
+/*
+ * Bytes of workspace the operation needs for this shape (0 if the shape is
+ * invalid or unsupported; km_last_error() says why).  The size is O(B*N + K*D)
+ * (plus 2*chunk_rows*D elements for KM_OP_FIT_HOST); never O(N*K).
+ */
+size_t km_workspace_size(int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows);
+
+/*
+ * Synchronise `stream`, read and clear the workspace status word.
+ * Returns KM_OK, or KM_ERR_TIMEOUT if a kernel that used this workspace gave
+ * up on a bounded wait since the status was last cleared.
+ */
+int km_workspace_status(void* workspace, void* stream);
+
+/*
+ * FlashAssign (Flash-KMeans §2.1): for every point i of every instance,
+ *   idx[i]     = argmin_k ||x_i - c_k||^2   (lowest k on exact ties)
+ *   mindist[i] = max(0, ||x_i||^2 - 2 x_i.c_idx + ||c_idx||^2)
+ * computed tile by tile with an online argmin; the N x K distances never
+ * reach device memory.
+ *   X        [B][N][D] dtype, device, read only.
+ *   C        [B][K][D] dtype, device, read only.
+ *   idx      [B][N] int32, device, written.
+ *   mindist  [B][N] float, device, written; may be NULL.
+ *   objective [B] double, device, written (sum of mindist per instance, in a
+ *            fixed order); may be NULL.
+ * X and C (bf16) must be 16-byte aligned.
+ */
+int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int dtype,
+              int32_t* idx, float* mindist, double* objective,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Sort-Inverse Update (Flash-KMeans §2.2): new centroids as member means.
+ * The assignment vector is argsorted by a device radix sort (stable, so the
+ * order is deterministic), same-cluster runs of the sorted order are summed on
+ * chip in float32, and only run boundaries are combined across thread blocks,
+ * in a fixed order (no atomics on centroid sums; results are bitwise
+ * reproducible run to run).
+ *   X       [B][N][D] dtype, device, read only.
+ *   idx     [B][N] int32 in [0, K), device, read only (values outside [0,K)
+ *           are undefined behaviour).
+ *   C       [B][K][D] float, device, in: previous centroids (kept for empty
+ *           clusters), out: updated centroids.
+ *   counts  [B][K] int32, device, written: members per cluster; may be NULL.
+ */
+int km_update(const void* X, const int32_t* idx, int B, int64_t N, int D, int K, int dtype,
+              float* C, int32_t* counts,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The explicit inverse map of the Sort-Inverse Update (Flash-KMeans §2.2:
+ * argsort of the assignment vector so that each cluster's points become a
+ * contiguous run).  Stable: points of one cluster keep increasing index, so
+ * the permutation is unique.
+ *   idx    [N] int32 in [0, K), device, read only (out-of-range ids are
+ *          clamped into [0, K); they are not valid input).
+ *   perm   [N] int32, device, written: point indices ordered by cluster.
+ *   start  [K+1] int32, device, written: start[k] = first position of
+ *          cluster k in perm, start[K] = N (so count_k = start[k+1]-start[k]);
+ *          may be NULL.
+ * Workspace: km_workspace_size(KM_OP_ARGSORT, 1, N, 0, K, 0, 0).
+ */
+int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* start,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * `iters` Lloyd iterations (assign then update) from the initial centroids C0.
+ * Iteration t (1-based) assigns under C_{t-1}; objective_hist[b*iters + t-1]
+ * is the sum of squared distances of that assignment.  After the call
+ * C_out = C_iters, idx_out = the assignment of iteration `iters`, and
+ * counts_out = its cluster sizes.  In bf16 mode the centroids are kept in
+ * float32 and a bfloat16 copy (round to nearest even) feeds the next
+ * assignment.
+ *   X              [B][N][D] dtype, device.
+ *   C0             [B][K][D] dtype, device (may alias nothing written).
+ *   C_out          [B][K][D] float, device, written.
+ *   idx_out        [B][N] int32, device, written; may be NULL.
+ *   counts_out     [B][K] int32, device, written; may be NULL.
+ *   objective_hist [B][iters] double, DEVICE, written; may be NULL.
+ */
+int km_fit(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
+           float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * km_fit with per-iteration phase timing, for profiling: CUDA events are
+ * recorded on `stream` right before and after the assignment kernel and after
+ * the update of every iteration.  Synchronous (waits for the stream).
+ *   phase_ms  [2*iters + 1] float, HOST, written: for iteration t,
+ *             phase_ms[2t] = milliseconds of the assignment kernel and
+ *             phase_ms[2t+1] = milliseconds of the whole update (argsort,
+ *             segmented sums, finalise); phase_ms[2*iters] = milliseconds from
+ *             the start of the first assignment to the end of the last update
+ *             (the iterations alone, without the one-time operand preparation).
+ * Other arguments as km_fit.
+ */
+int km_fit_profile(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
+                   float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist,
+                   void* workspace, size_t workspace_bytes, void* stream, float* phase_ms);
+
+/*
+ * Number of kernels this library has enqueued in this process since it was
+ * loaded (all entry points, all threads).  For accounting in benchmarks.
+ */
+uint64_t km_launch_count(void);
+
+/*
+ * km_fit for one instance whose points live in HOST memory (Flash-KMeans §2.3
+ * Chunked Stream Overlap, out-of-core execution).  Each iteration streams X to
+ * the device in chunks of `chunk_rows` rows through two device buffers: the
+ * copy of chunk c+1 runs on a library-owned copy stream while chunk c is
+ * assigned, sorted and reduced on `stream`.  Per-cluster sums are accumulated
+ * across chunks in float64, in chunk order.
+ *   X_host         [N][D] dtype, HOST, page-locked (cudaHostAlloc or
+ *                  cudaHostRegister); read only.
+ *   C0, C_out, idx_out, counts_out: as km_fit (device).
+ *   objective_hist [iters] double, HOST, written; may be NULL.
+ * This call is synchronous: it returns after all work finished, and reports a
+ * kernel timeout as KM_ERR_TIMEOUT.
+ */
+int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int dtype, int iters,
+                int64_t chunk_rows, float* C_out, int32_t* idx_out, int32_t* counts_out,
+                double* objective_hist, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one CTA that waits on a
+ * shared-memory barrier that nothing ever arrives on, with the given limit in
+ * nanoseconds (at most 10^9).  The kernel gives up, sets the workspace status
+ * word and returns, leaving the context usable.  Synchronous.  Returns the
+ * status km_workspace_status() then reports (KM_ERR_TIMEOUT when it works).
+ */
+int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KM_H_ */

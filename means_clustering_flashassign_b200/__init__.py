@@ -1,0 +1,297 @@
+"""Exact Lloyd K-Means on B200 (sm_100a): FlashAssign + Sort-Inverse Update.
+
+Thin Python binding of ``libkm.so`` (C ABI in ``include/km.h``).  This module
+only marshals arguments: it checks shapes, allocates outputs and workspace with
+torch (device memory and streams are the only things torch provides) and calls
+the C entry points, which run every step of the computation in CUDA kernels.
+There is no CPU or PyTorch fallback: if the library is missing or the GPU is
+not an sm_100 part, calls raise.
+
+Method: "Flash-KMeans: Fast and Memory-Efficient Exact K-Means", §2.1
+FlashAssign (fused distance tiles + online argmin, no N x K matrix in device
+memory), §2.2 Sort-Inverse Update (argsort of the assignment vector +
+segmented on-chip reduction), §2.3 Chunked Stream Overlap (host-resident points
+streamed in chunks).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+__all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
+           "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "OP_ARGSORT",
+           "F32", "BF16", "EXPORTS"]
+
+OP_ASSIGN, OP_UPDATE, OP_FIT, OP_FIT_HOST, OP_ARGSORT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_ERR_CUDA",
+          4: "KM_ERR_WORKSPACE", 5: "KM_ERR_TIMEOUT"}
+EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
+           "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
+           "km_launch_count"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KMError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+        self.message = message
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def library() -> ctypes.CDLL:
+    """Load libkm.so (building it first if the sources are newer)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if not _build.up_to_date():
+                path = _build.build()
+            if not os.path.exists(path):
+                raise RuntimeError(f"libkm.so not found at {path}; run means_clustering_flashassign_b200.build")
+            L = ctypes.CDLL(path)
+            P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+            L.km_version.restype = I
+            L.km_status_string.argtypes = [I]
+            L.km_status_string.restype = ctypes.c_char_p
+            L.km_last_error.restype = ctypes.c_char_p
+            L.km_workspace_size.argtypes = [I, I, I64, I, I, I, I64]
+            L.km_workspace_size.restype = SZ
+            L.km_workspace_status.argtypes = [P, P]
+            L.km_assign.argtypes = [P, P, I, I64, I, I, I, P, P, P, P, SZ, P]
+            L.km_update.argtypes = [P, P, I, I64, I, I, I, P, P, P, SZ, P]
+            L.km_fit.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P]
+            L.km_fit_host.argtypes = [P, P, I64, I, I, I, I, I64, P, P, P, P, P, SZ, P]
+            L.km_selftest_timeout.argtypes = [P, SZ, I64, P]
+            L.km_argsort.argtypes = [P, I64, I, P, P, P, SZ, P]
+            L.km_fit_profile.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
+            L.km_launch_count.restype = ctypes.c_uint64
+            for f in EXPORTS:
+                getattr(L, f).restype = getattr(L, f).restype or I
+            _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = library().km_last_error().decode(errors="replace")
+        raise KMError(status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"points must be bfloat16 or float32, got {t.dtype}")
+
+
+def _shape3(X: torch.Tensor, name: str):
+    if X.dim() == 2:
+        return 1, X.shape[0], X.shape[1], False
+    if X.dim() == 3:
+        return X.shape[0], X.shape[1], X.shape[2], True
+    raise ValueError(f"{name} must be (N, D) or (B, N, D)")
+
+
+def workspace_size(op: int, B: int, N: int, D: int, K: int, dtype: int, chunk_rows: int = 0) -> int:
+    n = library().km_workspace_size(op, B, N, D, K, dtype, chunk_rows)
+    if n == 0:
+        raise KMError(2, library().km_last_error().decode(errors="replace"))
+    return int(n)
+
+
+def _workspace(op, B, N, D, K, dtype, device, workspace=None, chunk_rows=0):
+    need = workspace_size(op, B, N, D, K, dtype, chunk_rows)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace has {workspace.numel()} bytes, needs {need}")
+    return workspace
+
+
+def _contig_cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def assign(X: torch.Tensor, C: torch.Tensor, *, idx=None, mindist=None, want_mindist: bool = True,
+           want_objective: bool = True, workspace=None, stream=None):
+    """FlashAssign: nearest centroid of every point (lowest index on ties).
+
+    X: (N, D) or (B, N, D) bf16/f32 CUDA tensor; C: (K, D) or (B, K, D), same dtype.
+    Returns (idx int32, mindist float32 or None, objective float64 [B] or None).
+    """
+    _contig_cuda(X, "X"), _contig_cuda(C, "C")
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C, "C")
+    if Bc != B or Dc != D or C.dtype != X.dtype:
+        raise ValueError("C must match X in batch, D and dtype")
+    dt = _dtype_code(X)
+    shp = (B, N) if batched else (N,)
+    idx = torch.empty(shp, dtype=torch.int32, device=X.device) if idx is None else idx
+    if mindist is None and want_mindist:
+        mindist = torch.empty(shp, dtype=torch.float32, device=X.device)
+    obj = torch.empty(B, dtype=torch.float64, device=X.device) if want_objective else None
+    ws = _workspace(OP_ASSIGN, B, N, D, K, dt, X.device, workspace)
+    _check(library().km_assign(_ptr(X), _ptr(C), B, N, D, K, dt, _ptr(idx), _ptr(mindist), _ptr(obj),
+                               _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, mindist, obj
+
+
+def update(X: torch.Tensor, idx: torch.Tensor, C: torch.Tensor, *, counts=None, want_counts: bool = True,
+           workspace=None, stream=None):
+    """Sort-Inverse Update: C (float32, in: previous, out: new) <- member means.
+
+    Returns (C, counts int32 or None).  C is updated in place.
+    """
+    _contig_cuda(X, "X"), _contig_cuda(idx, "idx"), _contig_cuda(C, "C")
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C, "C")
+    if Bc != B or Dc != D or C.dtype != torch.float32 or idx.dtype != torch.int32:
+        raise ValueError("C must be float32 (B, K, D) matching X; idx int32")
+    dt = _dtype_code(X)
+    if counts is None and want_counts:
+        counts = torch.empty((B, K) if batched else (K,), dtype=torch.int32, device=X.device)
+    ws = _workspace(OP_UPDATE, B, N, D, K, dt, X.device, workspace)
+    _check(library().km_update(_ptr(X), _ptr(idx), B, N, D, K, dt, _ptr(C), _ptr(counts), _ptr(ws), ws.numel(),
+                               _stream(stream)))
+    return C, counts
+
+
+def argsort(idx: torch.Tensor, K: int, *, workspace=None, stream=None):
+    """Stable argsort of an assignment vector by cluster id on the device.
+
+    Returns (perm int32 [N], start int32 [K+1]).
+    """
+    _contig_cuda(idx, "idx")
+    if idx.dtype != torch.int32 or idx.dim() != 1:
+        raise ValueError("idx must be a 1-D int32 tensor")
+    N = idx.shape[0]
+    perm = torch.empty(N, dtype=torch.int32, device=idx.device)
+    start = torch.empty(K + 1, dtype=torch.int32, device=idx.device)
+    ws = _workspace(OP_ARGSORT, 1, N, 0, K, 0, idx.device, workspace)
+    _check(library().km_argsort(_ptr(idx), N, K, _ptr(perm), _ptr(start), _ptr(ws), ws.numel(), _stream(stream)))
+    return perm, start
+
+
+def fit(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_out=None, counts_out=None,
+        objective=None, want_idx: bool = True, workspace=None, stream=None):
+    """`iters` exact Lloyd iterations from C0 on the device.
+
+    Returns dict(C float32, idx int32 or None, counts int32, objective float64 [B, iters] or [iters]).
+    """
+    _contig_cuda(X, "X"), _contig_cuda(C0, "C0")
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C0, "C0")
+    if Bc != B or Dc != D or C0.dtype != X.dtype:
+        raise ValueError("C0 must match X in batch, D and dtype")
+    dt = _dtype_code(X)
+    dev = X.device
+    C_out = torch.empty((B, K, D) if batched else (K, D), dtype=torch.float32, device=dev) if C_out is None else C_out
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((B, N) if batched else (N,), dtype=torch.int32, device=dev)
+    counts_out = torch.empty((B, K) if batched else (K,), dtype=torch.int32, device=dev) \
+        if counts_out is None else counts_out
+    objective = torch.empty((B, iters) if batched else (iters,), dtype=torch.float64, device=dev) \
+        if objective is None else objective
+    ws = _workspace(OP_FIT, B, N, D, K, dt, dev, workspace)
+    _check(library().km_fit(_ptr(X), _ptr(C0), B, N, D, K, dt, iters, _ptr(C_out), _ptr(idx_out),
+                            _ptr(counts_out), _ptr(objective), _ptr(ws), ws.numel(), _stream(stream)))
+    return dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective)
+
+
+def fit_profile(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_out=None, counts_out=None,
+                objective=None, workspace=None, stream=None):
+    """fit() with CUDA-event timing of each iteration's assignment and update.
+
+    Synchronous.  Returns the fit() dict plus "phase_ms": float32 [iters, 2]
+    (assignment kernel ms, update ms) and "iters_ms": device time of the
+    iterations (first assignment start to last update end).
+    """
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C0, "C0")
+    dt = _dtype_code(X)
+    dev = X.device
+    C_out = torch.empty((B, K, D) if batched else (K, D), dtype=torch.float32, device=dev) if C_out is None else C_out
+    counts_out = torch.empty((B, K) if batched else (K,), dtype=torch.int32, device=dev) \
+        if counts_out is None else counts_out
+    objective = torch.empty((B, iters) if batched else (iters,), dtype=torch.float64, device=dev) \
+        if objective is None else objective
+    phase = torch.zeros(2 * iters + 1, dtype=torch.float32)
+    ws = _workspace(OP_FIT, B, N, D, K, dt, dev, workspace)
+    _check(library().km_fit_profile(_ptr(X), _ptr(C0), B, N, D, K, dt, iters, _ptr(C_out), _ptr(idx_out),
+                                    _ptr(counts_out), _ptr(objective), _ptr(ws), ws.numel(), _stream(stream),
+                                    _ptr(phase)))
+    return dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective,
+                phase_ms=phase[:2 * iters].reshape(iters, 2), iters_ms=float(phase[2 * iters]))
+
+
+def launch_count() -> int:
+    """Kernels this library has enqueued in this process so far."""
+    return int(library().km_launch_count())
+
+
+def fit_host(X_host: torch.Tensor, C0: torch.Tensor, iters: int, chunk_rows: int, *, C_out=None, idx_out=None,
+             want_idx: bool = False, counts_out=None, workspace=None, stream=None):
+    """Out-of-core Lloyd: X_host is a pinned CPU tensor (N, D), streamed per iteration in chunks.
+
+    Synchronous.  Returns dict(C, idx or None, counts, objective (CPU float64 [iters])).
+    """
+    if X_host.is_cuda or not X_host.is_pinned():
+        raise ValueError("X_host must be a pinned CPU tensor")
+    if not X_host.is_contiguous():
+        raise ValueError("X_host must be contiguous")
+    _contig_cuda(C0, "C0")
+    N, D = X_host.shape
+    K = C0.shape[0]
+    dt = _dtype_code(X_host)
+    dev = C0.device
+    C_out = torch.empty((K, D), dtype=torch.float32, device=dev) if C_out is None else C_out
+    if idx_out is None and want_idx:
+        idx_out = torch.empty(N, dtype=torch.int32, device=dev)
+    counts_out = torch.empty(K, dtype=torch.int32, device=dev) if counts_out is None else counts_out
+    obj = torch.empty(iters, dtype=torch.float64)
+    ws = _workspace(OP_FIT_HOST, 1, N, D, K, dt, dev, workspace, chunk_rows)
+    _check(library().km_fit_host(_ptr(X_host), _ptr(C0), N, D, K, dt, iters, chunk_rows, _ptr(C_out),
+                                 _ptr(idx_out), _ptr(counts_out), _ptr(obj), _ptr(ws), ws.numel(),
+                                 _stream(stream)))
+    return dict(C=C_out, idx=idx_out, counts=counts_out, objective=obj)
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and read/clear the workspace status word (0 or KM_ERR_TIMEOUT)."""
+    return int(library().km_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def selftest_timeout(limit_ns: int = 1_000_000, device="cuda") -> int:
+    """Run the bounded-wait self-test kernel; returns the status it reports."""
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    return int(library().km_selftest_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(None)))

@@ -1,0 +1,119 @@
+// k_prep.cu -- operand preparation for FlashAssign (Flash-KMeans §2.1 uses
+// precomputed squared norms: the distance is ||x||^2 - 2 x.c + ||c||^2, and
+// only the cross term needs the tensor cores).
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "km_internal.h"
+#include "km_rows.cuh"
+
+namespace km {
+
+// One warp per point row: ||x||^2 in float32 and, in f32 mode, the TF32 split
+// operand [hi | hi | lo] (paired with the centroid split [hi | lo | hi] the
+// dot product becomes hi*hi + hi*lo + lo*hi).
+__global__ void k_xprep(const void* __restrict__ X, int dtype, int64_t rows, int D, int Dp,
+                        float* __restrict__ xn, float* __restrict__ x3) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= rows) return;
+  float s = 0.f;
+  if (dtype == kDtypeBF16) {
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(X) + r * D;
+    for (int j = lane; j < D; j += 32) {
+      float f = __bfloat162float(x[j]);
+      s = fmaf(f, f, s);
+    }
+  } else {
+    const float* x = reinterpret_cast<const float*>(X) + r * D;
+    float* o = x3 ? x3 + r * (3 * Dp) : nullptr;
+    for (int j = lane; j < Dp; j += 32) {
+      float v = j < D ? x[j] : 0.f;
+      s = fmaf(v, v, s);
+      if (o) {
+        float hi = tf32_round(v);
+        float lo = tf32_round(v - hi);
+        o[j] = hi;
+        o[Dp + j] = hi;
+        o[2 * Dp + j] = lo;
+      }
+    }
+  }
+  s = warp_sum_f(s);
+  if (lane == 0) xn[r] = s;
+}
+
+cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, float* xn, float* x3,
+                         cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (rows * 32 + threads - 1) / threads;
+  count_launch();
+  k_xprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(X, dtype, rows, D, Dp, xn, x3);
+  return cudaGetLastError();
+}
+
+// One warp per (instance, centroid row < Kp).
+__global__ void k_cprep(const void* __restrict__ src, int src_dtype, int B, int K, int Kp, int D, int Dp,
+                        int dtype, float* __restrict__ master, void* __restrict__ c_op, float* __restrict__ cn) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (g >= static_cast<int64_t>(B) * Kp) return;
+  const int b = static_cast<int>(g / Kp);
+  const int k = static_cast<int>(g - static_cast<int64_t>(b) * Kp);
+  if (k >= K) {
+    if (lane == 0) cn[g] = CUDART_INF_F;
+    return;
+  }
+  const int64_t row = static_cast<int64_t>(b) * K + k;
+  if (master) {
+    for (int j = lane; j < D; j += 32) master[row * D + j] = load_elem(src, src_dtype, row * D + j);
+  }
+  void* orow = nullptr;
+  if (c_op) {
+    orow = dtype == kDtypeBF16
+               ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(c_op) + row * D)
+               : static_cast<void*>(reinterpret_cast<float*>(c_op) + row * (3 * Dp));
+  }
+  float s = emit_operand_row([&](int j) { return load_elem(src, src_dtype, row * D + j); }, D, Dp, dtype, orow,
+                             lane);
+  if (lane == 0) cn[g] = s;
+}
+
+cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, int D, int Dp, int dtype,
+                         float* master, void* c_op, float* cn, cudaStream_t s) {
+  const int threads = 256;
+  const int64_t warps = static_cast<int64_t>(B) * Kp;
+  const int64_t blocks = (warps * 32 + threads - 1) / threads;
+  count_launch();
+  k_cprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(src, src_dtype, B, K, Kp, D, Dp, dtype, master, c_op,
+                                                           cn);
+  return cudaGetLastError();
+}
+
+// Objective per instance from the FlashAssign tile partials, in a fixed
+// order: each thread sums a strided subset sequentially, then a fixed tree.
+__global__ void k_objective(const double* __restrict__ tobj, int64_t per_inst, double* __restrict__ out,
+                            int out_stride) {
+  __shared__ double red[256];
+  const int b = blockIdx.x;
+  const double* p = tobj + static_cast<int64_t>(b) * per_inst;
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < per_inst; i += 256) s += p[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[static_cast<int64_t>(b) * out_stride] = red[0];
+}
+
+cudaError_t launch_objective(const double* tobj, int B, int64_t tiles_per_inst, double* out, int out_stride,
+                             cudaStream_t s) {
+  count_launch();
+  k_objective<<<B, 256, 0, s>>>(tobj, tiles_per_inst * 4, out, out_stride);
+  return cudaGetLastError();
+}
+
+}  // namespace km

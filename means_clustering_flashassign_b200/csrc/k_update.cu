@@ -1,0 +1,654 @@
+// k_update.cu -- segmented reduction of the Sort-Inverse Update ("Flash-KMeans:
+// Fast and Memory-Efficient Exact K-Means", §2.2 Sort-Inverse Update).
+//
+// After the argsort, points of one cluster occupy a contiguous run of sorted
+// positions.  Thread blocks take fixed chunks of sorted positions, gather the
+// point rows (one coalesced 16-byte load per lane) and sum each run in float32
+// registers.  Runs that lie inside one warp's range are final at once; a run
+// cut by a warp or block edge leaves a partial that is combined in the fixed
+// order of the cut positions.  The pages let thread blocks add their boundary
+// partials with atomics; here the combination is atomic-free and ordered, so
+// the result is bitwise reproducible, with the same O((K + N/B_N) d) boundary
+// writes (§2.2, "原子操作优化").
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "km_internal.h"
+#include "km_rows.cuh"
+
+namespace km {
+
+// --------------------------------------------------------- row gathering
+// Lanes are grouped: LPR lanes (16 bytes each) cover one point row; the
+// warp reads 32/LPR rows per step.
+template <int LPR>
+struct RowGeom {
+  static constexpr int RPS = 32 / LPR;                    // rows per step
+  static constexpr int STEPS = LPR < 16 ? LPR : 16;        // steps per batch
+  static constexpr int BATCH = STEPS * RPS;               // rows per batch (<= 32)
+};
+
+template <bool BF16>
+__device__ __forceinline__ void add16(float (&acc)[8], const uint4 v) {
+  if constexpr (BF16) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += __uint_as_float(w[i] << 16);
+      acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+    acc[0] += __uint_as_float(v.x);
+    acc[1] += __uint_as_float(v.y);
+    acc[2] += __uint_as_float(v.z);
+    acc[3] += __uint_as_float(v.w);
+  }
+}
+
+// Sum rows perm[lo..hi) into this lane's column chunk; every lane of the warp
+// must call it with the same lo/hi.  Afterwards lanes < LPR hold the column
+// sums of their 16-byte chunk (reduced across the row slots in a fixed order).
+template <int LPR, bool BF16>
+__device__ __forceinline__ void seg_rows_sum(const uint8_t* __restrict__ X, int row_bytes,
+                                             const int32_t* perm, int64_t lo, int64_t hi, int lane,
+                                             float (&acc)[8]) {
+  using G = RowGeom<LPR>;
+  const int sub = lane / LPR;
+  const int cl = lane % LPR;
+  const bool active = cl * 16 < row_bytes;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int64_t b0 = lo; b0 < hi; b0 += G::BATCH) {
+    const int myr = (lane < G::BATCH && b0 + lane < hi) ? perm[b0 + lane] : -1;
+    uint4 buf[G::STEPS];
+#pragma unroll
+    for (int s = 0; s < G::STEPS; ++s) {
+      const int r = __shfl_sync(0xffffffffu, myr, s * G::RPS + sub);
+      if (r >= 0 && active)
+        buf[s] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(r) * row_bytes + cl * 16));
+      else
+        buf[s] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int s = 0; s < G::STEPS; ++s) add16<BF16>(acc, buf[s]);
+  }
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+}
+
+// Store a lane's column sums (lanes < LPR) to dst[0..D) floats, scaled.
+template <int LPR, bool BF16>
+__device__ __forceinline__ void store_row(float* dst, int row_bytes, int lane, const float (&acc)[8], float scale) {
+  const int cl = lane;
+  if (lane >= LPR || cl * 16 >= row_bytes) return;
+  if constexpr (BF16) {
+    float4* d4 = reinterpret_cast<float4*>(dst + cl * 8);
+    d4[0] = make_float4(acc[0] * scale, acc[1] * scale, acc[2] * scale, acc[3] * scale);
+    d4[1] = make_float4(acc[4] * scale, acc[5] * scale, acc[6] * scale, acc[7] * scale);
+  } else {
+    reinterpret_cast<float4*>(dst + cl * 4)[0] =
+        make_float4(acc[0] * scale, acc[1] * scale, acc[2] * scale, acc[3] * scale);
+  }
+}
+
+__device__ __forceinline__ int find_cluster(const int32_t* start, int K, int64_t pos) {
+  int lo = 0, hi = K;  // start[lo] <= pos < start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (start[mid] <= pos) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// One warp sums the runs of sorted positions [q0, q1).  Runs inside the range
+// are written with `final_store(k, acc)`; a run crossing the left edge goes to
+// slot 0, one crossing only the right edge to slot 1 (cluster ids in slot_k,
+// -1 when unused, vectors in slot_v[2][D]).
+template <int LPR, bool BF16, class FinalStore>
+__device__ __forceinline__ void warp_range_sums(const uint8_t* X, int row_bytes, int D, const int32_t* perm,
+                                                const int32_t* start, int K, int64_t q0, int64_t q1, int lane,
+                                                int* slot_k, float* slot_v, FinalStore final_store) {
+  if (lane == 0) { slot_k[0] = -1; slot_k[1] = -1; }
+  if (q0 >= q1) return;
+  int k = find_cluster(start, K, q0);
+  int64_t pos = q0;
+  while (pos < q1) {
+    while (start[k + 1] <= pos) ++k;
+    const int64_t s0 = start[k], s1 = start[k + 1];
+    const int64_t hi = s1 < q1 ? s1 : q1;
+    float acc[8];
+    seg_rows_sum<LPR, BF16>(X, row_bytes, perm, pos, hi, lane, acc);
+    const bool cl = s0 < q0, cr = s1 > q1;
+    if (!cl && !cr) {
+      final_store(k, acc);
+    } else {
+      const int slot = cl ? 0 : 1;
+      store_row<LPR, BF16>(slot_v + slot * D, row_bytes, lane, acc, 1.f);
+      if (lane == 0) slot_k[slot] = k;
+    }
+    pos = hi;
+    ++k;
+  }
+}
+
+// ------------------------------------------------------------ big path
+template <int LPR, bool BF16>
+__global__ void __launch_bounds__(256) k_segsum(const uint8_t* __restrict__ X, int64_t n, int D, int row_bytes,
+                                                const int32_t* __restrict__ perm, const int32_t* __restrict__ start,
+                                                int K, int L, float* __restrict__ sums, float* __restrict__ pl,
+                                                float* __restrict__ pr) {
+  extern __shared__ float sm[];
+  constexpr int W = 8;
+  int* slot_k = reinterpret_cast<int*>(sm);          // [W][2]
+  float* slot_v = sm + 2 * W;                         // [W][2][D]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c = blockIdx.x;
+  const int64_t p0 = c * W * L;
+  const int64_t p1 = p0 + static_cast<int64_t>(W) * L < n ? p0 + static_cast<int64_t>(W) * L : n;
+  const int64_t q0 = p0 + static_cast<int64_t>(warp) * L;
+  const int64_t q1 = q0 + L < p1 ? q0 + L : p1;
+  warp_range_sums<LPR, BF16>(X, row_bytes, D, perm, start, K, q0, q1, lane, slot_k + 2 * warp,
+                             slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
+                               store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc, 1.f);
+                             });
+  __syncthreads();
+  // Ordered combine of the cut runs, one thread per column.
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+    int open = -1;
+    float a = 0.f;
+    auto flush = [&](int k, float v) {
+      const int64_t s0 = start[k], s1 = start[k + 1];
+      if (s0 >= p0 && s1 <= p1) sums[static_cast<int64_t>(k) * D + j] = v;
+      else if (s0 < p0) pl[c * D + j] = v;
+      else pr[c * D + j] = v;
+    };
+    for (int w = 0; w < W; ++w) {
+      for (int sl = 0; sl < 2; ++sl) {
+        const int k = slot_k[2 * w + sl];
+        if (k < 0) continue;
+        const float v = slot_v[(2 * w + sl) * D + j];
+        if (k == open) {
+          a += v;
+        } else {
+          if (open >= 0) flush(open, a);
+          open = k;
+          a = v;
+        }
+      }
+    }
+    if (open >= 0) flush(open, a);
+  }
+}
+
+template <int LPR>
+static cudaError_t launch_segsum_t(const Plan& p, const SegArgs& a, cudaStream_t s) {
+  const int row_bytes = p.D * p.es;
+  const int64_t nch = (a.n + p.gc.BNS - 1) / p.gc.BNS;
+  const size_t sm = (2 * 8 + 2 * 8 * static_cast<size_t>(p.D)) * 4;
+  count_launch();
+  if (p.dtype == kDtypeBF16)
+    k_segsum<LPR, true><<<static_cast<unsigned>(nch), 256, sm, s>>>(
+        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.start, p.K, p.gc.L, a.sums, a.pl, a.pr);
+  else
+    k_segsum<LPR, false><<<static_cast<unsigned>(nch), 256, sm, s>>>(
+        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.start, p.K, p.gc.L, a.sums, a.pl, a.pr);
+  return cudaGetLastError();
+}
+
+static int lanes_per_row(int row_bytes) {
+  int v = (row_bytes + 15) / 16, l = 1;
+  while (l < v) l <<= 1;
+  return l;
+}
+
+cudaError_t launch_segsum(const Plan& p, const SegArgs& a, cudaStream_t s) {
+  if (a.n <= 0) return cudaSuccess;
+  switch (lanes_per_row(p.D * p.es)) {
+    case 1: return launch_segsum_t<1>(p, a, s);
+    case 2: return launch_segsum_t<2>(p, a, s);
+    case 4: return launch_segsum_t<4>(p, a, s);
+    case 8: return launch_segsum_t<8>(p, a, s);
+    case 16: return launch_segsum_t<16>(p, a, s);
+    case 32: return launch_segsum_t<32>(p, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// --------------------------------------------------------------- finalize
+struct FinK {
+  int K, D, Dp, dtype, BNS, big_span;
+  int64_t n, nwarp_blocks;
+  const int32_t* start;
+  const float* sums;
+  const float* pl;
+  const float* pr;
+  int mode;
+  float* C;
+  void* c_op;
+  float* cn;
+  int32_t* counts;
+  double* acc64;
+  long long* cnt64;
+  const double* tobj;
+  int64_t ntiles;
+  double* obj;
+};
+
+__device__ __forceinline__ void* op_row(const FinK& f, int k) {
+  if (!f.c_op) return nullptr;
+  if (f.dtype == kDtypeBF16) return reinterpret_cast<__nv_bfloat16*>(f.c_op) + static_cast<int64_t>(k) * f.D;
+  return reinterpret_cast<float*>(f.c_op) + static_cast<int64_t>(k) * 3 * f.Dp;
+}
+
+// Finalise cluster k given its summed row in `srow` (shared or global), run
+// by one warp: centroid = sum / count (or keep), operand copy, norm, counts.
+__device__ void finish_cluster(const FinK& f, int k, int64_t cnt, const float* srow, int lane) {
+  float* crow = f.C + static_cast<int64_t>(k) * f.D;
+  if (f.mode == 0) {
+    if (cnt > 0) {
+      const float fc = static_cast<float>(cnt);
+      for (int j = lane; j < f.D; j += 32) crow[j] = srow[j] / fc;
+    }
+    __syncwarp();
+    const float s = emit_operand_row([&](int j) { return crow[j]; }, f.D, f.Dp, f.dtype, op_row(f, k), lane);
+    if (lane == 0) {
+      if (f.cn) f.cn[k] = s;
+      if (f.counts) f.counts[k] = static_cast<int32_t>(cnt);
+    }
+  } else if (cnt > 0) {
+    double* arow = f.acc64 + static_cast<int64_t>(k) * f.D;
+    for (int j = lane; j < f.D; j += 32) arow[j] += static_cast<double>(srow[j]);
+    if (lane == 0) f.cnt64[k] += cnt;
+  }
+}
+
+__global__ void __launch_bounds__(512) k_finalize(const FinK f) {
+  extern __shared__ float fsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && f.ntiles > 0) {
+    // objective of this pass: fixed-order reduction of the tile partials
+    double* red = reinterpret_cast<double*>(fsm);
+    double s = 0.0;
+    for (int64_t i = threadIdx.x; i < f.ntiles * 4; i += blockDim.x) s += f.tobj[i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      if (f.mode == 0) *f.obj = red[0];
+      else *f.obj += red[0];
+    }
+    __syncthreads();
+  }
+  if (blockIdx.x < f.nwarp_blocks) {
+    const int k = static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (k >= f.K) return;
+    const int64_t s0 = f.start[k], s1 = f.start[k + 1], cnt = s1 - s0;
+    if (cnt > 0) {
+      const int64_t ca = s0 / f.BNS, cb = (s1 - 1) / f.BNS;
+      if (cb - ca > f.big_span) return;  // handled by a whole block below
+      float* srow = fsm + (f.ntiles > 0 && blockIdx.x == 0 ? 1024 : 0) + warp * f.D;
+      if (ca == cb) {
+        for (int j = lane; j < f.D; j += 32) srow[j] = f.sums[static_cast<int64_t>(k) * f.D + j];
+      } else {
+        for (int j = lane; j < f.D; j += 32) {
+          float a = f.pr[ca * f.D + j];
+          for (int64_t c = ca + 1; c <= cb; ++c) a += f.pl[c * f.D + j];
+          srow[j] = a;
+        }
+      }
+      __syncwarp();
+      finish_cluster(f, k, cnt, srow, lane);
+    } else {
+      finish_cluster(f, k, 0, nullptr, lane);
+    }
+    return;
+  }
+  // Big clusters: block i owns the cluster containing position i*G (G =
+  // big_span*BNS) if that is the first multiple of G inside the cluster.
+  const int64_t G = static_cast<int64_t>(f.big_span) * f.BNS;
+  const int64_t P = (static_cast<int64_t>(blockIdx.x) - f.nwarp_blocks) * G;
+  if (P >= f.n) return;
+  const int k = find_cluster(f.start, f.K, P);
+  const int64_t s0 = f.start[k], s1 = f.start[k + 1];
+  const int64_t ca = s0 / f.BNS, cb = (s1 - 1) / f.BNS;
+  if (cb - ca <= f.big_span) return;
+  if ((s0 + G - 1) / G != P / G) return;
+  // column groups of 4 floats x slices of the chunk range
+  const int groups = f.D / 4;
+  const int slices = blockDim.x / groups;
+  const int tg = threadIdx.x % groups, sl = threadIdx.x / groups;
+  float* part = fsm;                       // [slices][D]
+  float* srow = fsm + slices * f.D;        // [D]
+  if (sl < slices) {
+    const int64_t nc = cb - ca + 1;
+    const int64_t per = (nc + slices - 1) / slices;
+    const int64_t c0 = ca + sl * per;
+    const int64_t c1 = c0 + per - 1 < cb ? c0 + per - 1 : cb;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t c = c0; c <= c1; ++c) {
+      const float* src = (c == ca ? f.pr : f.pl) + c * f.D + tg * 4;
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    }
+    reinterpret_cast<float4*>(part + sl * f.D)[tg] = a;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < f.D; j += blockDim.x) {
+    float a = 0.f;
+    for (int s2 = 0; s2 < slices; ++s2) a += part[s2 * f.D + j];
+    srow[j] = a;
+  }
+  __syncthreads();
+  if (warp == 0) finish_cluster(f, k, s1 - s0, srow, lane);
+}
+
+cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s) {
+  FinK f{};
+  f.K = p.K;
+  f.D = p.D;
+  f.Dp = p.Dp;
+  f.dtype = p.dtype;
+  f.BNS = p.gc.BNS;
+  f.big_span = p.gc.big_span;
+  f.n = p.rows;
+  f.start = a.start;
+  f.sums = a.sums;
+  f.pl = a.pl;
+  f.pr = a.pr;
+  f.mode = a.mode;
+  f.C = a.C;
+  f.c_op = a.c_op;
+  f.cn = a.cn;
+  f.counts = a.counts;
+  f.acc64 = a.acc64;
+  f.cnt64 = a.cnt64;
+  f.tobj = a.tobj;
+  f.ntiles = a.ntiles;
+  f.obj = a.obj;
+  const int threads = 512;
+  f.nwarp_blocks = (p.K + 15) / 16;
+  const int64_t G = static_cast<int64_t>(p.gc.big_span) * p.gc.BNS;
+  const int64_t nbig = (p.rows + G - 1) / G;
+  // block 0: 512 doubles of objective reduction (1024 floats) + 16 warp rows;
+  // big-cluster blocks: slices x D partial rows + one summed row.
+  const size_t fl_warp = 1024 + 16 * static_cast<size_t>(p.D);
+  const size_t fl_big = 2048 + 2 * static_cast<size_t>(p.D);
+  const size_t sm = 4 * (fl_warp > fl_big ? fl_warp : fl_big);
+  cudaError_t e = cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sm));
+  if (e != cudaSuccess) return e;
+  count_launch();
+  k_finalize<<<static_cast<unsigned>(f.nwarp_blocks + nbig), threads, sm, s>>>(f);
+  return cudaGetLastError();
+}
+
+// Out-of-core: float64 accumulators -> centroids; resets the accumulators.
+__global__ void k_finalize_acc(int K, int D, int Dp, int dtype, double* acc64, long long* cnt64, float* C,
+                               void* c_op, float* cn, int32_t* counts, double* objacc, double* obj_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (obj_out) *obj_out = *objacc;
+    *objacc = 0.0;
+  }
+  if (k >= K) return;
+  const long long cnt = cnt64[k];
+  float* crow = C + static_cast<int64_t>(k) * D;
+  double* arow = acc64 + static_cast<int64_t>(k) * D;
+  if (cnt > 0)
+    for (int j = lane; j < D; j += 32) crow[j] = static_cast<float>(arow[j] / static_cast<double>(cnt));
+  for (int j = lane; j < D; j += 32) arow[j] = 0.0;
+  __syncwarp();
+  void* orow = nullptr;
+  if (c_op)
+    orow = dtype == kDtypeBF16 ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(c_op) + static_cast<int64_t>(k) * D)
+                               : static_cast<void*>(reinterpret_cast<float*>(c_op) + static_cast<int64_t>(k) * 3 * Dp);
+  const float s = emit_operand_row([&](int j) { return crow[j]; }, D, Dp, dtype, orow, lane);
+  if (lane == 0) {
+    if (cn) cn[k] = s;
+    if (counts) counts[k] = static_cast<int32_t>(cnt);
+    cnt64[k] = 0;
+  }
+}
+
+cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, float* cn,
+                                int32_t* counts, double* objacc, double* obj_out, cudaStream_t s) {
+  const int threads = 256;
+  const int blocks = (p.K + 7) / 8;
+  count_launch();
+  k_finalize_acc<<<blocks, threads, 0, s>>>(p.K, p.D, p.Dp, p.dtype, acc64, cnt64, C, c_op, cn, counts, objacc,
+                                            obj_out);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------- fused small-problem path
+// One CTA per instance: stable counting sort of its assignment vector in
+// shared memory, segmented sums over the sorted order, ordered combine of
+// warp-boundary runs, centroids, operand copy, norms, counts and objective.
+struct SmallK {
+  int B, K, Kp, D, Dp, dtype;
+  int64_t N;
+  int row_bytes;
+  const uint8_t* X;
+  const int32_t* idx;
+  float* C;
+  void* c_op;
+  float* cn;
+  int32_t* counts;
+  const double* tobj;
+  int64_t tiles_per_inst;
+  double* obj;
+  int obj_stride;
+};
+
+__device__ __forceinline__ uint32_t lanemask_lt_u() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+template <int LPR, bool BF16>
+__global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
+  extern __shared__ __align__(16) int32_t ssm[];
+  constexpr int W = 8;
+  const int N = static_cast<int>(p.N), K = p.K, D = p.D;
+  // 16-byte aligned pieces first: slot vectors, the double reduction buffer,
+  // then the integer arrays.
+  float* slot_v = reinterpret_cast<float*>(ssm);                      // [W][2][D]
+  double* red = reinterpret_cast<double*>(slot_v + 2 * W * D);        // [256]
+  int32_t* keys = reinterpret_cast<int32_t*>(red + 256);              // [N]
+  int32_t* lrank = keys + N;           // [N]
+  int32_t* perm = lrank + N;           // [N]
+  int32_t* wcnt = perm + N;            // [W][K]
+  int32_t* start = wcnt + W * K;       // [K+1]
+  int32_t* tmp = start + K + 1;        // [256]
+  int* slot_k = tmp + 256;             // [W][2]
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* gidx = p.idx + static_cast<int64_t>(b) * N;
+  const uint8_t* X = p.X + static_cast<int64_t>(b) * N * p.row_bytes;
+  float* C = p.C + static_cast<int64_t>(b) * K * D;
+
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const int32_t v = gidx[i];  // ids outside [0, K) are clamped (memory safety only)
+    keys[i] = v < 0 ? 0 : (v >= K ? K - 1 : v);
+  }
+  for (int i = threadIdx.x; i < W * K; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  // stable ranks inside each warp's contiguous range
+  const int Lw = ((N + W - 1) / W + 31) / 32 * 32;
+  const uint32_t ltm = lanemask_lt_u();
+  for (int i0 = warp * Lw; i0 < (warp + 1) * Lw && i0 < N; i0 += 32) {
+    const int i = i0 + lane;
+    const bool v = i < N && i < (warp + 1) * Lw;
+    const int d = v ? keys[i] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    int before = 0;
+    if (v) before = wcnt[warp * K + d];
+    if (v) lrank[i] = before + __popc(peers & ltm);
+    __syncwarp();
+    if (v && lane == __ffs(peers) - 1) wcnt[warp * K + d] = before + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per-cluster warp prefixes, then cluster starts
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < W; ++w) {
+      const int c = wcnt[w * K + k];
+      wcnt[w * K + k] = run;
+      run += c;
+    }
+    start[k] = run;  // total, scanned below
+  }
+  __syncthreads();
+  {
+    const int per = (K + 255) / 256;
+    const int lo = threadIdx.x * per;
+    int s = 0;
+    for (int i = lo; i < lo + per && i < K; ++i) s += start[i];
+    tmp[threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int run = 0;
+      for (int i = 0; i < 256; ++i) { const int v = tmp[i]; tmp[i] = run; run += v; }
+    }
+    __syncthreads();
+    int run = tmp[threadIdx.x];
+    for (int i = lo; i < lo + per && i < K; ++i) { const int v = start[i]; start[i] = run; run += v; }
+    if (threadIdx.x == 0) start[K] = N;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const int w = i / Lw;
+    perm[start[keys[i]] + wcnt[w * K + keys[i]] + lrank[i]] = i;
+  }
+  __syncthreads();
+  // segmented sums: runs inside a warp range become centroids directly
+  const int L = (N + W - 1) / W;
+  const int q0 = warp * L < N ? warp * L : N;
+  const int q1 = q0 + L < N ? q0 + L : N;
+  warp_range_sums<LPR, BF16>(X, p.row_bytes, D, perm, start, K, q0, q1, lane, slot_k + 2 * warp,
+                             slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
+                               const float cntf = static_cast<float>(start[k + 1] - start[k]);
+                               // divide (not multiply by a reciprocal) to match sum / count
+                               float q[8];
+#pragma unroll
+                               for (int i = 0; i < 8; ++i) q[i] = acc[i] / cntf;
+                               store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q, 1.f);
+                             });
+  __syncthreads();
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+    int open = -1;
+    float a = 0.f;
+    auto flush = [&](int k, float v) {
+      C[static_cast<int64_t>(k) * D + j] = v / static_cast<float>(start[k + 1] - start[k]);
+    };
+    for (int w = 0; w < W; ++w)
+      for (int sl = 0; sl < 2; ++sl) {
+        const int k = slot_k[2 * w + sl];
+        if (k < 0) continue;
+        const float v = slot_v[(2 * w + sl) * D + j];
+        if (k == open) {
+          a += v;
+        } else {
+          if (open >= 0) flush(open, a);
+          open = k;
+          a = v;
+        }
+      }
+    if (open >= 0) flush(open, a);
+  }
+  __syncthreads();
+  // operand copies, norms and counts for every cluster (empty ones keep C)
+  for (int k = warp; k < K; k += W) {
+    float* crow = C + static_cast<int64_t>(k) * D;
+    const int64_t grow = static_cast<int64_t>(b) * K + k;
+    void* orow = nullptr;
+    if (p.c_op)
+      orow = p.dtype == kDtypeBF16
+                 ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(p.c_op) + grow * D)
+                 : static_cast<void*>(reinterpret_cast<float*>(p.c_op) + grow * 3 * p.Dp);
+    const float s = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, orow, lane);
+    if (lane == 0) {
+      if (p.cn) p.cn[static_cast<int64_t>(b) * p.Kp + k] = s;
+      if (p.counts) p.counts[grow] = start[k + 1] - start[k];
+    }
+  }
+  if (p.tobj && p.obj) {
+    const double* t = p.tobj + static_cast<int64_t>(b) * p.tiles_per_inst * 4;
+    double s = 0.0;
+    for (int64_t i = threadIdx.x; i < p.tiles_per_inst * 4; i += blockDim.x) s += t[i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) p.obj[static_cast<int64_t>(b) * p.obj_stride] = red[0];
+  }
+}
+
+size_t small_update_smem(int64_t N, int K, int D) {
+  const int W = 8;
+  size_t ints = 3 * static_cast<size_t>(N) + static_cast<size_t>(W) * K + K + 1 + 256 + 2 * W;
+  size_t floats = 2 * static_cast<size_t>(W) * D + 1;
+  return (ints + floats) * 4 + 16 + 256 * 8;
+}
+
+template <int LPR>
+static cudaError_t launch_small_t(const Plan& p, const SmallUpdateArgs& a, cudaStream_t s) {
+  SmallK k{};
+  k.B = p.B;
+  k.K = p.K;
+  k.Kp = p.Kp;
+  k.D = p.D;
+  k.Dp = p.Dp;
+  k.dtype = p.dtype;
+  k.N = p.N;
+  k.row_bytes = p.D * p.es;
+  k.X = static_cast<const uint8_t*>(a.X);
+  k.idx = a.idx;
+  k.C = a.C;
+  k.c_op = a.c_op;
+  k.cn = a.cn;
+  k.counts = a.counts;
+  k.tobj = a.tobj;
+  k.tiles_per_inst = a.tiles_per_inst;
+  k.obj = a.obj;
+  k.obj_stride = a.obj_stride;
+  const size_t sm = small_update_smem(p.N, p.K, p.D);
+  count_launch();
+  cudaError_t e;
+  if (p.dtype == kDtypeBF16) {
+    e = cudaFuncSetAttribute(k_small_update<LPR, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sm));
+    if (e != cudaSuccess) return e;
+    k_small_update<LPR, true><<<p.B, 256, sm, s>>>(k);
+  } else {
+    e = cudaFuncSetAttribute(k_small_update<LPR, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sm));
+    if (e != cudaSuccess) return e;
+    k_small_update<LPR, false><<<p.B, 256, sm, s>>>(k);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_small_update(const Plan& p, const SmallUpdateArgs& a, cudaStream_t s) {
+  switch (lanes_per_row(p.D * p.es)) {
+    case 1: return launch_small_t<1>(p, a, s);
+    case 2: return launch_small_t<2>(p, a, s);
+    case 4: return launch_small_t<4>(p, a, s);
+    case 8: return launch_small_t<8>(p, a, s);
+    case 16: return launch_small_t<16>(p, a, s);
+    case 32: return launch_small_t<32>(p, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace km

@@ -1,0 +1,665 @@
+// km_api.cu -- the C ABI of libkm.so (declared in include/km.h): argument
+// validation, the shape plan, workspace carving, TMA descriptors and the
+// launch sequences of FlashAssign, the Sort-Inverse Update, full Lloyd fits
+// and the out-of-core chunk stream ("Flash-KMeans: Fast and Memory-Efficient
+// Exact K-Means", §2.1-§2.3).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/km.h"
+#include "km_internal.h"
+
+namespace km {
+size_t assign_smem_for(int BN, int natoms, int XB, int CS);
+size_t small_update_smem(int64_t N, int K, int D);
+}  // namespace km
+
+using namespace km;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define KM_CUDA(call)                                                                        \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess)                                                                   \
+      return fail(KM_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kMaxHostIters = 1 << 16;
+constexpr int kSmemLimit = 232448;  // 227 KB per block on sm_100
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = getenv("KM_WAIT_LIMIT_NS");
+    uint64_t d = 2000000000ull;
+    if (e && *e) d = strtoull(e, nullptr, 10);
+    return d;
+  }();
+  return v;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D tensor map over [B][rows][inner] with a (epa x box_rows x 1) box and
+// the 128-byte swizzle; out-of-range rows/columns read as zero.
+int encode_map(CUtensorMap* m, const void* ptr, bool f32, int64_t inner, int64_t rows, int B, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return fail(KM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * es), static_cast<cuuint64_t>(inner * es * rows)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return KM_OK;
+}
+
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  KM_CUDA(cudaGetDevice(&dev));
+  KM_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  KM_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0)
+    return fail(KM_ERR_UNSUPPORTED, "device is sm_%d%d; this library is built for sm_100a only", major, minor);
+  return KM_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int ceil_log2(int k) {
+  int b = 0;
+  while ((1 << b) < k) ++b;
+  return b;
+}
+
+}  // namespace
+
+namespace km {
+
+int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, const char** why) {
+  static thread_local char msg[256];
+  auto bad = [&](int code, const char* fmt, auto... a) {
+    snprintf(msg, sizeof(msg), fmt, a...);
+    *why = msg;
+    return code;
+  };
+  if (op < KM_OP_ASSIGN || op > KM_OP_ARGSORT) return bad(KM_ERR_INVALID_ARG, "unknown op %d", op);
+  if (op == KM_OP_ARGSORT) {  // shape-independent of D and dtype
+    D = 8;
+    dtype = KM_BF16;
+    B = 1;
+  }
+  if (dtype != KM_F32 && dtype != KM_BF16) return bad(KM_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (B < 1 || N < 1 || K < 1) return bad(KM_ERR_INVALID_ARG, "need B >= 1, N >= 1, K >= 1 (B=%d N=%lld K=%d)", B,
+                                          static_cast<long long>(N), K);
+  if (K > N) return bad(KM_ERR_INVALID_ARG, "K=%d exceeds N=%lld", K, static_cast<long long>(N));
+  if (K > (1 << 20)) return bad(KM_ERR_UNSUPPORTED, "K=%d above 2^20", K);
+  if (N >= (int64_t(1) << 31)) return bad(KM_ERR_UNSUPPORTED, "N=%lld must be below 2^31", static_cast<long long>(N));
+  if (D % 8 != 0) return bad(KM_ERR_UNSUPPORTED, "D=%d must be a multiple of 8", D);
+  if (dtype == KM_BF16 && (D < 8 || D > 256)) return bad(KM_ERR_UNSUPPORTED, "bf16 needs 8 <= D <= 256 (D=%d)", D);
+  if (dtype == KM_F32 && (D < 8 || D > 64)) return bad(KM_ERR_UNSUPPORTED, "f32 needs 8 <= D <= 64 (D=%d)", D);
+  if (op == KM_OP_FIT_HOST && B != 1) return bad(KM_ERR_INVALID_ARG, "%s", "host-resident fits take one instance");
+  p = Plan{};
+  p.op = op;
+  p.B = B;
+  p.N = N;
+  p.D = D;
+  p.K = K;
+  p.dtype = dtype;
+  p.es = dtype == KM_BF16 ? 2 : 4;
+  p.Dp = (D + 31) / 32 * 32;
+  p.Dop = dtype == KM_BF16 ? D : 3 * p.Dp;
+  if (op == KM_OP_FIT_HOST) {
+    if (chunk_rows < 1) return bad(KM_ERR_INVALID_ARG, "%s", "chunk_rows must be >= 1");
+    p.chunk_rows = chunk_rows < N ? chunk_rows : N;
+    p.rows = p.chunk_rows;
+  } else {
+    p.rows = N;
+  }
+  // ---- FlashAssign tile configuration: widest centroid tile that fits
+  AssignCfg& ac = p.ac;
+  ac.epa = 128 / p.es;
+  ac.natoms = (p.Dop * p.es + 127) / 128;
+  int bn0 = K <= 64 ? 64 : (K <= 128 ? 128 : 256);
+  bool found = false;
+  for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
+    for (int xb = 2; xb >= 1 && !found; --xb) {
+      for (int cs = 4; cs >= 2 && !found; --cs) {
+        const size_t sm = assign_smem_for(bn, ac.natoms, xb, cs);
+        if (sm <= static_cast<size_t>(kSmemLimit)) {
+          ac.BN = bn;
+          ac.XB = xb;
+          ac.CS = cs;
+          ac.smem = sm;
+          found = true;
+        }
+      }
+    }
+  }
+  if (!found) return bad(KM_ERR_UNSUPPORTED, "no FlashAssign tiling fits shared memory for D=%d", D);
+  ac.tmem_cols = 2 * ac.BN;
+  p.Kp = (K + ac.BN - 1) / ac.BN * ac.BN;
+  p.tiles_per_inst = (p.rows + kTileM - 1) / kTileM;
+  p.ntiles = p.tiles_per_inst * B;
+  // ---- update configuration
+  p.small_update = B > 1 && N <= kSmallMaxN && K <= kSmallMaxK &&
+                   small_update_smem(N, K, D) <= static_cast<size_t>(kSmemLimit) && op != KM_OP_FIT_HOST;
+  SortCfg& sc = p.sc;
+  const int bits = ceil_log2(K) < 1 ? 1 : ceil_log2(K);
+  if (bits <= 12) {
+    sc.passes = 1;
+    sc.bits[0] = bits;
+  } else {
+    sc.passes = 2;
+    sc.bits[0] = bits / 2;
+    sc.bits[1] = bits - bits / 2;
+    sc.shift[1] = sc.bits[0];
+  }
+  sc.W = 8;
+  sc.IPT = 16;
+  sc.T = sc.W * 32 * sc.IPT;
+  sc.nblk = (p.rows + sc.T - 1) / sc.T;
+  sc.Rmax = 1 << (sc.bits[0] > sc.bits[1] ? sc.bits[0] : sc.bits[1]);
+  SegCfg& gc = p.gc;
+  gc.W = 8;
+  gc.L = p.rows >= int64_t(148) * 8 * 2048 ? 256 : 128;
+  gc.BNS = gc.W * gc.L;
+  gc.nchunks = (p.rows + gc.BNS - 1) / gc.BNS;
+  gc.big_span = 8;
+  // ---- workspace layout
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  const int64_t BR = static_cast<int64_t>(B) * p.rows;
+  p.off_hdr = take(kAlign);
+  if (op == KM_OP_ARGSORT) {
+    p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
+    p.off_total = take(sizeof(int32_t) * sc.Rmax);
+    if (sc.passes > 1) {
+      p.off_keys = take(sizeof(int32_t) * 2 * p.rows);
+      p.off_vals = take(sizeof(int32_t) * p.rows);
+    }
+    p.off_start = take(sizeof(int32_t) * (K + 1));
+    p.total = off;
+    return KM_OK;
+  }
+  p.off_xn = take(sizeof(float) * BR);
+  p.off_cn = take(sizeof(float) * static_cast<size_t>(B) * p.Kp);
+  if (op != KM_OP_ASSIGN || dtype == KM_F32)
+    p.off_clp = take(static_cast<size_t>(B) * K * p.Dop * (dtype == KM_BF16 ? 2 : 4));
+  if (dtype == KM_F32) p.off_x3 = take(sizeof(float) * BR * 3 * p.Dp);
+  p.off_tobj = take(sizeof(double) * 4 * static_cast<size_t>(p.ntiles));
+  if (op == KM_OP_FIT || op == KM_OP_FIT_HOST) p.off_idx = take(sizeof(int32_t) * BR);
+  p.off_obj = take(sizeof(double) * (op == KM_OP_FIT_HOST ? kMaxHostIters : B));
+  if (op != KM_OP_ASSIGN && !p.small_update) {
+    p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
+    p.off_total = take(sizeof(int32_t) * sc.Rmax);
+    if (sc.passes > 1) {
+      p.off_keys = take(sizeof(int32_t) * 2 * p.rows);
+      p.off_vals = take(sizeof(int32_t) * p.rows);
+    }
+    p.off_perm = take(sizeof(int32_t) * p.rows);
+    p.off_start = take(sizeof(int32_t) * (K + 1));
+    p.off_sums = take(sizeof(float) * static_cast<size_t>(K) * D);
+    p.off_pl = take(sizeof(float) * gc.nchunks * D);
+    p.off_pr = take(sizeof(float) * gc.nchunks * D);
+  }
+  if (op == KM_OP_FIT_HOST) {
+    p.off_dbuf0 = take(static_cast<size_t>(p.chunk_rows) * D * p.es);
+    p.off_dbuf1 = take(static_cast<size_t>(p.chunk_rows) * D * p.es);
+    p.off_acc64 = take(sizeof(double) * static_cast<size_t>(K) * D);
+    p.off_cnt64 = take(sizeof(long long) * K);
+    p.off_objacc = take(sizeof(double));
+  }
+  p.total = off;
+  return KM_OK;
+}
+
+}  // namespace km
+
+namespace {
+
+struct Ctx {
+  Plan p;
+  void* ws;
+  cudaStream_t s;
+  unsigned int* status() const { return at<unsigned int>(ws, p.off_hdr); }
+};
+
+int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, void* ws,
+            size_t ws_bytes, void* stream) {
+  const char* why = "";
+  int r = make_plan(c.p, op, B, N, D, K, dtype, chunk_rows, &why);
+  if (r != KM_OK) return fail(r, "%s", why);
+  if (!ws) return fail(KM_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(KM_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < c.p.total)
+    return fail(KM_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, c.p.total);
+  r = check_device();
+  if (r != KM_OK) return r;
+  c.ws = ws;
+  c.s = static_cast<cudaStream_t>(stream);
+  return KM_OK;
+}
+
+// Update of one instance through the multi-kernel path.
+int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, float* cnb,
+                    int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode) {
+  const Plan& p = c.p;
+  SortArgs sa{idxb,
+              n,
+              p.K,
+              at<int32_t>(c.ws, p.off_blkhist),
+              at<int32_t>(c.ws, p.off_total),
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
+              at<int32_t>(c.ws, p.off_perm),
+              at<int32_t>(c.ws, p.off_start)};
+  KM_CUDA(launch_sort(p, sa, c.s));
+  SegArgs ga{Xb, n, sa.perm, sa.start, at<float>(c.ws, p.off_sums), at<float>(c.ws, p.off_pl),
+             at<float>(c.ws, p.off_pr)};
+  KM_CUDA(launch_segsum(p, ga, c.s));
+  FinalizeArgs fa{};
+  fa.start = sa.start;
+  fa.sums = ga.sums;
+  fa.pl = ga.pl;
+  fa.pr = ga.pr;
+  fa.mode = mode;
+  fa.C = Cb;
+  fa.c_op = c_opb;
+  fa.cn = cnb;
+  fa.counts = countsb;
+  fa.acc64 = mode == 1 ? at<double>(c.ws, p.off_acc64) : nullptr;
+  fa.cnt64 = mode == 1 ? at<long long>(c.ws, p.off_cnt64) : nullptr;
+  fa.tobj = tobjb;
+  fa.ntiles = obj ? ntiles : 0;
+  fa.obj = obj;
+  Plan pp = p;
+  pp.rows = n;
+  KM_CUDA(launch_finalize(pp, fa, c.s));
+  return KM_OK;
+}
+
+size_t op_row_bytes(const Plan& p) { return static_cast<size_t>(p.Dop) * (p.dtype == KM_BF16 ? 2 : 4); }
+
+}  // namespace
+
+extern "C" {
+
+int km_version(void) { return KM_VERSION; }
+
+uint64_t km_launch_count(void) { return km::launch_counter().load(std::memory_order_relaxed); }
+
+const char* km_status_string(int status) {
+  switch (status) {
+    case KM_OK: return "ok";
+    case KM_ERR_INVALID_ARG: return "invalid argument";
+    case KM_ERR_UNSUPPORTED: return "unsupported";
+    case KM_ERR_CUDA: return "cuda error";
+    case KM_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case KM_ERR_TIMEOUT: return "bounded in-kernel wait ran out";
+    default: return "unknown status";
+  }
+}
+
+const char* km_last_error(void) { return g_err.c_str(); }
+
+size_t km_workspace_size(int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows) {
+  Plan p;
+  const char* why = "";
+  if (make_plan(p, op, B, N, D, K, dtype, chunk_rows, &why) != KM_OK) {
+    g_err = why;
+    return 0;
+  }
+  return p.total;
+}
+
+int km_workspace_status(void* workspace, void* stream) {
+  if (!workspace) return fail(KM_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int v = 0;
+  KM_CUDA(cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s));
+  KM_CUDA(cudaStreamSynchronize(s));
+  KM_CUDA(cudaMemsetAsync(workspace, 0, sizeof(v), s));
+  KM_CUDA(cudaStreamSynchronize(s));
+  if (v) return fail(KM_ERR_TIMEOUT, "a kernel gave up on a bounded wait (status 0x%x)", v);
+  return KM_OK;
+}
+
+int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int dtype, int32_t* idx, float* mindist,
+              double* objective, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!X || !C || !idx) return fail(KM_ERR_INVALID_ARG, "X, C and idx are required");
+  if (!aligned16(X) || !aligned16(C)) return fail(KM_ERR_INVALID_ARG, "X and C must be 16-byte aligned");
+  Ctx c;
+  int r = prepare(c, KM_OP_ASSIGN, B, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  const Plan& p = c.p;
+  float* xn = at<float>(c.ws, p.off_xn);
+  float* cn = at<float>(c.ws, p.off_cn);
+  KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+  CUtensorMap xmap, cmap;
+  if (dtype == KM_BF16) {
+    KM_CUDA(launch_xprep(X, kDtypeBF16, static_cast<int64_t>(B) * N, D, p.Dp, xn, nullptr, c.s));
+    KM_CUDA(launch_cprep(C, kDtypeBF16, B, K, p.Kp, D, p.Dp, kDtypeBF16, nullptr, nullptr, cn, c.s));
+    if ((r = encode_map(&xmap, X, false, D, N, B, kTileM)) != KM_OK) return r;
+    if ((r = encode_map(&cmap, C, false, D, K, B, p.ac.BN)) != KM_OK) return r;
+  } else {
+    float* x3 = at<float>(c.ws, p.off_x3);
+    float* c3 = at<float>(c.ws, p.off_clp);
+    KM_CUDA(launch_xprep(X, kDtypeF32, static_cast<int64_t>(B) * N, D, p.Dp, xn, x3, c.s));
+    KM_CUDA(launch_cprep(C, kDtypeF32, B, K, p.Kp, D, p.Dp, kDtypeF32, nullptr, c3, cn, c.s));
+    if ((r = encode_map(&xmap, x3, true, p.Dop, N, B, kTileM)) != KM_OK) return r;
+    if ((r = encode_map(&cmap, c3, true, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
+  }
+  double* tobj = at<double>(c.ws, p.off_tobj);
+  AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, mindist, tobj, c.status(), wait_limit_ns()};
+  KM_CUDA(launch_assign(p, a, c.s));
+  if (objective) KM_CUDA(launch_objective(tobj, B, p.tiles_per_inst, objective, 1, c.s));
+  return KM_OK;
+}
+
+int km_update(const void* X, const int32_t* idx, int B, int64_t N, int D, int K, int dtype, float* C, int32_t* counts,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!X || !idx || !C) return fail(KM_ERR_INVALID_ARG, "X, idx and C are required");
+  if (!aligned16(X) || !aligned16(C)) return fail(KM_ERR_INVALID_ARG, "X and C must be 16-byte aligned");
+  Ctx c;
+  int r = prepare(c, KM_OP_UPDATE, B, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  const Plan& p = c.p;
+  if (p.small_update) {
+    SmallUpdateArgs a{X, idx, C, nullptr, nullptr, counts, nullptr, 0, nullptr, 0};
+    KM_CUDA(launch_small_update(p, a, c.s));
+    return KM_OK;
+  }
+  const size_t xstride = static_cast<size_t>(N) * D * p.es;
+  for (int b = 0; b < B; ++b) {
+    r = update_instance(c, static_cast<const uint8_t*>(X) + b * xstride, idx + static_cast<int64_t>(b) * N, N,
+                        C + static_cast<int64_t>(b) * K * D, nullptr, nullptr,
+                        counts ? counts + static_cast<int64_t>(b) * K : nullptr, nullptr, 0, nullptr, 0);
+    if (r != KM_OK) return r;
+  }
+  return KM_OK;
+}
+
+static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
+                    float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
+                    size_t workspace_bytes, void* stream, cudaEvent_t* ev) {
+  if (!X || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X, C0 and C_out are required");
+  if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  if (!aligned16(X) || !aligned16(C0) || !aligned16(C_out))
+    return fail(KM_ERR_INVALID_ARG, "X, C0 and C_out must be 16-byte aligned");
+  Ctx c;
+  int r = prepare(c, KM_OP_FIT, B, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  const Plan& p = c.p;
+  float* xn = at<float>(c.ws, p.off_xn);
+  float* cn = at<float>(c.ws, p.off_cn);
+  void* clp = at<void>(c.ws, p.off_clp);
+  double* tobj = at<double>(c.ws, p.off_tobj);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(c.ws, p.off_idx);
+  double* objs = at<double>(c.ws, p.off_obj);
+  KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+  CUtensorMap xmap, cmap;
+  if (dtype == KM_BF16) {
+    KM_CUDA(launch_xprep(X, kDtypeBF16, static_cast<int64_t>(B) * N, D, p.Dp, xn, nullptr, c.s));
+    if ((r = encode_map(&xmap, X, false, D, N, B, kTileM)) != KM_OK) return r;
+    if ((r = encode_map(&cmap, clp, false, D, K, B, p.ac.BN)) != KM_OK) return r;
+  } else {
+    float* x3 = at<float>(c.ws, p.off_x3);
+    KM_CUDA(launch_xprep(X, kDtypeF32, static_cast<int64_t>(B) * N, D, p.Dp, xn, x3, c.s));
+    if ((r = encode_map(&xmap, x3, true, p.Dop, N, B, kTileM)) != KM_OK) return r;
+    if ((r = encode_map(&cmap, clp, true, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
+  }
+  KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, cn, c.s));
+  const size_t xstride = static_cast<size_t>(N) * D * p.es;
+  const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
+  for (int t = 0; t < iters; ++t) {
+    AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, nullptr, tobj, c.status(), wait_limit_ns()};
+    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t], c.s));
+    KM_CUDA(launch_assign(p, a, c.s));
+    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
+    if (p.small_update) {
+      SmallUpdateArgs u{X,    idx,       C_out, clp, cn, counts_out, tobj, p.tiles_per_inst,
+                        objective_hist ? objective_hist + t : objs, objective_hist ? iters : 1};
+      KM_CUDA(launch_small_update(p, u, c.s));
+    } else {
+      for (int b = 0; b < B; ++b) {
+        double* ob = objective_hist ? objective_hist + static_cast<int64_t>(b) * iters + t : objs + b;
+        r = update_instance(c, static_cast<const uint8_t*>(X) + b * xstride, idx + static_cast<int64_t>(b) * N, N,
+                            C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
+                            cn + static_cast<int64_t>(b) * p.Kp,
+                            counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
+                            tobj + static_cast<int64_t>(b) * p.tiles_per_inst * 4, p.tiles_per_inst, ob, 0);
+        if (r != KM_OK) return r;
+      }
+    }
+    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 2], c.s));
+  }
+  return KM_OK;
+}
+
+int km_fit(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters, float* C_out,
+           int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace, size_t workspace_bytes,
+           void* stream) {
+  g_err.clear();
+  return fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
+                  workspace_bytes, stream, nullptr);
+}
+
+int km_fit_profile(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
+                   float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
+                   size_t workspace_bytes, void* stream, float* phase_ms) {
+  g_err.clear();
+  if (!phase_ms) return fail(KM_ERR_INVALID_ARG, "phase_ms is required");
+  if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  std::vector<cudaEvent_t> ev(3 * static_cast<size_t>(iters), nullptr);
+  auto destroy = [&]() {
+    for (auto e : ev)
+      if (e) cudaEventDestroy(e);
+  };
+  for (auto& e : ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      destroy();
+      return fail(KM_ERR_CUDA, "cudaEventCreate failed");
+    }
+  }
+  int r = fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
+                   workspace_bytes, stream, iters > 0 ? ev.data() : nullptr);
+  if (r == KM_OK && cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    r = fail(KM_ERR_CUDA, "stream synchronisation failed");
+  for (int t = 0; r == KM_OK && t < iters; ++t) {
+    if (cudaEventElapsedTime(&phase_ms[2 * t], ev[3 * t], ev[3 * t + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&phase_ms[2 * t + 1], ev[3 * t + 1], ev[3 * t + 2]) != cudaSuccess)
+      r = fail(KM_ERR_CUDA, "cudaEventElapsedTime failed");
+  }
+  if (r == KM_OK) {
+    phase_ms[2 * static_cast<size_t>(iters)] = 0.f;
+    if (iters > 0 && cudaEventElapsedTime(&phase_ms[2 * static_cast<size_t>(iters)], ev[0],
+                                          ev[3 * static_cast<size_t>(iters) - 1]) != cudaSuccess)
+      r = fail(KM_ERR_CUDA, "cudaEventElapsedTime failed");
+  }
+  destroy();
+  return r;
+}
+
+int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int dtype, int iters, int64_t chunk_rows,
+                float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!X_host || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X_host, C0 and C_out are required");
+  if (iters < 0 || iters > kMaxHostIters) return fail(KM_ERR_INVALID_ARG, "iters must be in [0, %lld]",
+                                                      static_cast<long long>(kMaxHostIters));
+  if (!aligned16(C0) || !aligned16(C_out)) return fail(KM_ERR_INVALID_ARG, "C0 and C_out must be 16-byte aligned");
+  Ctx c;
+  int r = prepare(c, KM_OP_FIT_HOST, 1, N, D, K, dtype, chunk_rows, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  const Plan& p = c.p;
+  cudaPointerAttributes pa;
+  KM_CUDA(cudaPointerGetAttributes(&pa, X_host));
+  if (pa.type != cudaMemoryTypeHost) return fail(KM_ERR_INVALID_ARG, "X_host must be page-locked host memory");
+  float* xn = at<float>(c.ws, p.off_xn);
+  float* cn = at<float>(c.ws, p.off_cn);
+  void* clp = at<void>(c.ws, p.off_clp);
+  double* tobj = at<double>(c.ws, p.off_tobj);
+  double* objs = at<double>(c.ws, p.off_obj);
+  void* dbuf[2] = {at<void>(c.ws, p.off_dbuf0), at<void>(c.ws, p.off_dbuf1)};
+  double* acc64 = at<double>(c.ws, p.off_acc64);
+  long long* cnt64 = at<long long>(c.ws, p.off_cnt64);
+  double* objacc = at<double>(c.ws, p.off_objacc);
+  float* x3 = dtype == KM_F32 ? at<float>(c.ws, p.off_x3) : nullptr;
+
+  cudaStream_t cs = nullptr;
+  cudaEvent_t ev_copied[2] = {nullptr, nullptr}, ev_free[2] = {nullptr, nullptr};
+  auto cleanup = [&]() {
+    for (int i = 0; i < 2; ++i) {
+      if (ev_copied[i]) cudaEventDestroy(ev_copied[i]);
+      if (ev_free[i]) cudaEventDestroy(ev_free[i]);
+    }
+    if (cs) cudaStreamDestroy(cs);
+  };
+  auto run = [&]() -> int {
+    KM_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      KM_CUDA(cudaEventCreateWithFlags(&ev_copied[i], cudaEventDisableTiming));
+      KM_CUDA(cudaEventCreateWithFlags(&ev_free[i], cudaEventDisableTiming));
+    }
+    KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+    KM_CUDA(cudaMemsetAsync(acc64, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
+    KM_CUDA(cudaMemsetAsync(cnt64, 0, sizeof(long long) * K, c.s));
+    KM_CUDA(cudaMemsetAsync(objacc, 0, sizeof(double), c.s));
+    KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, cn, c.s));
+    for (int i = 0; i < 2; ++i) KM_CUDA(cudaEventRecord(ev_free[i], c.s));
+    CUtensorMap cmap;
+    int rr = encode_map(&cmap, clp, dtype == KM_F32, p.Dop, K, 1, p.ac.BN);
+    if (rr != KM_OK) return rr;
+    const int64_t nch = (N + p.chunk_rows - 1) / p.chunk_rows;
+    const size_t rowb = static_cast<size_t>(D) * p.es;
+    int64_t g = 0;
+    for (int t = 0; t < iters; ++t) {
+      for (int64_t ch = 0; ch < nch; ++ch, ++g) {
+        const int bi = static_cast<int>(g & 1);
+        const int64_t r0 = ch * p.chunk_rows;
+        const int64_t nr = N - r0 < p.chunk_rows ? N - r0 : p.chunk_rows;
+        KM_CUDA(cudaStreamWaitEvent(cs, ev_free[bi], 0));
+        KM_CUDA(cudaMemcpyAsync(dbuf[bi], static_cast<const uint8_t*>(X_host) + r0 * rowb, nr * rowb,
+                                cudaMemcpyHostToDevice, cs));
+        KM_CUDA(cudaEventRecord(ev_copied[bi], cs));
+        KM_CUDA(cudaStreamWaitEvent(c.s, ev_copied[bi], 0));
+        CUtensorMap xmap;
+        KM_CUDA(launch_xprep(dbuf[bi], dtype, nr, D, p.Dp, xn, x3, c.s));
+        rr = dtype == KM_BF16 ? encode_map(&xmap, dbuf[bi], false, D, nr, 1, kTileM)
+                              : encode_map(&xmap, x3, true, p.Dop, nr, 1, kTileM);
+        if (rr != KM_OK) return rr;
+        int32_t* idxc = idx_out ? idx_out + r0 : at<int32_t>(c.ws, p.off_idx);
+        Plan pc = p;
+        pc.rows = nr;
+        pc.tiles_per_inst = (nr + kTileM - 1) / kTileM;
+        pc.ntiles = pc.tiles_per_inst;
+        AssignArgs a{&xmap, &cmap, 1, nr, K, p.Kp, xn, cn, idxc, nullptr, tobj, c.status(), wait_limit_ns()};
+        KM_CUDA(launch_assign(pc, a, c.s));
+        Ctx cc = c;
+        cc.p = pc;
+        rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, pc.tiles_per_inst,
+                             objacc, 1);
+        if (rr != KM_OK) return rr;
+        KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
+      }
+      KM_CUDA(launch_finalize_acc(p, acc64, cnt64, C_out, clp, cn, counts_out, objacc, objs + t, c.s));
+    }
+    KM_CUDA(cudaStreamSynchronize(c.s));
+    if (objective_hist && iters > 0)
+      KM_CUDA(cudaMemcpy(objective_hist, objs, sizeof(double) * iters, cudaMemcpyDeviceToHost));
+    return km_workspace_status(c.ws, c.s);
+  };
+  r = run();
+  if (r != KM_OK) cudaStreamSynchronize(c.s);
+  cleanup();
+  return r;
+}
+
+int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* start, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!idx || !perm) return fail(KM_ERR_INVALID_ARG, "idx and perm are required");
+  Ctx c;
+  int r = prepare(c, KM_OP_ARGSORT, 1, N, 8, K, KM_BF16, 0, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  const Plan& p = c.p;
+  SortArgs sa{idx,
+              N,
+              K,
+              at<int32_t>(c.ws, p.off_blkhist),
+              at<int32_t>(c.ws, p.off_total),
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
+              perm,
+              start ? start : at<int32_t>(c.ws, p.off_start)};
+  KM_CUDA(launch_sort(p, sa, c.s));
+  return KM_OK;
+}
+
+int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_ns, void* stream) {
+  g_err.clear();
+  if (!workspace || workspace_bytes < kAlign) return fail(KM_ERR_WORKSPACE, "need at least 256 bytes of workspace");
+  if (limit_ns < 1 || limit_ns > 1000000000) return fail(KM_ERR_INVALID_ARG, "limit_ns must be in [1, 1e9]");
+  int r = check_device();
+  if (r != KM_OK) return r;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  KM_CUDA(cudaMemsetAsync(workspace, 0, sizeof(unsigned int), s));
+  KM_CUDA(launch_timeout_probe(static_cast<unsigned int*>(workspace), static_cast<uint64_t>(limit_ns), s));
+  return km_workspace_status(workspace, s);
+}
+
+}  // extern "C"

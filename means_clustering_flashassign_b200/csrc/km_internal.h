@@ -1,0 +1,191 @@
+// km_internal.h -- host-side plan, workspace layout and kernel launchers
+// shared by the translation units of libkm.so.
+#pragma once
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace km {
+
+constexpr int kDtypeF32 = 0;
+constexpr int kDtypeBF16 = 1;
+
+// Rows of points per FlashAssign tile (UMMA M) and warps of that kernel.
+constexpr int kTileM = 128;
+constexpr int kAssignThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kCnStages = 4;         // ring of centroid-norm tiles
+
+// Largest problem the single-CTA fused update handles (batched path).
+constexpr int kSmallMaxN = 8192;
+constexpr int kSmallMaxK = 1024;
+
+// Process-wide count of kernels enqueued by this library (km_launch_count).
+inline std::atomic<uint64_t>& launch_counter() {
+  static std::atomic<uint64_t> c{0};
+  return c;
+}
+inline void count_launch(uint64_t n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
+
+struct AssignCfg {
+  int BN = 0;          // centroids per UMMA tile (N of the MMA), 64/128/256
+  int XB = 0;          // point-tile buffers (1 or 2)
+  int CS = 0;          // centroid-tile stages
+  int natoms = 0;      // 128-byte K-atoms per operand row
+  int epa = 0;         // elements per atom (64 bf16, 32 fp32)
+  size_t smem = 0;     // dynamic shared memory bytes
+  int tmem_cols = 0;   // 2 * BN
+};
+
+struct SortCfg {
+  int passes = 0;
+  int bits[2] = {0, 0};
+  int shift[2] = {0, 0};
+  int W = 8;         // warps per block
+  int IPT = 16;      // items per thread
+  int T = 0;         // keys per block
+  int64_t nblk = 0;  // blocks per pass
+  int Rmax = 0;      // largest radix
+};
+
+struct SegCfg {
+  int W = 8;          // warps per block
+  int L = 0;          // sorted positions per warp
+  int BNS = 0;        // sorted positions per block (W * L)
+  int64_t nchunks = 0;
+  int big_span = 8;   // clusters spanning more chunks than this use a whole block in finalize
+  int64_t nbig = 0;   // finalize blocks reserved for such clusters
+};
+
+struct Plan {
+  int op = 0, B = 1, D = 0, K = 0, dtype = 0;
+  int64_t N = 0;       // points per instance
+  int64_t rows = 0;    // points per device pass (N in core; chunk rows out of core)
+  int64_t chunk_rows = 0;
+  int es = 2;          // bytes per X element
+  int Dp = 0;          // fp32: D padded to 32
+  int Dop = 0;         // operand row length in elements (bf16: D, fp32: 3 * Dp)
+  int Kp = 0;          // K padded to a multiple of BN
+  int64_t tiles_per_inst = 0, ntiles = 0;
+  bool small_update = false;
+  AssignCfg ac;
+  SortCfg sc;
+  SegCfg gc;
+  // workspace offsets (bytes)
+  size_t off_hdr = 0, off_xn = 0, off_cn = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
+  size_t off_blkhist = 0, off_total = 0, off_keys = 0, off_vals = 0, off_perm = 0, off_start = 0;
+  size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
+  size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
+  size_t total = 0;
+};
+
+// Fills `p` for the request; returns 0 or a km_status code (message in *why).
+int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows,
+              const char** why);
+
+// ------------------------------------------------------------- launchers
+// Row norms ||x||^2 (float32) of `rows` points; in f32 mode also writes the
+// TF32 split operand x3 = [hi | hi | lo] (rows x 3*Dp floats).
+cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, float* xn, float* x3,
+                         cudaStream_t s);
+
+// Centroid operand preparation for B instances of K centroids:
+//   src (dtype src_dtype: bf16 or f32) -> optional float32 master copy,
+//   bf16 operand copy (bf16 mode) or TF32 split [hi | lo | hi] (f32 mode),
+//   and ||c||^2 of the values the MMA sees; rows K..Kp-1 get +inf norms.
+cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, int D, int Dp, int dtype,
+                         float* master, void* c_op, float* cn, cudaStream_t s);
+
+// FlashAssign over B instances of `rows` points (tcgen05 / TMEM / TMA).
+struct AssignArgs {
+  const CUtensorMap* xmap;  // host copies, passed by value to the kernel
+  const CUtensorMap* cmap;
+  int B;
+  int64_t rows;
+  int K, Kp;
+  const float* xn;
+  const float* cn;
+  int32_t* idx;
+  float* mindist;
+  double* tobj;  // [B * tiles_per_inst][4]
+  unsigned int* status;
+  uint64_t limit_ns;
+};
+cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s);
+
+// Objective of each instance from the assign tile partials (fixed order).
+cudaError_t launch_objective(const double* tobj, int B, int64_t tiles_per_inst, double* out, int out_stride,
+                             cudaStream_t s);
+
+// Stable LSD radix sort of one instance's assignment vector; writes perm and
+// start[K+1] (start[k] = first sorted position of cluster k).
+struct SortArgs {
+  const int32_t* keys;
+  int64_t n;
+  int K;
+  int32_t* blkhist;
+  int32_t* total;
+  int32_t* keys_tmp;
+  int32_t* vals_tmp;
+  int32_t* perm;
+  int32_t* start;
+};
+cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s);
+
+// Segmented sums over the sorted order + ordered boundary fix-up + centroid
+// finalisation for one instance.
+struct SegArgs {
+  const void* X;
+  int64_t n;
+  const int32_t* perm;
+  const int32_t* start;
+  float* sums;  // [K][D]
+  float* pl;    // [nchunks][D]
+  float* pr;    // [nchunks][D]
+};
+cudaError_t launch_segsum(const Plan& p, const SegArgs& a, cudaStream_t s);
+
+struct FinalizeArgs {
+  const int32_t* start;
+  const float* sums;
+  const float* pl;
+  const float* pr;
+  int mode;          // 0: write centroids; 1: accumulate into acc64/cnt64
+  float* C;          // [K][D] float master (in: previous, out: new)
+  void* c_op;        // operand copy for the next assign (bf16 or TF32 split)
+  float* cn;         // [Kp]
+  int32_t* counts;   // [K] or null
+  double* acc64;     // [K][D] (mode 1)
+  long long* cnt64;  // [K] (mode 1)
+  const double* tobj;
+  int64_t ntiles;    // tile partials to reduce into *obj (0: none)
+  double* obj;       // objective output (mode 0) or accumulator (mode 1)
+};
+cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s);
+
+// Final step of the out-of-core update: centroids from float64 accumulators.
+cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, float* cn,
+                                int32_t* counts, double* objacc, double* obj_out, cudaStream_t s);
+
+// Fused single-CTA-per-instance update (sort + segmented sums + finalise) for
+// B instances with N <= kSmallMaxN, K <= kSmallMaxK.
+struct SmallUpdateArgs {
+  const void* X;
+  const int32_t* idx;
+  float* C;
+  void* c_op;  // may be null
+  float* cn;   // may be null
+  int32_t* counts;
+  const double* tobj;  // may be null
+  int64_t tiles_per_inst;
+  double* obj;  // [B] with stride obj_stride, may be null
+  int obj_stride;
+};
+cudaError_t launch_small_update(const Plan& p, const SmallUpdateArgs& a, cudaStream_t s);
+
+// Test hook: one CTA waits on a barrier nothing arrives on.
+cudaError_t launch_timeout_probe(unsigned int* status, uint64_t limit_ns, cudaStream_t s);
+
+}  // namespace km

@@ -1,0 +1,96 @@
+"""C-ABI boundary checks that need no GPU: the library builds, loads and
+exports every function include/km.h declares; workspace sizing is linear in
+N and K*D (never N*K); invalid shapes are rejected before any launch."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import means_clustering_flashassign_b200 as km
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "km.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(km_[a-z_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_header_symbols():
+    L = km.library()
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in km.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", km.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (km_\w+)", out))
+    assert set(names) == exported, (set(names) ^ exported)
+    assert set(km.EXPORTS) == set(names)
+    assert L.km_version() == 1
+
+
+def test_status_strings():
+    L = km.library()
+    for code in range(6):
+        assert L.km_status_string(code)
+    assert L.km_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("op", [km.OP_ASSIGN, km.OP_UPDATE, km.OP_FIT])
+def test_workspace_is_linear_not_nk(op):
+    # doubling N at fixed K grows the workspace by at most ~2x; doubling K at
+    # fixed N grows it by O(K*D), not by N*K
+    a = km.workspace_size(op, 1, 1 << 20, 128, 1024, km.BF16)
+    b = km.workspace_size(op, 1, 1 << 21, 128, 1024, km.BF16)
+    c = km.workspace_size(op, 1, 1 << 20, 128, 4096, km.BF16)
+    assert b < 2.2 * a
+    assert c - a < 64 * (4096 - 1024) * 128 + (1 << 22)
+    # an N x K fp32 score matrix would be 4 GiB here
+    assert a < (1 << 20) * 1024 * 4 / 50
+
+
+def test_workspace_host_stream_scales_with_chunk():
+    w1 = km.workspace_size(km.OP_FIT_HOST, 1, 1 << 28, 128, 4096, km.BF16, 1 << 20)
+    w2 = km.workspace_size(km.OP_FIT_HOST, 1, 1 << 28, 128, 4096, km.BF16, 1 << 21)
+    # two chunk buffers of chunk_rows * D * 2 bytes dominate the growth
+    assert abs((w2 - w1) - 2 * (1 << 20) * 128 * 2) < 0.5 * 2 * (1 << 20) * 128 * 2
+
+
+@pytest.mark.parametrize("args", [
+    (km.OP_FIT, 1, 100, 128, 200, km.BF16),   # K > N
+    (km.OP_FIT, 1, 1000, 12, 10, km.BF16),    # D not a multiple of 8
+    (km.OP_FIT, 1, 1000, 512, 10, km.BF16),   # D too large
+    (km.OP_FIT, 1, 1000, 128, 10, km.F32),    # f32 D too large
+    (km.OP_FIT, 0, 1000, 64, 10, km.BF16),    # B < 1
+    (km.OP_FIT, 1, 1000, 64, 0, km.BF16),     # K < 1
+    (7, 1, 1000, 64, 10, km.BF16),            # unknown op
+    (km.OP_FIT, 1, 1000, 64, 10, 5),          # unknown dtype
+])
+def test_invalid_shapes_rejected(args):
+    L = km.library()
+    assert L.km_workspace_size(*args, 0) == 0
+    assert L.km_last_error()
+
+
+def test_calls_without_gpu_fail_cleanly():
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    L = km.library()
+    ws = (ctypes.c_uint8 * 4096)()
+    st = L.km_selftest_timeout(ctypes.cast(ws, ctypes.c_void_p), 4096, 1000, None)
+    assert st == 3  # KM_ERR_CUDA: no device
+    assert b"cuda" in L.km_last_error().lower() or b"device" in L.km_last_error().lower()
+
+
+def test_null_arguments_rejected_before_device_use():
+    L = km.library()
+    assert L.km_assign(None, None, 1, 100, 64, 10, 1, None, None, None, None, 0, None) == 1
+    assert L.km_update(None, None, 1, 100, 64, 10, 1, None, None, None, 0, None) == 1
+    assert L.km_fit(None, None, 1, 100, 64, 10, 1, 3, None, None, None, None, None, 0, None) == 1
+    assert L.km_argsort(None, 100, 10, None, None, None, 0, None) == 1
