@@ -309,7 +309,7 @@ def main():
     ap.add_argument("--workload", default="1m_k1024", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-sample", type=int, default=131072)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -51,7 +51,10 @@ def check_assignment(X, C, idx_gpu, mindist_gpu=None, kind="bf16", rows=None):
         err = np.abs(md - dg)
         lim = 1e-5 * (xn + cn[ig]) + 1e-6
         assert np.all(err <= lim), f"mindist off by {np.max(err - lim)} beyond the limit"
-    return dict(n_clear=int(clear.sum()), n=int(clear.size), d1=d1)
+    # objective bound: relative JTOL plus the fp32 cancellation floor of the
+    # expanded form, summed over points (it matters only when J is ~0)
+    jfloor = float((1e-6 * (xn + cn[ig])).sum())
+    return dict(n_clear=int(clear.sum()), n=int(clear.size), d1=d1, jfloor=jfloor)
 
 
 def centroid_rel_err(C_gpu, C_ref):

@@ -35,7 +35,7 @@ def test_assign_bf16(N, D, K):
     r = check_assignment(X, C, idx, md, "bf16")
     assert r["n_clear"] > 0.5 * r["n"]
     J = r["d1"].sum()
-    assert abs(obj.item() - J) <= JTOL * J + 1e-6
+    assert abs(obj.item() - J) <= JTOL * J + r["jfloor"]
 
 
 ASSIGN_F32 = [(16384, 32, 64), (3000, 64, 100), (1000, 8, 5), (1000, 40, 70), (257, 32, 257), (5000, 16, 300)]
@@ -49,7 +49,7 @@ def test_assign_f32_tf32_split(N, D, K):
     r = check_assignment(X, C, idx, md, "f32")
     assert r["n_clear"] > 0.9 * r["n"]
     J = r["d1"].sum()
-    assert abs(obj.item() - J) <= JTOL * J
+    assert abs(obj.item() - J) <= JTOL * J + r["jfloor"]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -80,7 +80,7 @@ def test_assign_batched_instances():
     torch.cuda.synchronize()
     for b in range(3):
         r = check_assignment(X[b], C[b], idx[b], md[b], "bf16")
-        assert abs(obj[b].item() - r["d1"].sum()) <= JTOL * r["d1"].sum()
+        assert abs(obj[b].item() - r["d1"].sum()) <= JTOL * r["d1"].sum() + r["jfloor"]
 
 
 @pytest.mark.parametrize("N,K,kind", [(100000, 1024, "uniform"), (50000, 16384, "zipf"), (7777, 5000, "uniform"),
@@ -104,16 +104,16 @@ def test_argsort_is_the_stable_inverse_map(N, K, kind):
     assert np.array_equal(start.cpu().numpy().astype(np.int64), ref_start)
 
 
-UPDATE_CASES = [(20000, 128, 100, "bf16", "equal"), (50000, 128, 1000, "bf16", "zipf"),
+UPDATE_CASES = [(20000, 128, 100, "bf16", "equal"), (50000, 128, 1000, "bf16", "zipf1.2"),
                 (16384, 32, 64, "f32", "equal"), (3001, 64, 300, "bf16", "equal"), (1000, 256, 10, "bf16", "equal"),
-                (9000, 8, 20, "f32", "equal"), (200000, 64, 16384, "bf16", "zipf")]
+                (9000, 8, 20, "f32", "equal"), (200000, 64, 16384, "bf16", "zipf1.2")]
 
 
 @pytest.mark.parametrize("N,D,K,dtype,weights", UPDATE_CASES)
 def test_update_matches_member_means(N, D, K, dtype, weights):
     X, _ = _mixture(N, D, K, dtype, seed=N, weights=weights)
     rng = np.random.default_rng(K)
-    if weights == "zipf":
+    if weights.startswith("zipf"):
         w = np.arange(1, K + 1) ** -1.2
         idx = rng.choice(K, N, p=w / w.sum()).astype(np.int32)
     else:
@@ -202,7 +202,7 @@ def test_fit_batched_matches_per_instance_oracle():
 
 
 def test_fit_is_bitwise_deterministic():
-    X, C0 = _mixture(200000, 128, 1024, "bf16", seed=2, weights="zipf")
+    X, C0 = _mixture(200000, 128, 1024, "bf16", seed=2, weights="zipf1.2")
     a = km.fit(X, C0, 3)
     b = km.fit(X, C0, 3)
     torch.cuda.synchronize()
