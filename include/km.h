@@ -213,6 +213,33 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
                 double* objective_hist, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * km_assign for callers that cannot allocate device memory.  Some callers
+ * own every byte of device memory: a host framework that serves memory only
+ * from its own pool and forbids side allocations, or a latency-critical loop
+ * that cannot afford cudaMalloc's synchronisation and cost.  They pass inputs
+ * and outputs as for km_assign, but no workspace: the scratch comes from one
+ * static device array of KM_ASSIGN_STATIC_SCRATCH_BYTES (16 MiB) inside
+ * libkm.so, which every GPU that loads the library holds until the process
+ * exits.  The paper has no counterpart to this entry point.
+ *   - Arguments and results are those of km_assign (same kernels).
+ *   - A shape whose km_assign workspace (km_workspace_size(KM_OP_ASSIGN, ...))
+ *     exceeds KM_ASSIGN_STATIC_SCRATCH_BYTES is refused with
+ *     KM_ERR_UNSUPPORTED before anything is launched (bf16 with D=128 and
+ *     K=1024 fits up to about 3.9 million points per call).
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, with the device current) and caches it;
+ *     make that first call before any stream capture.
+ *   - All calls on one device share the array and it keeps the last call's
+ *     contents; each call clears what must start at zero.  Calls that may
+ *     overlap on the GPU (different streams, other threads) race on it: order
+ *     them, or use km_assign with separate workspaces.
+ */
+#define KM_ASSIGN_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+int km_assign_static(const void* X, const void* C, int B, int64_t N, int D, int K, int dtype,
+                     int32_t* idx, float* mindist, double* objective, void* stream);
+
+/*
  * Test hook for the bounded-wait machinery: launches one CTA that waits on a
  * shared-memory barrier that nothing ever arrives on, with the given limit in
  * nanoseconds (at most 10^9).  The kernel gives up, sets the workspace status

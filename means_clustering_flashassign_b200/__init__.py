@@ -26,7 +26,7 @@ import torch
 from . import build as _build
 
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
-           "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -36,7 +36,7 @@ STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_E
           4: "KM_ERR_WORKSPACE", 5: "KM_ERR_TIMEOUT"}
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
-           "km_launch_count"]
+           "km_launch_count", "km_assign_static"]
 
 _lock = threading.Lock()
 _lib = None
@@ -80,6 +80,7 @@ def library() -> ctypes.CDLL:
             L.km_argsort.argtypes = [P, I64, I, P, P, P, SZ, P]
             L.km_fit_profile.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
             L.km_launch_count.restype = ctypes.c_uint64
+            L.km_assign_static.argtypes = [P, P, I, I64, I, I, I, P, P, P, P]
             for f in EXPORTS:
                 getattr(L, f).restype = getattr(L, f).restype or I
             _lib = L
@@ -163,6 +164,27 @@ def assign(X: torch.Tensor, C: torch.Tensor, *, idx=None, mindist=None, want_min
     ws = _workspace(OP_ASSIGN, B, N, D, K, dt, X.device, workspace)
     _check(library().km_assign(_ptr(X), _ptr(C), B, N, D, K, dt, _ptr(idx), _ptr(mindist), _ptr(obj),
                                _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, mindist, obj
+
+
+def assign_static(X: torch.Tensor, C: torch.Tensor, *, idx=None, mindist=None, want_mindist: bool = True,
+                  want_objective: bool = True, stream=None):
+    """assign() without a workspace: scratch comes from the library's fixed
+    16 MiB static device area (for callers that cannot allocate; shapes that
+    need more are refused).  Same results as assign()."""
+    _contig_cuda(X, "X"), _contig_cuda(C, "C")
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C, "C")
+    if Bc != B or Dc != D or C.dtype != X.dtype:
+        raise ValueError("C must match X in batch, D and dtype")
+    dt = _dtype_code(X)
+    shp = (B, N) if batched else (N,)
+    idx = torch.empty(shp, dtype=torch.int32, device=X.device) if idx is None else idx
+    if mindist is None and want_mindist:
+        mindist = torch.empty(shp, dtype=torch.float32, device=X.device)
+    obj = torch.empty(B, dtype=torch.float64, device=X.device) if want_objective else None
+    _check(library().km_assign_static(_ptr(X), _ptr(C), B, N, D, K, dt, _ptr(idx), _ptr(mindist), _ptr(obj),
+                                      _stream(stream)))
     return idx, mindist, obj
 
 

@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 OBJ_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkm.so")
-SOURCES = ["km_api.cu", "k_prep.cu", "k_assign.cu", "k_sort.cu", "k_update.cu"]
+SOURCES = ["km_api.cu", "k_prep.cu", "k_assign.cu", "k_sort.cu", "k_update.cu", "km_noalloc.cu"]
 HEADERS = ["km_internal.h", "km_ptx.cuh", "km_rows.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -123,6 +123,8 @@ int ceil_log2(int k) {
 
 namespace km {
 
+void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+
 int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, const char** why) {
   static thread_local char msg[256];
   auto bad = [&](int code, const char* fmt, auto... a) {

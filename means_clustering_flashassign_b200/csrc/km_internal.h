@@ -81,6 +81,9 @@ struct Plan {
   size_t total = 0;
 };
 
+// Sets the message km_last_error() returns on the calling thread.
+void set_last_error(const char* msg);
+
 // Fills `p` for the request; returns 0 or a km_status code (message in *why).
 int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows,
               const char** why);
