@@ -40,6 +40,7 @@ struct AssignK {
   int32_t* idx;
   float* mindist;
   double* tobj;
+  int obj_per_cta;  // 1: tobj[cta][4] sums over the CTA's tiles in order; 0: tobj[tile][4]
   unsigned int* status;
   uint64_t limit_ns;
 };
@@ -214,6 +215,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     int ab = 0, ns = 0;
     uint32_t aph = 0, nph = 0, mph = 0;
     bool ok = true;
+    double cta_obj = 0.0;
     for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
       const int b = static_cast<int>(t / p.tiles_per_inst);
       const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
@@ -288,10 +290,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         double ds = static_cast<double>(md);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-        if (lane == 0 && p.tobj) p.tobj[t * 4 + q] = ds;
+        if (p.obj_per_cta) cta_obj += ds;
+        else if (lane == 0 && p.tobj) p.tobj[t * 4 + q] = ds;
       }
       mph ^= 1u;
     }
+    if (h == 0 && p.obj_per_cta && lane == 0 && p.tobj) p.tobj[static_cast<int64_t>(blockIdx.x) * 4 + q] = cta_obj;
   }
 
   __syncthreads();
@@ -319,6 +323,7 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.idx = a.idx;
   k.mindist = a.mindist;
   k.tobj = a.tobj;
+  k.obj_per_cta = a.B == 1 ? 1 : 0;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN>(k.natoms, k.XB, k.CS);
@@ -329,6 +334,7 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = k.ntiles < nsm ? k.ntiles : nsm;
+  if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles_per_inst;
   if (grid <= 0) return cudaSuccess;
   count_launch();
   k_assign<BN, TF32><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.cmap, k);

@@ -43,9 +43,59 @@ __global__ void k_xprep(const void* __restrict__ X, int dtype, int64_t rows, int
   if (lane == 0) xn[r] = s;
 }
 
+// bf16 row norms with one 16-byte load per lane: LPR lanes cover a row (LPR a
+// power of two with LPR * 16 >= 2 * D), 32 / LPR rows per warp step.
+template <int LPR>
+__global__ void __launch_bounds__(256) k_xnorm_bf16(const uint8_t* __restrict__ X, int64_t rows, int row_bytes,
+                                                    float* __restrict__ xn) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, cl = lane % LPR;
+  constexpr int RPW = 32 / LPR;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  for (int64_t r0 = w0 * RPW; r0 < rows; r0 += warps * RPW) {
+    const int64_t r = r0 + sub;
+    float s = 0.f;
+    if (r < rows && cl * 16 < row_bytes) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + r * row_bytes + cl * 16));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+        s = fmaf(lo, lo, s);
+        s = fmaf(hi, hi, s);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (r < rows && cl == 0) xn[r] = s;
+  }
+}
+
 cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, float* xn, float* x3,
                          cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  if (dtype == kDtypeBF16) {
+    const int row_bytes = 2 * D;
+    int lpr = 1;
+    while (lpr * 16 < row_bytes) lpr <<= 1;
+    int dev = 0, nsm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t need = (rows * lpr + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(need < int64_t(nsm) * 8 ? need : int64_t(nsm) * 8);
+    const uint8_t* Xb = static_cast<const uint8_t*>(X);
+    count_launch();
+    switch (lpr) {
+      case 1: k_xnorm_bf16<1><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      case 2: k_xnorm_bf16<2><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      case 4: k_xnorm_bf16<4><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      case 8: k_xnorm_bf16<8><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      case 16: k_xnorm_bf16<16><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      default: k_xnorm_bf16<32><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+    }
+    return cudaGetLastError();
+  }
   const int threads = 256;
   const int64_t blocks = (rows * 32 + threads - 1) / threads;
   count_launch();
@@ -109,10 +159,10 @@ __global__ void k_objective(const double* __restrict__ tobj, int64_t per_inst, d
   if (threadIdx.x == 0) out[static_cast<int64_t>(b) * out_stride] = red[0];
 }
 
-cudaError_t launch_objective(const double* tobj, int B, int64_t tiles_per_inst, double* out, int out_stride,
+cudaError_t launch_objective(const double* tobj, int B, int64_t groups_per_inst, double* out, int out_stride,
                              cudaStream_t s) {
   count_launch();
-  k_objective<<<B, 256, 0, s>>>(tobj, tiles_per_inst * 4, out, out_stride);
+  k_objective<<<B, 256, 0, s>>>(tobj, groups_per_inst * 4, out, out_stride);
   return cudaGetLastError();
 }
 

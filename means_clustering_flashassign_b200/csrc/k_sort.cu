@@ -30,16 +30,21 @@ __device__ __forceinline__ int32_t clamp_key(int32_t k, int K) { return k < 0 ? 
 __global__ void k_sort_hist(const int32_t* __restrict__ keys, int64_t n, int T, int shift, int R,
                             int64_t nblk, int32_t* __restrict__ blkhist, int K) {
   extern __shared__ int32_t sh[];
+  constexpr int kPer = 16;  // keys per thread (T == blockDim.x * kPer)
   for (int d = threadIdx.x; d < R; d += blockDim.x) sh[d] = 0;
-  __syncthreads();
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
   const int lane = threadIdx.x & 31;
-  for (int64_t i0 = t0; i0 < t0 + T && i0 < n; i0 += blockDim.x) {
-    const int64_t i = i0 + threadIdx.x;
-    const bool v = i < n && i < t0 + T;
-    const int d = v ? ((clamp_key(keys[i], K) >> shift) & (R - 1)) : -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-    if (v && lane == __ffs(peers) - 1) atomicAdd(&sh[d], __popc(peers));
+  int dig[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {  // all loads first, then the counting
+    const int64_t i = t0 + static_cast<int64_t>(j) * blockDim.x + threadIdx.x;
+    dig[j] = (i < n && j * static_cast<int>(blockDim.x) < T) ? ((clamp_key(keys[i], K) >> shift) & (R - 1)) : -1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, dig[j]);
+    if (dig[j] >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh[dig[j]], __popc(peers));
   }
   __syncthreads();
   for (int d = threadIdx.x; d < R; d += blockDim.x) blkhist[static_cast<int64_t>(d) * nblk + blockIdx.x] = sh[d];
@@ -68,25 +73,36 @@ __global__ void k_sort_colscan(int32_t* __restrict__ blkhist, int R, int64_t nbl
   if (lane == 0) total[d] = carry;
 }
 
-// Block-wide exclusive scan of total[0..R) into base[0..R) (shared memory).
+// Block-wide exclusive scan of total[0..R) into base[0..R) (shared memory):
+// contiguous per-thread runs, a warp-shuffle scan of the run sums, then a
+// scan of the warp sums by warp 0.  tmp needs blockDim.x / 32 ints.
 __device__ void block_exclusive_scan(const int32_t* __restrict__ total, int R, int32_t* base, int32_t* tmp) {
   const int nt = blockDim.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nt >> 5;
   const int per = (R + nt - 1) / nt;
   const int lo = threadIdx.x * per;
   int32_t s = 0;
   for (int i = lo; i < lo + per && i < R; ++i) s += total[i];
-  tmp[threadIdx.x] = s;
+  int32_t x = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t run = 0;
-    for (int i = 0; i < nt; ++i) {
-      const int32_t v = tmp[i];
-      tmp[i] = run;
-      run += v;
+  if (warp == 0) {
+    int32_t w = lane < nw ? tmp[lane] : 0;
+    int32_t v = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
     }
+    if (lane < nw) tmp[lane] = v - w;
   }
   __syncthreads();
-  int32_t run = tmp[threadIdx.x];
+  int32_t run = tmp[warp] + x - s;
   for (int i = lo; i < lo + per && i < R; ++i) {
     base[i] = run;
     run += total[i];
@@ -103,7 +119,7 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int32_
   const int W = blockDim.x >> 5;
   int32_t* base = sh;               // [R]
   int32_t* wcnt = sh + R;           // [W][R]
-  int32_t* tmp = wcnt + W * R;      // [blockDim.x]
+  int32_t* tmp = wcnt + W * R;      // [blockDim.x / 32]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   block_exclusive_scan(total, R, base, tmp);
@@ -121,11 +137,15 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int32_
   int32_t key[IPT];
   const uint32_t ltm = lanemask_lt();
 #pragma unroll
+  for (int s = 0; s < IPT; ++s) {  // all loads first
+    const int64_t i = w0 + s * 32 + lane;
+    key[s] = i < n ? clamp_key(keys_in[i], K) : 0;
+    dig[s] = i < n ? ((key[s] >> shift) & (R - 1)) : -1;
+  }
+#pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int64_t i = w0 + s * 32 + lane;
     const bool v = i < n;
-    key[s] = v ? clamp_key(keys_in[i], K) : 0;
-    dig[s] = v ? ((key[s] >> shift) & (R - 1)) : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, dig[s]);
     int before = 0;
     if (v) before = wcnt[warp * R + dig[s]];
@@ -184,21 +204,10 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
                                                                 a.K);
     const int cw = 8;
     k_sort_colscan<<<(R + cw - 1) / cw, cw * 32, 0, s>>>(a.blkhist, R, nblk, a.total);
-    // pass 0 of two writes (keys_tmp[0..n), vals_tmp); the last pass writes
-    // perm, and for two passes also the sorted keys (keys_tmp[n..2n)) that
-    // the segment-bounds kernel reads.
-    int32_t* kout;
-    int32_t* vout;
-    if (!last) {
-      kout = a.keys_tmp;
-      vout = a.vals_tmp;
-    } else if (c.passes > 1) {
-      kout = a.keys_tmp + a.n;
-      vout = a.perm;
-    } else {
-      kout = nullptr;
-      vout = a.perm;
-    }
+    // pass 0 of two writes (keys_tmp, vals_tmp); the last pass writes perm
+    // and the sorted keys (the segment id of every sorted position).
+    int32_t* kout = last ? a.skeys : a.keys_tmp;
+    int32_t* vout = last ? a.perm : a.vals_tmp;
     const size_t sm = scatter_smem(R, c.W, threads);
     int32_t* st = (last && c.passes == 1) ? a.start : nullptr;
     cudaError_t e = cudaFuncSetAttribute(k_sort_scatter<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -212,7 +221,7 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
   if (c.passes > 1) {
     const int64_t cnt = a.n + 1;
     count_launch();
-    k_bounds<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(a.keys_tmp + a.n, a.n, a.K, a.start);
+    k_bounds<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(a.skeys, a.n, a.K, a.start);
   }
   return cudaGetLastError();
 }

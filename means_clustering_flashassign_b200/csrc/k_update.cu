@@ -133,52 +133,143 @@ __device__ __forceinline__ void warp_range_sums(const uint8_t* X, int row_bytes,
   }
 }
 
+// One warp sums the runs of sorted positions [q0, q1) using the sorted keys:
+// the cluster of every position is known, so run starts are found with a
+// warp ballot on key changes and the row ids / keys of the next batch are
+// prefetched while the current batch is summed.  Runs inside the range go to
+// `final_store(k, acc)`; a run continuing past the left edge goes to slot 0,
+// one continuing only past the right edge to slot 1 (cluster ids in slot_k,
+// -1 when unused, vectors in slot_v[2][D]).
+template <int LPR, bool BF16, class FinalStore>
+__device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D,
+                                                      const int32_t* __restrict__ perm,
+                                                      const int32_t* __restrict__ skeys, int64_t n, int64_t q0,
+                                                      int64_t q1, int lane, int* slot_k, float* slot_v,
+                                                      FinalStore final_store) {
+  using G = RowGeom<LPR>;
+  if (lane == 0) { slot_k[0] = -1; slot_k[1] = -1; }
+  if (q0 >= q1) return;
+  const int sub = lane / LPR;
+  const int cl = lane % LPR;
+  const bool active = cl * 16 < row_bytes;
+  const int kfirst = skeys[q0];
+  const bool left_cont = q0 > 0 && skeys[q0 - 1] == kfirst;
+  const int klast = skeys[q1 - 1];
+  const bool right_cont = q1 < n && skeys[q1] == klast;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  int open_k = kfirst;
+  bool open_left = left_cont;
+  auto flush = [&](bool right) {
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (!open_left && !right) {
+      final_store(open_k, acc);
+    } else {
+      const int slot = open_left ? 0 : 1;
+      store_row<LPR, BF16>(slot_v + slot * D, row_bytes, lane, acc, 1.f);
+      if (lane == 0) slot_k[slot] = open_k;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  };
+  const bool in_batch = lane < G::BATCH;
+  int pv = (in_batch && q0 + lane < q1) ? perm[q0 + lane] : -1;
+  int kv = (in_batch && q0 + lane < q1) ? skeys[q0 + lane] : -1;
+  for (int64_t p = q0; p < q1; p += G::BATCH) {
+    const int cur_p = pv, cur_k = kv;
+    const int64_t pn = p + G::BATCH;
+    pv = (in_batch && pn + lane < q1) ? perm[pn + lane] : -1;
+    kv = (in_batch && pn + lane < q1) ? skeys[pn + lane] : -1;
+    const int nb = q1 - p < G::BATCH ? static_cast<int>(q1 - p) : G::BATCH;
+    int prevk = __shfl_up_sync(0xffffffffu, cur_k, 1);
+    if (lane == 0) prevk = open_k;
+    const uint32_t starts = __ballot_sync(0xffffffffu, lane < nb && cur_k != prevk);
+    int a = 0;
+    while (a < nb) {
+      if ((starts >> a) & 1u) {
+        flush(false);
+        open_k = __shfl_sync(0xffffffffu, cur_k, a);
+        open_left = false;
+      }
+      const uint32_t later = a + 1 < 32 ? (starts >> (a + 1)) << (a + 1) : 0u;
+      const int e = later ? __ffs(later) - 1 : nb;
+      uint4 buf[G::STEPS];
+#pragma unroll
+      for (int s = 0; s < G::STEPS; ++s) {
+        const int slot = s * G::RPS + sub;
+        const int r = __shfl_sync(0xffffffffu, cur_p, slot);
+        if (slot >= a && slot < e && active)
+          buf[s] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(r) * row_bytes + cl * 16));
+        else
+          buf[s] = make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int s = 0; s < G::STEPS; ++s) add16<BF16>(acc, buf[s]);
+      a = e;
+    }
+  }
+  flush(right_cont);
+}
+
 // ------------------------------------------------------------ big path
+// Persistent blocks walk chunks of W*L sorted positions.  Per chunk: each
+// warp sums its L positions, then the block combines the runs cut at warp
+// edges in position order; runs inside the chunk become final sums, a run
+// continuing past the chunk's left edge goes to pl[chunk], one continuing
+// only past its right edge to pr[chunk].
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256) k_segsum(const uint8_t* __restrict__ X, int64_t n, int D, int row_bytes,
-                                                const int32_t* __restrict__ perm, const int32_t* __restrict__ start,
-                                                int K, int L, float* __restrict__ sums, float* __restrict__ pl,
+                                                const int32_t* __restrict__ perm, const int32_t* __restrict__ skeys,
+                                                const int32_t* __restrict__ start, int L, int64_t nchunks,
+                                                float* __restrict__ sums, float* __restrict__ pl,
                                                 float* __restrict__ pr) {
   extern __shared__ float sm[];
   constexpr int W = 8;
   int* slot_k = reinterpret_cast<int*>(sm);          // [W][2]
   float* slot_v = sm + 2 * W;                         // [W][2][D]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t c = blockIdx.x;
-  const int64_t p0 = c * W * L;
-  const int64_t p1 = p0 + static_cast<int64_t>(W) * L < n ? p0 + static_cast<int64_t>(W) * L : n;
-  const int64_t q0 = p0 + static_cast<int64_t>(warp) * L;
-  const int64_t q1 = q0 + L < p1 ? q0 + L : p1;
-  warp_range_sums<LPR, BF16>(X, row_bytes, D, perm, start, K, q0, q1, lane, slot_k + 2 * warp,
-                             slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
-                               store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc, 1.f);
-                             });
-  __syncthreads();
-  // Ordered combine of the cut runs, one thread per column.
-  for (int j = threadIdx.x; j < D; j += blockDim.x) {
-    int open = -1;
-    float a = 0.f;
-    auto flush = [&](int k, float v) {
-      const int64_t s0 = start[k], s1 = start[k + 1];
-      if (s0 >= p0 && s1 <= p1) sums[static_cast<int64_t>(k) * D + j] = v;
-      else if (s0 < p0) pl[c * D + j] = v;
-      else pr[c * D + j] = v;
-    };
-    for (int w = 0; w < W; ++w) {
-      for (int sl = 0; sl < 2; ++sl) {
-        const int k = slot_k[2 * w + sl];
-        if (k < 0) continue;
-        const float v = slot_v[(2 * w + sl) * D + j];
-        if (k == open) {
-          a += v;
-        } else {
-          if (open >= 0) flush(open, a);
-          open = k;
-          a = v;
+  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
+    const int64_t p0 = c * W * L;
+    const int64_t p1 = p0 + static_cast<int64_t>(W) * L < n ? p0 + static_cast<int64_t>(W) * L : n;
+    const int64_t q0 = p0 + static_cast<int64_t>(warp) * L < p1 ? p0 + static_cast<int64_t>(warp) * L : p1;
+    const int64_t q1 = q0 + L < p1 ? q0 + L : p1;
+    warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, perm, skeys, n, q0, q1, lane, slot_k + 2 * warp,
+                                     slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
+                                       store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane,
+                                                            acc, 1.f);
+                                     });
+    __syncthreads();
+    // Ordered combine of the cut runs, one thread per column.
+    for (int j = threadIdx.x; j < D; j += blockDim.x) {
+      int open = -1;
+      float a = 0.f;
+      auto flush = [&](int k, float v) {
+        const int64_t s0 = start[k], s1 = start[k + 1];
+        if (s0 >= p0 && s1 <= p1) sums[static_cast<int64_t>(k) * D + j] = v;
+        else if (s0 < p0) pl[c * D + j] = v;
+        else pr[c * D + j] = v;
+      };
+      for (int w = 0; w < W; ++w) {
+        for (int sl = 0; sl < 2; ++sl) {
+          const int k = slot_k[2 * w + sl];
+          if (k < 0) continue;
+          const float v = slot_v[(2 * w + sl) * D + j];
+          if (k == open) {
+            a += v;
+          } else {
+            if (open >= 0) flush(open, a);
+            open = k;
+            a = v;
+          }
         }
       }
+      if (open >= 0) flush(open, a);
     }
-    if (open >= 0) flush(open, a);
+    __syncthreads();
   }
 }
 
@@ -187,13 +278,23 @@ static cudaError_t launch_segsum_t(const Plan& p, const SegArgs& a, cudaStream_t
   const int row_bytes = p.D * p.es;
   const int64_t nch = (a.n + p.gc.BNS - 1) / p.gc.BNS;
   const size_t sm = (2 * 8 + 2 * 8 * static_cast<size_t>(p.D)) * 4;
+  int dev = 0, nsm = 0, occ = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   count_launch();
-  if (p.dtype == kDtypeBF16)
-    k_segsum<LPR, true><<<static_cast<unsigned>(nch), 256, sm, s>>>(
-        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.start, p.K, p.gc.L, a.sums, a.pl, a.pr);
-  else
-    k_segsum<LPR, false><<<static_cast<unsigned>(nch), 256, sm, s>>>(
-        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.start, p.K, p.gc.L, a.sums, a.pl, a.pr);
+  if (p.dtype == kDtypeBF16) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_segsum<LPR, true>, 256, sm);
+    const int64_t grid = nch < static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1) ? nch : static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1);
+    k_segsum<LPR, true><<<static_cast<unsigned>(grid), 256, sm, s>>>(
+        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.skeys, a.start, p.gc.L, nch, a.sums,
+        a.pl, a.pr);
+  } else {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_segsum<LPR, false>, 256, sm);
+    const int64_t grid = nch < static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1) ? nch : static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1);
+    k_segsum<LPR, false><<<static_cast<unsigned>(grid), 256, sm, s>>>(
+        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.skeys, a.start, p.gc.L, nch, a.sums,
+        a.pl, a.pr);
+  }
   return cudaGetLastError();
 }
 

@@ -228,10 +228,11 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
     if (sc.passes > 1) {
-      p.off_keys = take(sizeof(int32_t) * 2 * p.rows);
+      p.off_keys = take(sizeof(int32_t) * p.rows);
       p.off_vals = take(sizeof(int32_t) * p.rows);
     }
     p.off_start = take(sizeof(int32_t) * (K + 1));
+    p.off_skeys = take(sizeof(int32_t) * p.rows);
     p.total = off;
     return KM_OK;
   }
@@ -247,10 +248,11 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
     if (sc.passes > 1) {
-      p.off_keys = take(sizeof(int32_t) * 2 * p.rows);
+      p.off_keys = take(sizeof(int32_t) * p.rows);
       p.off_vals = take(sizeof(int32_t) * p.rows);
     }
     p.off_perm = take(sizeof(int32_t) * p.rows);
+    p.off_skeys = take(sizeof(int32_t) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));
     p.off_sums = take(sizeof(float) * static_cast<size_t>(K) * D);
     p.off_pl = take(sizeof(float) * gc.nchunks * D);
@@ -306,9 +308,10 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
               at<int32_t>(c.ws, p.off_perm),
-              at<int32_t>(c.ws, p.off_start)};
+              at<int32_t>(c.ws, p.off_start),
+              at<int32_t>(c.ws, p.off_skeys)};
   KM_CUDA(launch_sort(p, sa, c.s));
-  SegArgs ga{Xb, n, sa.perm, sa.start, at<float>(c.ws, p.off_sums), at<float>(c.ws, p.off_pl),
+  SegArgs ga{Xb, n, sa.perm, sa.start, sa.skeys, at<float>(c.ws, p.off_sums), at<float>(c.ws, p.off_pl),
              at<float>(c.ws, p.off_pr)};
   KM_CUDA(launch_segsum(p, ga, c.s));
   FinalizeArgs fa{};
@@ -405,9 +408,10 @@ int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int 
     if ((r = encode_map(&cmap, c3, true, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
   }
   double* tobj = at<double>(c.ws, p.off_tobj);
-  AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, mindist, tobj, c.status(), wait_limit_ns()};
+  int64_t groups = 0;
+  AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, mindist, tobj, c.status(), wait_limit_ns(), &groups};
   KM_CUDA(launch_assign(p, a, c.s));
-  if (objective) KM_CUDA(launch_objective(tobj, B, p.tiles_per_inst, objective, 1, c.s));
+  if (objective) KM_CUDA(launch_objective(tobj, B, groups, objective, 1, c.s));
   return KM_OK;
 }
 
@@ -468,7 +472,8 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
   for (int t = 0; t < iters; ++t) {
-    AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, nullptr, tobj, c.status(), wait_limit_ns()};
+    int64_t groups = 0;
+    AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, nullptr, tobj, c.status(), wait_limit_ns(), &groups};
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t], c.s));
     KM_CUDA(launch_assign(p, a, c.s));
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
@@ -483,7 +488,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
                             C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
                             cn + static_cast<int64_t>(b) * p.Kp,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
-                            tobj + static_cast<int64_t>(b) * p.tiles_per_inst * 4, p.tiles_per_inst, ob, 0);
+                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0);
         if (r != KM_OK) return r;
       }
     }
@@ -609,12 +614,13 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         pc.rows = nr;
         pc.tiles_per_inst = (nr + kTileM - 1) / kTileM;
         pc.ntiles = pc.tiles_per_inst;
-        AssignArgs a{&xmap, &cmap, 1, nr, K, p.Kp, xn, cn, idxc, nullptr, tobj, c.status(), wait_limit_ns()};
+        int64_t groups = 0;
+        AssignArgs a{&xmap, &cmap, 1, nr, K, p.Kp, xn, cn, idxc, nullptr, tobj, c.status(), wait_limit_ns(),
+                     &groups};
         KM_CUDA(launch_assign(pc, a, c.s));
         Ctx cc = c;
         cc.p = pc;
-        rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, pc.tiles_per_inst,
-                             objacc, 1);
+        rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
       }
@@ -647,7 +653,8 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
               perm,
-              start ? start : at<int32_t>(c.ws, p.off_start)};
+              start ? start : at<int32_t>(c.ws, p.off_start),
+              at<int32_t>(c.ws, p.off_skeys)};
   KM_CUDA(launch_sort(p, sa, c.s));
   return KM_OK;
 }

@@ -75,7 +75,7 @@ struct Plan {
   SegCfg gc;
   // workspace offsets (bytes)
   size_t off_hdr = 0, off_xn = 0, off_cn = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
-  size_t off_blkhist = 0, off_total = 0, off_keys = 0, off_vals = 0, off_perm = 0, off_start = 0;
+  size_t off_blkhist = 0, off_total = 0, off_keys = 0, off_vals = 0, off_perm = 0, off_start = 0, off_skeys = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
   size_t total = 0;
@@ -112,14 +112,16 @@ struct AssignArgs {
   const float* cn;
   int32_t* idx;
   float* mindist;
-  double* tobj;  // [B * tiles_per_inst][4]
+  double* tobj;  // B == 1: [assign CTAs][4]; else [B * tiles_per_inst][4]
   unsigned int* status;
   uint64_t limit_ns;
+  int64_t* obj_groups;  // host out (may be null): 4-double groups of partials per instance
 };
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s);
 
-// Objective of each instance from the assign tile partials (fixed order).
-cudaError_t launch_objective(const double* tobj, int B, int64_t tiles_per_inst, double* out, int out_stride,
+// Objective of each instance from the assign partials (fixed order);
+// groups_per_inst groups of 4 doubles per instance.
+cudaError_t launch_objective(const double* tobj, int B, int64_t groups_per_inst, double* out, int out_stride,
                              cudaStream_t s);
 
 // Stable LSD radix sort of one instance's assignment vector; writes perm and
@@ -134,6 +136,7 @@ struct SortArgs {
   int32_t* vals_tmp;
   int32_t* perm;
   int32_t* start;
+  int32_t* skeys;  // [n] sorted keys (cluster id of each sorted position)
 };
 cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s);
 
@@ -144,6 +147,7 @@ struct SegArgs {
   int64_t n;
   const int32_t* perm;
   const int32_t* start;
+  const int32_t* skeys;
   float* sums;  // [K][D]
   float* pl;    // [nchunks][D]
   float* pr;    // [nchunks][D]
