@@ -225,7 +225,7 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
  *   - A shape whose km_assign workspace (km_workspace_size(KM_OP_ASSIGN, ...))
  *     exceeds KM_ASSIGN_STATIC_SCRATCH_BYTES is refused with
  *     KM_ERR_UNSUPPORTED before anything is launched (bf16 with D=128 and
- *     K=1024 fits up to about 3.9 million points per call).
+ *     K=1024 fits up to about 500 thousand points per call).
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress, with the device current) and caches it;

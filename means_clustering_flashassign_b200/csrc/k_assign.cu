@@ -2,25 +2,35 @@
 // Memory-Efficient Exact K-Means", §2.1 FlashAssign).
 //
 // For a tile of 128 points the kernel streams every centroid tile through the
-// tensor cores and keeps, per point, the running minimum of
-//     score_k = ||c_k||^2 - 2 x.c_k
-// and its index (the §2.1 online argmin: each point carries its current best
-// distance and cluster id, each new tile's local minimum is merged into it).
-// The N x K scores live only in tensor memory; device memory sees X once, the
-// centroid tiles (from L2) and the N-long outputs, i.e. O(Nd + Kd) traffic
-// instead of O(NK) (§2.1, "效果").
+// tensor cores and keeps, per point, the running minimum distance and its
+// centroid index (the §2.1 online argmin: each point carries its current best
+// distance and cluster id; each new tile's local minimum is merged into it).
+// The N x K distances live only in tensor memory; device memory sees X once,
+// the centroid tiles (from L2) and the N-long outputs, i.e. O(Nd + Kd)
+// traffic instead of O(NK) (§2.1, "效果").
 //
-// Structure: persistent CTAs (one per SM) with warp-specialised roles
-//   warp 0      TMA producer: point tile (resident for the whole centroid
-//               sweep, double buffered across tiles), centroid tiles through a
-//               ring of stages (the §2.1 "异步预取" double-buffered prefetch),
-//               and the matching ||c||^2 slices through a separate ring;
-//   warp 1      tcgen05.mma issuer (one thread): M=128 x N=BN x K=16 (bf16)
-//               or K=8 (tf32) steps into a double-buffered TMEM accumulator;
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator, score = cn - 2*acc,
-//               per-lane argmin with the lowest index winning exact ties; two
-//               warps per TMEM lane quarter split the BN columns in halves and
-//               merge at the end of the point tile.
+// The tensor cores produce the whole distance, not just the cross term: the
+// operands carry one extra 32-byte K-slice (km_rows.cuh, "norm augmentation")
+// so that one UMMA chain accumulates
+//     ||x||^2 + ||c||^2 - 2 x.c        (centroid operand holds -2c)
+// and the epilogue is a pure argmin.  Per score it forms a key -- the float
+// bits with the 5 low mantissa bits replaced by the column inside its
+// 32-column chunk -- and reduces keys with 3-input float minimum; equal
+// distances therefore resolve to the lowest column, and a chunk's winner is
+// merged into the running best only on a strictly smaller distance, so the
+// lowest index wins exact ties.  (Distances closer than 2^-18 relative also
+// compare equal; that is far inside the parity rule's near-tie band.)
+//
+// Structure: persistent CTAs (one per SM), warp-specialised:
+//   warp 0       TMA producer: point tile + its augmentation (resident for the
+//                whole centroid sweep, double buffered across tiles), centroid
+//                tiles + augmentation through a ring of stages (the §2.1
+//                asynchronous double-buffered prefetch);
+//   warp 1       tcgen05.mma issuer (one thread): M=128 x N=BN x K=16 (bf16)
+//                or K=8 (tf32) steps into a double-buffered TMEM accumulator;
+//   warps 2..17  epilogue: 4 warps per TMEM lane quarter, each owning a
+//                quarter of the BN columns; tcgen05.ld, key, min tree; the
+//                four column quarters merge at the end of the point tile.
 // Every wait is an mbarrier wait bounded in time (see km_ptx.cuh).
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -35,72 +45,150 @@ struct AssignK {
   int64_t rows;
   int K, Kp, natoms, XB, CS, nct;
   int64_t tiles_per_inst, ntiles;
-  const float* xn;
-  const float* cn;
   int32_t* idx;
   float* mindist;
   double* tobj;
   int obj_per_cta;  // 1: tobj[cta][4] sums over the CTA's tiles in order; 0: tobj[tile][4]
+  uint32_t zero;    // always 0; keeps the epilogue's column constants in registers
   unsigned int* status;
   uint64_t limit_ns;
 };
 
 constexpr int kAtomBytesPerRow = 128;
 constexpr int kXAtomBytes = kTileM * kAtomBytesPerRow;  // 16 KB per point-tile atom
+constexpr int kAugRowBytes = 32;
+constexpr int kEpiWarps = 16;
+
+__host__ __device__ constexpr size_t x_buf_bytes(int natoms) {
+  return static_cast<size_t>(natoms) * kXAtomBytes + kTileM * kAugRowBytes;
+}
+__host__ __device__ constexpr size_t c_stage_bytes(int natoms, int BN) {
+  return static_cast<size_t>(natoms) * BN * kAtomBytesPerRow + static_cast<size_t>(BN) * kAugRowBytes;
+}
 
 template <int BN>
 __host__ __device__ constexpr size_t assign_smem_bytes(int natoms, int XB, int CS) {
-  return 1024 /* alignment slack */ + static_cast<size_t>(XB) * natoms * kXAtomBytes +
-         static_cast<size_t>(CS) * natoms * BN * kAtomBytesPerRow + kCnStages * BN * 4 + kTileM * 8 +
-         32 * 8 /* barriers */ + 16;
+  return 1024 /* alignment slack */ + XB * x_buf_bytes(natoms) + CS * c_stage_bytes(natoms, BN) +
+         3 * kTileM * 8 /* merge slots */ + 32 * 8 /* barriers */ + 16;
+}
+
+// Shared-memory descriptor for the 32-byte augmentation slice (K-major,
+// 32-byte swizzle: rows of 32 bytes, 8-row groups 256 bytes apart).
+__device__ __forceinline__ uint64_t sw32_kmajor_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(256u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(6u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Load CW (16 or 32) consecutive TMEM columns of this thread's lane and wait.
+template <int CW>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CW]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
+  tmem_ld32(taddr, v);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Minimum key of CW scores: key = score bits with the low 5 bits replaced by
+// the column index in [0, CW) (held in registers: ci[i] == i, mask == ~31),
+// so each key is one three-input bitwise operation.  Reduced with 3-input
+// minima.
+template <int CW>
+__device__ __forceinline__ uint32_t chunk_min_key(const float (&v)[CW], const uint32_t (&ci)[CW], uint32_t mask) {
+  float k[CW];
+#pragma unroll
+  for (int i = 0; i < CW; ++i) k[i] = __uint_as_float((__float_as_uint(v[i]) & mask) | ci[i]);
+  constexpr int L1 = CW / 3 + (CW % 3);  // CW=32: 10 triples + 2 singles; CW=16: 5 triples + 1 single
+  float a[L1];
+#pragma unroll
+  for (int i = 0; i < CW / 3; ++i) a[i] = fmin3(k[3 * i], k[3 * i + 1], k[3 * i + 2]);
+#pragma unroll
+  for (int i = 0; i < CW % 3; ++i) a[CW / 3 + i] = k[3 * (CW / 3) + i];
+  constexpr int L2 = L1 / 3 + (L1 % 3);
+  float b[L2];
+#pragma unroll
+  for (int i = 0; i < L1 / 3; ++i) b[i] = fmin3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+#pragma unroll
+  for (int i = 0; i < L1 % 3; ++i) b[L1 / 3 + i] = a[3 * (L1 / 3) + i];
+  float m = b[0];
+  int i = 1;
+#pragma unroll
+  for (; i + 1 < L2; i += 2) m = fmin3(m, b[i], b[i + 1]);
+  if (i < L2) m = fminf(m, b[i]);
+  return __float_as_uint(m);
 }
 
 template <int BN, bool TF32>
 __global__ void __launch_bounds__(kAssignThreads, 1)
-    k_assign(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, const AssignK p) {
+    k_assign(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap xamap,
+             const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap camap, const AssignK p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int natoms = p.natoms;
   const int XB = p.XB, CS = p.CS;
+  const size_t xbb = x_buf_bytes(natoms), csb = c_stage_bytes(natoms, BN);
   uint8_t* xs = base;
-  uint8_t* cs = xs + static_cast<size_t>(XB) * natoms * kXAtomBytes;
-  float* cns = reinterpret_cast<float*>(cs + static_cast<size_t>(CS) * natoms * BN * kAtomBytesPerRow);
-  float* mval = cns + kCnStages * BN;
-  int* midx = reinterpret_cast<int*>(mval + kTileM);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(midx + kTileM);
+  uint8_t* cs = xs + XB * xbb;
+  float* mval = reinterpret_cast<float*>(cs + CS * csb);  // [3][128]
+  int* midx = reinterpret_cast<int*>(mval + 3 * kTileM);  // [3][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(midx + 3 * kTileM);
   uint64_t* x_full = bars + 0;    // [2]
   uint64_t* x_empty = bars + 2;   // [2]
   uint64_t* c_full = bars + 4;    // [4]
   uint64_t* c_empty = bars + 8;   // [4]
-  uint64_t* n_full = bars + 12;   // [4]
-  uint64_t* n_empty = bars + 16;  // [4]
-  uint64_t* a_full = bars + 20;   // [2]
-  uint64_t* a_empty = bars + 22;  // [2]
-  uint64_t* m_full = bars + 24;
-  uint64_t* m_empty = bars + 25;
-  uint64_t* drain = bars + 26;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 32);
+  uint64_t* a_full = bars + 12;   // [2]
+  uint64_t* a_empty = bars + 14;  // [2]
+  uint64_t* m_full = bars + 16;
+  uint64_t* m_empty = bars + 17;
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr uint32_t kTmemCols = 2 * BN;
-  constexpr int kHalf = BN / 2;
+  constexpr int kQ = BN / 4;                 // columns per epilogue warp per tile
+  constexpr int CW = kQ < 32 ? kQ : 32;      // columns per TMEM load
+  constexpr int kChunks = kQ / CW;
+  constexpr int kElem = TF32 ? 32 : 64;      // elements per 128-byte atom row
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 8);
+      mbar_init(&a_empty[i], kEpiWarps);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&c_full[i], 1);
       mbar_init(&c_empty[i], 1);
-      mbar_init(&n_full[i], 1);
-      mbar_init(&n_empty[i], 8);
     }
-    mbar_init(m_full, kTileM);
+    mbar_init(m_full, 3 * kTileM);
     mbar_init(m_empty, kTileM);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -122,35 +210,35 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       prefetch_tensormap(&xmap);
+      prefetch_tensormap(&xamap);
       prefetch_tensormap(&cmap);
-      int xb = 0, cst = 0, ns = 0;
-      uint32_t xph = 0, cph = 0, nph = 0;
-      int x_iss[2] = {-1, -1}, c_iss[4] = {-1, -1, -1, -1}, n_iss[4] = {-1, -1, -1, -1};
+      prefetch_tensormap(&camap);
+      int xb = 0, cst = 0;
+      uint32_t xph = 0, cph = 0;
+      int x_iss[2] = {-1, -1}, c_iss[4] = {-1, -1, -1, -1};
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
         const int b = static_cast<int>(t / p.tiles_per_inst);
         const int rt = static_cast<int>(t - static_cast<int64_t>(b) * p.tiles_per_inst);
         if (!mbar_wait(&x_empty[xb], xph ^ 1u, g)) { ok = false; break; }
-        mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(natoms) * kXAtomBytes);
+        uint8_t* xdst = xs + xb * xbb;
+        mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(xbb));
         for (int a = 0; a < natoms; ++a)
-          tma_load_3d(xs + (static_cast<size_t>(xb) * natoms + a) * kXAtomBytes, &xmap,
-                      a * (TF32 ? 32 : 64), rt * kTileM, b, &x_full[xb]);
+          tma_load_3d(xdst + a * kXAtomBytes, &xmap, a * kElem, rt * kTileM, b, &x_full[xb]);
+        tma_load_3d(xdst + natoms * kXAtomBytes, &xamap, 0, rt * kTileM, b, &x_full[xb]);
         x_iss[xb] = static_cast<int>(xph);
         if (++xb == XB) { xb = 0; xph ^= 1u; }
         for (int j = 0; j < nct; ++j) {
           if (!mbar_wait(&c_empty[cst], cph ^ 1u, g)) { ok = false; break; }
-          mbar_arrive_expect_tx(&c_full[cst], static_cast<uint32_t>(natoms) * BN * kAtomBytesPerRow);
+          uint8_t* cdst = cs + cst * csb;
+          mbar_arrive_expect_tx(&c_full[cst], static_cast<uint32_t>(csb));
           for (int a = 0; a < natoms; ++a)
-            tma_load_3d(cs + (static_cast<size_t>(cst) * natoms + a) * BN * kAtomBytesPerRow, &cmap,
-                        a * (TF32 ? 32 : 64), j * BN, b, &c_full[cst]);
+            tma_load_3d(cdst + static_cast<size_t>(a) * BN * kAtomBytesPerRow, &cmap, a * kElem, j * BN, b,
+                        &c_full[cst]);
+          tma_load_3d(cdst + static_cast<size_t>(natoms) * BN * kAtomBytesPerRow, &camap, 0, j * BN, b,
+                      &c_full[cst]);
           c_iss[cst] = static_cast<int>(cph);
           if (++cst == CS) { cst = 0; cph ^= 1u; }
-          if (!mbar_wait(&n_empty[ns], nph ^ 1u, g)) { ok = false; break; }
-          mbar_arrive_expect_tx(&n_full[ns], BN * 4);
-          bulk_load(cns + ns * BN, p.cn + static_cast<int64_t>(b) * p.Kp + static_cast<int64_t>(j) * BN, BN * 4,
-                    &n_full[ns]);
-          n_iss[ns] = static_cast<int>(nph);
-          if (++ns == kCnStages) { ns = 0; nph ^= 1u; }
         }
       }
       if (!ok) {
@@ -160,8 +248,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         g2.abort_flag = &never;
         for (int i = 0; i < XB; ++i) if (x_iss[i] >= 0) mbar_wait(&x_full[i], static_cast<uint32_t>(x_iss[i]), g2);
         for (int i = 0; i < CS; ++i) if (c_iss[i] >= 0) mbar_wait(&c_full[i], static_cast<uint32_t>(c_iss[i]), g2);
-        for (int i = 0; i < kCnStages; ++i)
-          if (n_iss[i] >= 0) mbar_wait(&n_full[i], static_cast<uint32_t>(n_iss[i]), g2);
       }
     }
   } else if (warp == 1) {
@@ -174,12 +260,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
         if (!mbar_wait(&x_full[xb], xph, g)) { ok = false; break; }
-        const uint32_t xaddr = smem_addr(xs + static_cast<size_t>(xb) * natoms * kXAtomBytes);
+        const uint32_t xaddr = smem_addr(xs + xb * xbb);
         for (int j = 0; j < nct; ++j) {
           if (!mbar_wait(&c_full[cst], cph, g)) { ok = false; break; }
           if (!mbar_wait(&a_empty[ab], aph ^ 1u, g)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t caddr = smem_addr(cs + static_cast<size_t>(cst) * natoms * BN * kAtomBytesPerRow);
+          const uint32_t caddr = smem_addr(cs + cst * csb);
           const uint32_t dtm = tmem_base + static_cast<uint32_t>(ab * BN);
           for (int a = 0; a < natoms; ++a) {
 #pragma unroll
@@ -189,6 +275,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
               umma_ss<TF32>(dtm, ad, bd, idesc, (a | s) != 0 ? 1u : 0u);
             }
           }
+          umma_ss<TF32>(dtm, sw32_kmajor_desc(xaddr + natoms * kXAtomBytes),
+                        sw32_kmajor_desc(caddr + natoms * BN * kAtomBytesPerRow), idesc, 1u);
           umma_commit(&c_empty[cst]);
           umma_commit(&a_full[ab]);
           if (++cst == CS) { cst = 0; cph ^= 1u; }
@@ -209,13 +297,17 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     // -------------------------------------------------- epilogue warps
     const int ew = warp - 2;
     const int q = warp & 3;   // TMEM lane quarter this warp may access
-    const int h = ew >> 2;    // column half of each accumulator tile
+    const int h = ew >> 2;    // column quarter of each accumulator tile
     const int r_local = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    int ab = 0, ns = 0;
-    uint32_t aph = 0, nph = 0, mph = 0;
+    int ab = 0;
+    uint32_t aph = 0, mph = 0;
     bool ok = true;
     double cta_obj = 0.0;
+    uint32_t ci[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) ci[i] = static_cast<uint32_t>(i) + p.zero;
+    const uint32_t kmask = ~31u + p.zero;
     for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
       const int b = static_cast<int>(t / p.tiles_per_inst);
       const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
@@ -224,66 +316,47 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       float best = CUDART_INF_F;
       int bk = 0;
       for (int j = 0; j < nct; ++j) {
-        if (!mbar_wait(&a_full[ab], aph, g) || !mbar_wait(&n_full[ns], nph, g)) { ok = false; break; }
+        if (!mbar_wait(&a_full[ab], aph, g)) { ok = false; break; }
         tc_fence_after();
-        const float* cnp = cns + ns * BN + h * kHalf;
-        float lb[4] = {CUDART_INF_F, CUDART_INF_F, CUDART_INF_F, CUDART_INF_F};
-        int li[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int c = 0; c < kHalf / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(ab * BN + h * kHalf + c * 32), v);
-#pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(cnp + c * 32 + i4 * 4);
-            const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float s = fmaf(-2.f, v[i4 * 4 + u], cv[u]);
-              const bool pr = s < lb[u];
-              lb[u] = pr ? s : lb[u];
-              li[u] = pr ? (c * 32 + i4 * 4 + u) : li[u];
-            }
+        for (int c = 0; c < kChunks; ++c) {
+          float v[CW];
+          tmem_ld<CW>(tmem_base + lane_off + static_cast<uint32_t>(ab * BN + h * kQ + c * CW), v);
+          const uint32_t m = chunk_min_key<CW>(v, ci, kmask);
+          const float mv = __uint_as_float(m & ~31u);
+          if (mv < best) {
+            best = mv;
+            bk = j * BN + h * kQ + c * CW + static_cast<int>(m & 31u);
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&a_empty[ab]);
-          mbar_arrive(&n_empty[ns]);
-        }
-        const int kbase = j * BN + h * kHalf;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int k = kbase + li[u];
-          if (lb[u] < best || (lb[u] == best && k < bk)) {
-            best = lb[u];
-            bk = k;
-          }
-        }
+        if (lane == 0) mbar_arrive(&a_empty[ab]);
         if (++ab == 2) { ab = 0; aph ^= 1u; }
-        if (++ns == kCnStages) { ns = 0; nph ^= 1u; }
       }
       if (!ok) break;
-      // merge the two column halves of this point tile
-      if (h == 1) {
+      // merge the four column quarters of this point tile
+      if (h != 0) {
         if (!mbar_wait(m_empty, mph ^ 1u, g)) { ok = false; break; }
-        mval[r_local] = best;
-        midx[r_local] = bk;
+        mval[(h - 1) * kTileM + r_local] = best;
+        midx[(h - 1) * kTileM + r_local] = bk;
         mbar_arrive(m_full);
       } else {
         if (!mbar_wait(m_full, mph, g)) { ok = false; break; }
-        const float ob = mval[r_local];
-        const int ok_ = midx[r_local];
-        mbar_arrive(m_empty);
-        if (ob < best || (ob == best && ok_ < bk)) {
-          best = ob;
-          bk = ok_;
+#pragma unroll
+        for (int hh = 0; hh < 3; ++hh) {
+          const float ov = mval[hh * kTileM + r_local];
+          const int ok_ = midx[hh * kTileM + r_local];
+          if (ov < best || (ov == best && ok_ < bk)) {
+            best = ov;
+            bk = ok_;
+          }
         }
+        mbar_arrive(m_empty);
         float md = 0.f;
         if (valid) {
           const int64_t o = static_cast<int64_t>(b) * p.rows + row;
-          md = fmaxf(0.f, p.xn[o] + best);
+          md = fmaxf(0.f, best);
           p.idx[o] = bk;
           if (p.mindist) p.mindist[o] = md;
         }
@@ -318,12 +391,11 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.nct = a.Kp / BN;
   k.tiles_per_inst = (a.rows + kTileM - 1) / kTileM;
   k.ntiles = k.tiles_per_inst * a.B;
-  k.xn = a.xn;
-  k.cn = a.cn;
   k.idx = a.idx;
   k.mindist = a.mindist;
   k.tobj = a.tobj;
   k.obj_per_cta = a.B == 1 ? 1 : 0;
+  k.zero = 0;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN>(k.natoms, k.XB, k.CS);
@@ -337,7 +409,8 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles_per_inst;
   if (grid <= 0) return cudaSuccess;
   count_launch();
-  k_assign<BN, TF32><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.cmap, k);
+  k_assign<BN, TF32><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
+                                                                               *a.camap, k);
   return cudaGetLastError();
 }
 

@@ -9,11 +9,11 @@
 
 namespace km {
 
-// One warp per point row: ||x||^2 in float32 and, in f32 mode, the TF32 split
-// operand [hi | hi | lo] (paired with the centroid split [hi | lo | hi] the
-// dot product becomes hi*hi + hi*lo + lo*hi).
+// One warp per point row (f32 mode): ||x||^2 into the augmentation row and
+// the TF32 split operand [hi | hi | lo] (paired with the centroid split
+// -2 [hi | lo | hi] the dot product becomes -2 (hi*hi + hi*lo + lo*hi)).
 __global__ void k_xprep(const void* __restrict__ X, int dtype, int64_t rows, int D, int Dp,
-                        float* __restrict__ xn, float* __restrict__ x3) {
+                        uint8_t* __restrict__ xaug, float* __restrict__ x3) {
   const int lane = threadIdx.x & 31;
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (r >= rows) return;
@@ -40,14 +40,14 @@ __global__ void k_xprep(const void* __restrict__ X, int dtype, int64_t rows, int
     }
   }
   s = warp_sum_f(s);
-  if (lane == 0) xn[r] = s;
+  if (lane == 0) write_aug_row(xaug + r * kAugBytes, dtype, s, 0);
 }
 
 // bf16 row norms with one 16-byte load per lane: LPR lanes cover a row (LPR a
 // power of two with LPR * 16 >= 2 * D), 32 / LPR rows per warp step.
 template <int LPR>
 __global__ void __launch_bounds__(256) k_xnorm_bf16(const uint8_t* __restrict__ X, int64_t rows, int row_bytes,
-                                                    float* __restrict__ xn) {
+                                                    uint8_t* __restrict__ xaug) {
   const int lane = threadIdx.x & 31;
   const int sub = lane / LPR, cl = lane % LPR;
   constexpr int RPW = 32 / LPR;
@@ -68,12 +68,13 @@ __global__ void __launch_bounds__(256) k_xnorm_bf16(const uint8_t* __restrict__ 
     }
 #pragma unroll
     for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (r < rows && cl == 0) xn[r] = s;
+    if (r < rows && cl == 0) write_aug_row(xaug + r * kAugBytes, kDtypeBF16, s, 0);
   }
 }
 
-cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, float* xn, float* x3,
+cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, void* xaug_v, float* x3,
                          cudaStream_t s) {
+  uint8_t* xaug = static_cast<uint8_t*>(xaug_v);
   if (rows <= 0) return cudaSuccess;
   if (dtype == kDtypeBF16) {
     const int row_bytes = 2 * D;
@@ -87,32 +88,32 @@ cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, 
     const uint8_t* Xb = static_cast<const uint8_t*>(X);
     count_launch();
     switch (lpr) {
-      case 1: k_xnorm_bf16<1><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
-      case 2: k_xnorm_bf16<2><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
-      case 4: k_xnorm_bf16<4><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
-      case 8: k_xnorm_bf16<8><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
-      case 16: k_xnorm_bf16<16><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
-      default: k_xnorm_bf16<32><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xn); break;
+      case 1: k_xnorm_bf16<1><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
+      case 2: k_xnorm_bf16<2><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
+      case 4: k_xnorm_bf16<4><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
+      case 8: k_xnorm_bf16<8><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
+      case 16: k_xnorm_bf16<16><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
+      default: k_xnorm_bf16<32><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
     }
     return cudaGetLastError();
   }
   const int threads = 256;
   const int64_t blocks = (rows * 32 + threads - 1) / threads;
   count_launch();
-  k_xprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(X, dtype, rows, D, Dp, xn, x3);
+  k_xprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(X, dtype, rows, D, Dp, xaug, x3);
   return cudaGetLastError();
 }
 
 // One warp per (instance, centroid row < Kp).
 __global__ void k_cprep(const void* __restrict__ src, int src_dtype, int B, int K, int Kp, int D, int Dp,
-                        int dtype, float* __restrict__ master, void* __restrict__ c_op, float* __restrict__ cn) {
+                        int dtype, float* __restrict__ master, void* __restrict__ c_op, uint8_t* __restrict__ caug) {
   const int lane = threadIdx.x & 31;
   const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (g >= static_cast<int64_t>(B) * Kp) return;
   const int b = static_cast<int>(g / Kp);
   const int k = static_cast<int>(g - static_cast<int64_t>(b) * Kp);
   if (k >= K) {
-    if (lane == 0) cn[g] = CUDART_INF_F;
+    if (lane == 0) write_aug_row(caug + g * kAugBytes, dtype, 0.f, 2);
     return;
   }
   const int64_t row = static_cast<int64_t>(b) * K + k;
@@ -127,17 +128,17 @@ __global__ void k_cprep(const void* __restrict__ src, int src_dtype, int B, int 
   }
   float s = emit_operand_row([&](int j) { return load_elem(src, src_dtype, row * D + j); }, D, Dp, dtype, orow,
                              lane);
-  if (lane == 0) cn[g] = s;
+  if (lane == 0) write_aug_row(caug + g * kAugBytes, dtype, s, 1);
 }
 
 cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, int D, int Dp, int dtype,
-                         float* master, void* c_op, float* cn, cudaStream_t s) {
+                         float* master, void* c_op, void* caug, cudaStream_t s) {
   const int threads = 256;
   const int64_t warps = static_cast<int64_t>(B) * Kp;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
   count_launch();
   k_cprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(src, src_dtype, B, K, Kp, D, Dp, dtype, master, c_op,
-                                                           cn);
+                                                           static_cast<uint8_t*>(caug));
   return cudaGetLastError();
 }
 

@@ -328,7 +328,7 @@ struct FinK {
   int mode;
   float* C;
   void* c_op;
-  float* cn;
+  uint8_t* caug;
   int32_t* counts;
   double* acc64;
   long long* cnt64;
@@ -355,7 +355,7 @@ __device__ void finish_cluster(const FinK& f, int k, int64_t cnt, const float* s
     __syncwarp();
     const float s = emit_operand_row([&](int j) { return crow[j]; }, f.D, f.Dp, f.dtype, op_row(f, k), lane);
     if (lane == 0) {
-      if (f.cn) f.cn[k] = s;
+      if (f.caug) write_aug_row(f.caug + static_cast<int64_t>(k) * kAugBytes, f.dtype, s, 1);
       if (f.counts) f.counts[k] = static_cast<int32_t>(cnt);
     }
   } else if (cnt > 0) {
@@ -464,7 +464,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.mode = a.mode;
   f.C = a.C;
   f.c_op = a.c_op;
-  f.cn = a.cn;
+  f.caug = static_cast<uint8_t*>(a.caug);
   f.counts = a.counts;
   f.acc64 = a.acc64;
   f.cnt64 = a.cnt64;
@@ -490,7 +490,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
 
 // Out-of-core: float64 accumulators -> centroids; resets the accumulators.
 __global__ void k_finalize_acc(int K, int D, int Dp, int dtype, double* acc64, long long* cnt64, float* C,
-                               void* c_op, float* cn, int32_t* counts, double* objacc, double* obj_out) {
+                               void* c_op, uint8_t* caug, int32_t* counts, double* objacc, double* obj_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * (blockDim.x >> 5) + warp;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -511,18 +511,18 @@ __global__ void k_finalize_acc(int K, int D, int Dp, int dtype, double* acc64, l
                                : static_cast<void*>(reinterpret_cast<float*>(c_op) + static_cast<int64_t>(k) * 3 * Dp);
   const float s = emit_operand_row([&](int j) { return crow[j]; }, D, Dp, dtype, orow, lane);
   if (lane == 0) {
-    if (cn) cn[k] = s;
+    if (caug) write_aug_row(caug + static_cast<int64_t>(k) * kAugBytes, dtype, s, 1);
     if (counts) counts[k] = static_cast<int32_t>(cnt);
     cnt64[k] = 0;
   }
 }
 
-cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, float* cn,
+cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, void* caug,
                                 int32_t* counts, double* objacc, double* obj_out, cudaStream_t s) {
   const int threads = 256;
   const int blocks = (p.K + 7) / 8;
   count_launch();
-  k_finalize_acc<<<blocks, threads, 0, s>>>(p.K, p.D, p.Dp, p.dtype, acc64, cnt64, C, c_op, cn, counts, objacc,
+  k_finalize_acc<<<blocks, threads, 0, s>>>(p.K, p.D, p.Dp, p.dtype, acc64, cnt64, C, c_op, static_cast<uint8_t*>(caug), counts, objacc,
                                             obj_out);
   return cudaGetLastError();
 }
@@ -539,7 +539,7 @@ struct SmallK {
   const int32_t* idx;
   float* C;
   void* c_op;
-  float* cn;
+  uint8_t* caug;
   int32_t* counts;
   const double* tobj;
   int64_t tiles_per_inst;
@@ -677,7 +677,7 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
                  : static_cast<void*>(reinterpret_cast<float*>(p.c_op) + grow * 3 * p.Dp);
     const float s = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, orow, lane);
     if (lane == 0) {
-      if (p.cn) p.cn[static_cast<int64_t>(b) * p.Kp + k] = s;
+      if (p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, s, 1);
       if (p.counts) p.counts[grow] = start[k + 1] - start[k];
     }
   }
@@ -717,7 +717,7 @@ static cudaError_t launch_small_t(const Plan& p, const SmallUpdateArgs& a, cudaS
   k.idx = a.idx;
   k.C = a.C;
   k.c_op = a.c_op;
-  k.cn = a.cn;
+  k.caug = static_cast<uint8_t*>(a.caug);
   k.counts = a.counts;
   k.tobj = a.tobj;
   k.tiles_per_inst = a.tiles_per_inst;

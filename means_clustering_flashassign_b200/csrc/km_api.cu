@@ -79,21 +79,29 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// 3-D tensor map over [B][rows][inner] with a (epa x box_rows x 1) box and
-// the 128-byte swizzle; out-of-range rows/columns read as zero.
-int encode_map(CUtensorMap* m, const void* ptr, bool f32, int64_t inner, int64_t rows, int B, int box_rows) {
+// 3-D tensor map over [B][rows][inner] with a (box_inner x box_rows x 1) box;
+// swizzle_bytes 128 or 32 (the box's inner extent in bytes); out-of-range
+// rows/columns read as zero.
+int encode_map(CUtensorMap* m, const void* ptr, bool f32, int64_t inner, int64_t rows, int B, int box_rows,
+               int swizzle_bytes = 128) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return fail(KM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * es), static_cast<cuuint64_t>(inner * es * rows)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(swizzle_bytes / es), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return KM_OK;
+}
+
+// Augmentation rows: 32 bytes per row (16 bf16 or 8 fp32), 32-byte swizzle.
+int encode_aug_map(CUtensorMap* m, const void* ptr, bool f32, int64_t rows, int B, int box_rows) {
+  return encode_map(m, ptr, f32, f32 ? 8 : 16, rows, B, box_rows, 32);
 }
 
 int check_device() {
@@ -236,10 +244,9 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     p.total = off;
     return KM_OK;
   }
-  p.off_xn = take(sizeof(float) * BR);
-  p.off_cn = take(sizeof(float) * static_cast<size_t>(B) * p.Kp);
-  if (op != KM_OP_ASSIGN || dtype == KM_F32)
-    p.off_clp = take(static_cast<size_t>(B) * K * p.Dop * (dtype == KM_BF16 ? 2 : 4));
+  p.off_xaug = take(32 * static_cast<size_t>(BR));
+  p.off_caug = take(32 * static_cast<size_t>(B) * p.Kp);
+  p.off_clp = take(static_cast<size_t>(B) * K * p.Dop * (dtype == KM_BF16 ? 2 : 4));
   if (dtype == KM_F32) p.off_x3 = take(sizeof(float) * BR * 3 * p.Dp);
   p.off_tobj = take(sizeof(double) * 4 * static_cast<size_t>(p.ntiles));
   if (op == KM_OP_FIT || op == KM_OP_FIT_HOST) p.off_idx = take(sizeof(int32_t) * BR);
@@ -297,7 +304,7 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 }
 
 // Update of one instance through the multi-kernel path.
-int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, float* cnb,
+int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
@@ -322,7 +329,7 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
   fa.mode = mode;
   fa.C = Cb;
   fa.c_op = c_opb;
-  fa.cn = cnb;
+  fa.caug = caugb;
   fa.counts = countsb;
   fa.acc64 = mode == 1 ? at<double>(c.ws, p.off_acc64) : nullptr;
   fa.cnt64 = mode == 1 ? at<long long>(c.ws, p.off_cnt64) : nullptr;
@@ -390,26 +397,23 @@ int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int 
   int r = prepare(c, KM_OP_ASSIGN, B, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
   if (r != KM_OK) return r;
   const Plan& p = c.p;
-  float* xn = at<float>(c.ws, p.off_xn);
-  float* cn = at<float>(c.ws, p.off_cn);
+  void* xaug = at<void>(c.ws, p.off_xaug);
+  void* caug = at<void>(c.ws, p.off_caug);
+  void* clp = at<void>(c.ws, p.off_clp);
+  const bool f32 = dtype == KM_F32;
   KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
-  CUtensorMap xmap, cmap;
-  if (dtype == KM_BF16) {
-    KM_CUDA(launch_xprep(X, kDtypeBF16, static_cast<int64_t>(B) * N, D, p.Dp, xn, nullptr, c.s));
-    KM_CUDA(launch_cprep(C, kDtypeBF16, B, K, p.Kp, D, p.Dp, kDtypeBF16, nullptr, nullptr, cn, c.s));
-    if ((r = encode_map(&xmap, X, false, D, N, B, kTileM)) != KM_OK) return r;
-    if ((r = encode_map(&cmap, C, false, D, K, B, p.ac.BN)) != KM_OK) return r;
-  } else {
-    float* x3 = at<float>(c.ws, p.off_x3);
-    float* c3 = at<float>(c.ws, p.off_clp);
-    KM_CUDA(launch_xprep(X, kDtypeF32, static_cast<int64_t>(B) * N, D, p.Dp, xn, x3, c.s));
-    KM_CUDA(launch_cprep(C, kDtypeF32, B, K, p.Kp, D, p.Dp, kDtypeF32, nullptr, c3, cn, c.s));
-    if ((r = encode_map(&xmap, x3, true, p.Dop, N, B, kTileM)) != KM_OK) return r;
-    if ((r = encode_map(&cmap, c3, true, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
-  }
+  float* x3 = f32 ? at<float>(c.ws, p.off_x3) : nullptr;
+  KM_CUDA(launch_xprep(X, dtype, static_cast<int64_t>(B) * N, D, p.Dp, xaug, x3, c.s));
+  KM_CUDA(launch_cprep(C, dtype, B, K, p.Kp, D, p.Dp, dtype, nullptr, clp, caug, c.s));
+  CUtensorMap xmap, xamap, cmap, camap;
+  if ((r = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : X, f32, p.Dop, N, B, kTileM)) != KM_OK) return r;
+  if ((r = encode_aug_map(&xamap, xaug, f32, N, B, kTileM)) != KM_OK) return r;
+  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
+  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, p.ac.BN)) != KM_OK) return r;
   double* tobj = at<double>(c.ws, p.off_tobj);
   int64_t groups = 0;
-  AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, mindist, tobj, c.status(), wait_limit_ns(), &groups};
+  AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, mindist, tobj, c.status(), wait_limit_ns(),
+               &groups};
   KM_CUDA(launch_assign(p, a, c.s));
   if (objective) KM_CUDA(launch_objective(tobj, B, groups, objective, 1, c.s));
   return KM_OK;
@@ -450,35 +454,33 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   int r = prepare(c, KM_OP_FIT, B, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
   if (r != KM_OK) return r;
   const Plan& p = c.p;
-  float* xn = at<float>(c.ws, p.off_xn);
-  float* cn = at<float>(c.ws, p.off_cn);
+  void* xaug = at<void>(c.ws, p.off_xaug);
+  uint8_t* caug = at<uint8_t>(c.ws, p.off_caug);
   void* clp = at<void>(c.ws, p.off_clp);
   double* tobj = at<double>(c.ws, p.off_tobj);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(c.ws, p.off_idx);
   double* objs = at<double>(c.ws, p.off_obj);
+  const bool f32 = dtype == KM_F32;
   KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
-  CUtensorMap xmap, cmap;
-  if (dtype == KM_BF16) {
-    KM_CUDA(launch_xprep(X, kDtypeBF16, static_cast<int64_t>(B) * N, D, p.Dp, xn, nullptr, c.s));
-    if ((r = encode_map(&xmap, X, false, D, N, B, kTileM)) != KM_OK) return r;
-    if ((r = encode_map(&cmap, clp, false, D, K, B, p.ac.BN)) != KM_OK) return r;
-  } else {
-    float* x3 = at<float>(c.ws, p.off_x3);
-    KM_CUDA(launch_xprep(X, kDtypeF32, static_cast<int64_t>(B) * N, D, p.Dp, xn, x3, c.s));
-    if ((r = encode_map(&xmap, x3, true, p.Dop, N, B, kTileM)) != KM_OK) return r;
-    if ((r = encode_map(&cmap, clp, true, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
-  }
-  KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, cn, c.s));
+  float* x3 = f32 ? at<float>(c.ws, p.off_x3) : nullptr;
+  KM_CUDA(launch_xprep(X, dtype, static_cast<int64_t>(B) * N, D, p.Dp, xaug, x3, c.s));
+  CUtensorMap xmap, xamap, cmap, camap;
+  if ((r = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : X, f32, p.Dop, N, B, kTileM)) != KM_OK) return r;
+  if ((r = encode_aug_map(&xamap, xaug, f32, N, B, kTileM)) != KM_OK) return r;
+  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
+  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, p.ac.BN)) != KM_OK) return r;
+  KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
-    AssignArgs a{&xmap, &cmap, B, N, K, p.Kp, xn, cn, idx, nullptr, tobj, c.status(), wait_limit_ns(), &groups};
+    AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
+                 &groups};
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t], c.s));
     KM_CUDA(launch_assign(p, a, c.s));
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
     if (p.small_update) {
-      SmallUpdateArgs u{X,    idx,       C_out, clp, cn, counts_out, tobj, p.tiles_per_inst,
+      SmallUpdateArgs u{X,    idx,       C_out, clp, caug, counts_out, tobj, p.tiles_per_inst,
                         objective_hist ? objective_hist + t : objs, objective_hist ? iters : 1};
       KM_CUDA(launch_small_update(p, u, c.s));
     } else {
@@ -486,7 +488,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
         double* ob = objective_hist ? objective_hist + static_cast<int64_t>(b) * iters + t : objs + b;
         r = update_instance(c, static_cast<const uint8_t*>(X) + b * xstride, idx + static_cast<int64_t>(b) * N, N,
                             C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
-                            cn + static_cast<int64_t>(b) * p.Kp,
+                            caug + static_cast<int64_t>(b) * p.Kp * 32,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
                             tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0);
         if (r != KM_OK) return r;
@@ -556,8 +558,8 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
   cudaPointerAttributes pa;
   KM_CUDA(cudaPointerGetAttributes(&pa, X_host));
   if (pa.type != cudaMemoryTypeHost) return fail(KM_ERR_INVALID_ARG, "X_host must be page-locked host memory");
-  float* xn = at<float>(c.ws, p.off_xn);
-  float* cn = at<float>(c.ws, p.off_cn);
+  void* xaug = at<void>(c.ws, p.off_xaug);
+  void* caug = at<void>(c.ws, p.off_caug);
   void* clp = at<void>(c.ws, p.off_clp);
   double* tobj = at<double>(c.ws, p.off_tobj);
   double* objs = at<double>(c.ws, p.off_obj);
@@ -586,11 +588,13 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
     KM_CUDA(cudaMemsetAsync(acc64, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
     KM_CUDA(cudaMemsetAsync(cnt64, 0, sizeof(long long) * K, c.s));
     KM_CUDA(cudaMemsetAsync(objacc, 0, sizeof(double), c.s));
-    KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, cn, c.s));
+    KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
     for (int i = 0; i < 2; ++i) KM_CUDA(cudaEventRecord(ev_free[i], c.s));
-    CUtensorMap cmap;
-    int rr = encode_map(&cmap, clp, dtype == KM_F32, p.Dop, K, 1, p.ac.BN);
+    const bool f32 = dtype == KM_F32;
+    CUtensorMap cmap, camap;
+    int rr = encode_map(&cmap, clp, f32, p.Dop, K, 1, p.ac.BN);
     if (rr != KM_OK) return rr;
+    if ((rr = encode_aug_map(&camap, caug, f32, p.Kp, 1, p.ac.BN)) != KM_OK) return rr;
     const int64_t nch = (N + p.chunk_rows - 1) / p.chunk_rows;
     const size_t rowb = static_cast<size_t>(D) * p.es;
     int64_t g = 0;
@@ -604,19 +608,19 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
                                 cudaMemcpyHostToDevice, cs));
         KM_CUDA(cudaEventRecord(ev_copied[bi], cs));
         KM_CUDA(cudaStreamWaitEvent(c.s, ev_copied[bi], 0));
-        CUtensorMap xmap;
-        KM_CUDA(launch_xprep(dbuf[bi], dtype, nr, D, p.Dp, xn, x3, c.s));
-        rr = dtype == KM_BF16 ? encode_map(&xmap, dbuf[bi], false, D, nr, 1, kTileM)
-                              : encode_map(&xmap, x3, true, p.Dop, nr, 1, kTileM);
+        CUtensorMap xmap, xamap;
+        KM_CUDA(launch_xprep(dbuf[bi], dtype, nr, D, p.Dp, xaug, x3, c.s));
+        rr = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : dbuf[bi], f32, p.Dop, nr, 1, kTileM);
         if (rr != KM_OK) return rr;
+        if ((rr = encode_aug_map(&xamap, xaug, f32, nr, 1, kTileM)) != KM_OK) return rr;
         int32_t* idxc = idx_out ? idx_out + r0 : at<int32_t>(c.ws, p.off_idx);
         Plan pc = p;
         pc.rows = nr;
         pc.tiles_per_inst = (nr + kTileM - 1) / kTileM;
         pc.ntiles = pc.tiles_per_inst;
         int64_t groups = 0;
-        AssignArgs a{&xmap, &cmap, 1, nr, K, p.Kp, xn, cn, idxc, nullptr, tobj, c.status(), wait_limit_ns(),
-                     &groups};
+        AssignArgs a{&xmap, &xamap, &cmap, &camap, 1, nr, K, p.Kp, idxc, nullptr, tobj, c.status(),
+                     wait_limit_ns(), &groups};
         KM_CUDA(launch_assign(pc, a, c.s));
         Ctx cc = c;
         cc.p = pc;
@@ -624,7 +628,7 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
       }
-      KM_CUDA(launch_finalize_acc(p, acc64, cnt64, C_out, clp, cn, counts_out, objacc, objs + t, c.s));
+      KM_CUDA(launch_finalize_acc(p, acc64, cnt64, C_out, clp, caug, counts_out, objacc, objs + t, c.s));
     }
     KM_CUDA(cudaStreamSynchronize(c.s));
     if (objective_hist && iters > 0)

@@ -15,8 +15,7 @@ constexpr int kDtypeBF16 = 1;
 
 // Rows of points per FlashAssign tile (UMMA M) and warps of that kernel.
 constexpr int kTileM = 128;
-constexpr int kAssignThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
-constexpr int kCnStages = 4;         // ring of centroid-norm tiles
+constexpr int kAssignThreads = 576;  // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
 
 // Largest problem the single-CTA fused update handles (batched path).
 constexpr int kSmallMaxN = 8192;
@@ -74,7 +73,7 @@ struct Plan {
   SortCfg sc;
   SegCfg gc;
   // workspace offsets (bytes)
-  size_t off_hdr = 0, off_xn = 0, off_cn = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
+  size_t off_hdr = 0, off_xaug = 0, off_caug = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
   size_t off_blkhist = 0, off_total = 0, off_keys = 0, off_vals = 0, off_perm = 0, off_start = 0, off_skeys = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
@@ -89,27 +88,29 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
               const char** why);
 
 // ------------------------------------------------------------- launchers
-// Row norms ||x||^2 (float32) of `rows` points; in f32 mode also writes the
-// TF32 split operand x3 = [hi | hi | lo] (rows x 3*Dp floats).
-cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, float* xn, float* x3,
+// Norm augmentation rows (32 bytes per point, see km_rows.cuh) of `rows`
+// points; in f32 mode also the TF32 split operand x3 = [hi | hi | lo]
+// (rows x 3*Dp floats).
+cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, void* xaug, float* x3,
                          cudaStream_t s);
 
 // Centroid operand preparation for B instances of K centroids:
 //   src (dtype src_dtype: bf16 or f32) -> optional float32 master copy,
-//   bf16 operand copy (bf16 mode) or TF32 split [hi | lo | hi] (f32 mode),
-//   and ||c||^2 of the values the MMA sees; rows K..Kp-1 get +inf norms.
+//   -2c operand copy (bf16, or the TF32 split -2 [hi | lo | hi]) and the
+//   augmentation rows [B][Kp] holding ||c||^2 of the values the MMA sees;
+//   rows K..Kp-1 get the +inf padding row.
 cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, int D, int Dp, int dtype,
-                         float* master, void* c_op, float* cn, cudaStream_t s);
+                         float* master, void* c_op, void* caug, cudaStream_t s);
 
 // FlashAssign over B instances of `rows` points (tcgen05 / TMEM / TMA).
 struct AssignArgs {
-  const CUtensorMap* xmap;  // host copies, passed by value to the kernel
-  const CUtensorMap* cmap;
+  const CUtensorMap* xmap;   // host copies, passed by value to the kernel
+  const CUtensorMap* xamap;  // point augmentation rows
+  const CUtensorMap* cmap;   // -2c operand
+  const CUtensorMap* camap;  // centroid augmentation rows (Kp rows)
   int B;
   int64_t rows;
   int K, Kp;
-  const float* xn;
-  const float* cn;
   int32_t* idx;
   float* mindist;
   double* tobj;  // B == 1: [assign CTAs][4]; else [B * tiles_per_inst][4]
@@ -161,8 +162,8 @@ struct FinalizeArgs {
   const float* pr;
   int mode;          // 0: write centroids; 1: accumulate into acc64/cnt64
   float* C;          // [K][D] float master (in: previous, out: new)
-  void* c_op;        // operand copy for the next assign (bf16 or TF32 split)
-  float* cn;         // [Kp]
+  void* c_op;        // operand copy for the next assign (-2c, bf16 or TF32 split)
+  void* caug;        // [Kp] augmentation rows
   int32_t* counts;   // [K] or null
   double* acc64;     // [K][D] (mode 1)
   long long* cnt64;  // [K] (mode 1)
@@ -173,7 +174,7 @@ struct FinalizeArgs {
 cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s);
 
 // Final step of the out-of-core update: centroids from float64 accumulators.
-cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, float* cn,
+cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, void* caug,
                                 int32_t* counts, double* objacc, double* obj_out, cudaStream_t s);
 
 // Fused single-CTA-per-instance update (sort + segmented sums + finalise) for
@@ -183,7 +184,7 @@ struct SmallUpdateArgs {
   const int32_t* idx;
   float* C;
   void* c_op;  // may be null
-  float* cn;   // may be null
+  void* caug;  // [B][Kp] augmentation rows, may be null
   int32_t* counts;
   const double* tobj;  // may be null
   int64_t tiles_per_inst;
