@@ -27,56 +27,78 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 
 __device__ __forceinline__ int32_t clamp_key(int32_t k, int K) { return k < 0 ? 0 : (k >= K ? K - 1 : k); }
 
-__global__ void k_sort_hist(const int32_t* __restrict__ keys, int64_t n, int T, int shift, int R,
-                            int64_t nblk, int32_t* __restrict__ blkhist, int K) {
+// Digit counts of each block's T keys, block-major: blkhist[b][d].
+// Pass 0 reads the assignment vector, later passes the (point, key) pairs.
+template <bool PAIRS>
+__global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ keys, const int2* __restrict__ pairs,
+                                                   int64_t n, int T, int shift, int R, int32_t* __restrict__ blkhist,
+                                                   int K) {
   extern __shared__ int32_t sh[];
   constexpr int kPer = 16;  // keys per thread (T == blockDim.x * kPer)
   for (int d = threadIdx.x; d < R; d += blockDim.x) sh[d] = 0;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
-  const int lane = threadIdx.x & 31;
   int dig[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {  // all loads first, then the counting
     const int64_t i = t0 + static_cast<int64_t>(j) * blockDim.x + threadIdx.x;
-    dig[j] = (i < n && j * static_cast<int>(blockDim.x) < T) ? ((clamp_key(keys[i], K) >> shift) & (R - 1)) : -1;
+    int key = 0;
+    if (i < n) key = PAIRS ? pairs[i].y : clamp_key(keys[i], K);
+    dig[j] = i < n ? ((key >> shift) & (R - 1)) : -1;
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const uint32_t peers = __match_any_sync(0xffffffffu, dig[j]);
-    if (dig[j] >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh[dig[j]], __popc(peers));
-  }
+  for (int j = 0; j < kPer; ++j)
+    if (dig[j] >= 0) atomicAdd(&sh[dig[j]], 1);
   __syncthreads();
-  for (int d = threadIdx.x; d < R; d += blockDim.x) blkhist[static_cast<int64_t>(d) * nblk + blockIdx.x] = sh[d];
+  int32_t* out = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  for (int d = threadIdx.x; d < R; d += blockDim.x) out[d] = sh[d];
 }
 
-// One warp per digit: in-place exclusive scan of blkhist[d][0..nblk) and the
-// digit total.
-__global__ void k_sort_colscan(int32_t* __restrict__ blkhist, int R, int64_t nblk, int32_t* __restrict__ total) {
-  const int lane = threadIdx.x & 31;
-  const int d = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  if (d >= R) return;
-  int32_t* row = blkhist + static_cast<int64_t>(d) * nblk;
-  int32_t carry = 0;
-  for (int64_t b0 = 0; b0 < nblk; b0 += 32) {
-    const int64_t b = b0 + lane;
-    const int32_t v = b < nblk ? row[b] : 0;
-    int32_t x = v;
+// In-place exclusive scan of blkhist[0..nblk)[d] over the blocks, and the
+// digit totals.  A block takes 32 digits (one per lane, so every load is
+// coalesced) and splits the block range among its 8 warps: each warp sums
+// its part, the parts are scanned in shared memory, and each warp rewrites
+// its part as running prefixes.
+__global__ void __launch_bounds__(256) k_sort_colscan(int32_t* __restrict__ blkhist, int R, int64_t nblk,
+                                                      int32_t* __restrict__ total) {
+  __shared__ int32_t part[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int d = blockIdx.x * 32 + lane;
+  const bool ok = d < R;
+  const int64_t seg = (nblk + 7) / 8;
+  const int64_t b0 = warp * seg < nblk ? warp * seg : nblk;
+  const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
+  constexpr int CH = 8;
+  int32_t s = 0;
+  for (int64_t b = b0; b < b1; b += CH) {
+    int32_t v[CH];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+    for (int u = 0; u < CH; ++u) v[u] = (ok && b + u < b1) ? blkhist[(b + u) * R + d] : 0;
+#pragma unroll
+    for (int u = 0; u < CH; ++u) s += v[u];
+  }
+  part[warp][lane] = s;
+  __syncthreads();
+  int32_t run = 0;
+  for (int w = 0; w < warp; ++w) run += part[w][lane];
+  if (warp == 7 && ok) total[d] = run + s;
+  for (int64_t b = b0; b < b1; b += CH) {
+    int32_t v[CH];
+#pragma unroll
+    for (int u = 0; u < CH; ++u) v[u] = (ok && b + u < b1) ? blkhist[(b + u) * R + d] : 0;
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      if (ok && b + u < b1) blkhist[(b + u) * R + d] = run;
+      run += v[u];
     }
-    if (b < nblk) row[b] = carry + x - v;
-    carry += __shfl_sync(0xffffffffu, x, 31);
   }
-  if (lane == 0) total[d] = carry;
 }
 
-// Block-wide exclusive scan of total[0..R) into base[0..R) (shared memory):
-// contiguous per-thread runs, a warp-shuffle scan of the run sums, then a
-// scan of the warp sums by warp 0.  tmp needs blockDim.x / 32 ints.
-__device__ void block_exclusive_scan(const int32_t* __restrict__ total, int R, int32_t* base, int32_t* tmp) {
+// Block-wide exclusive scan of total[0..R) into base[0..R) (shared memory;
+// base may alias total): contiguous per-thread runs, a warp-shuffle scan of
+// the run sums, then a scan of the warp sums by warp 0.  tmp needs
+// blockDim.x / 32 ints.
+__device__ void block_exclusive_scan(const int32_t* total, int R, int32_t* base, int32_t* tmp) {
   const int nt = blockDim.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nt >> 5;
   const int per = (R + nt - 1) / nt;
@@ -104,22 +126,31 @@ __device__ void block_exclusive_scan(const int32_t* __restrict__ total, int R, i
   __syncthreads();
   int32_t run = tmp[warp] + x - s;
   for (int i = lo; i < lo + per && i < R; ++i) {
+    const int32_t t = total[i];
     base[i] = run;
-    run += total[i];
+    run += t;
   }
   __syncthreads();
 }
 
-template <int IPT>
-__global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int64_t n,
-                               int T, int shift, int R, int64_t nblk, const int32_t* __restrict__ blkhist,
-                               const int32_t* __restrict__ total, int32_t* __restrict__ keys_out,
-                               int32_t* __restrict__ vals_out, int32_t* __restrict__ start, int K) {
+// Stable scatter of one pass: per-warp counters rank equal digits in point
+// order (match.any groups equal digits inside a warp step).  The block first
+// places its elements in digit order in shared memory, then writes them out
+// in that order, so elements of one digit leave as one contiguous run at
+// base[d] + (earlier blocks' d).  Writes one 8-byte (point, key) pair per
+// element, and optionally the bare point index (perm_out) on the last pass.
+template <int IPT, bool PAIRS>
+__global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n,
+                               int T, int shift, int R, const int32_t* __restrict__ blkhist,
+                               const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
+                               int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
   extern __shared__ int32_t sh[];
   const int W = blockDim.x >> 5;
-  int32_t* base = sh;               // [R]
-  int32_t* wcnt = sh + R;           // [W][R]
-  int32_t* tmp = wcnt + W * R;      // [blockDim.x / 32]
+  int2* stage = reinterpret_cast<int2*>(sh);   // [T]
+  int32_t* base = sh + 2 * T;                  // [R]  global start of each digit in this block
+  int32_t* lstart = base + R;                  // [R]  block-local start of each digit
+  int32_t* wcnt = lstart + R;                  // [W][R]
+  int32_t* tmp = wcnt + W * R;                 // [blockDim.x / 32]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   block_exclusive_scan(total, R, base, tmp);
@@ -134,12 +165,19 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int32_
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
   const int64_t w0 = t0 + static_cast<int64_t>(warp) * (T / W);
   int dig[IPT], rank[IPT];
-  int32_t key[IPT];
+  int32_t key[IPT], val[IPT];
   const uint32_t ltm = lanemask_lt();
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {  // all loads first
     const int64_t i = w0 + s * 32 + lane;
-    key[s] = i < n ? clamp_key(keys_in[i], K) : 0;
+    if (PAIRS) {
+      const int2 pk = i < n ? pairs_in[i] : make_int2(0, 0);
+      val[s] = pk.x;
+      key[s] = pk.y;
+    } else {
+      val[s] = static_cast<int32_t>(i);
+      key[s] = i < n ? clamp_key(keys_in[i], K) : 0;
+    }
     dig[s] = i < n ? ((key[s] >> shift) & (R - 1)) : -1;
   }
 #pragma unroll
@@ -155,38 +193,52 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int32_
     __syncwarp();
   }
   __syncthreads();
+  // per digit: block count -> block-local starts (scan over digits), then
+  // warp offsets inside the digit's local run
   for (int d = threadIdx.x; d < R; d += blockDim.x) {
-    int32_t run = base[d] + blkhist[static_cast<int64_t>(d) * nblk + blockIdx.x];
+    int32_t c = 0;
+    for (int w = 0; w < W; ++w) c += wcnt[w * R + d];
+    lstart[d] = c;
+  }
+  __syncthreads();
+  block_exclusive_scan(lstart, R, lstart, tmp);
+  const int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  for (int d = threadIdx.x; d < R; d += blockDim.x) {
+    int32_t run = lstart[d];
     for (int w = 0; w < W; ++w) {
       const int32_t c = wcnt[w * R + d];
       wcnt[w * R + d] = run;
       run += c;
     }
+    base[d] += boff[d] - lstart[d];  // global position = base[d] + local position
   }
   __syncthreads();
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
-    const int64_t i = w0 + s * 32 + lane;
-    if (i < n) {
-      const int32_t pos = wcnt[warp * R + dig[s]] + rank[s];
-      vals_out[pos] = vals_in ? vals_in[i] : static_cast<int32_t>(i);
-      if (keys_out) keys_out[pos] = key[s];
-    }
+    if (dig[s] >= 0) stage[wcnt[warp * R + dig[s]] + rank[s]] = make_int2(val[s], key[s]);
+  }
+  __syncthreads();
+  const int nvalid = static_cast<int>((n - t0) < T ? (n - t0) : T);
+  for (int i = threadIdx.x; i < nvalid; i += blockDim.x) {
+    const int2 pk = stage[i];
+    const int32_t pos = base[(pk.y >> shift) & (R - 1)] + i;
+    pairs_out[pos] = pk;
+    if (perm_out) perm_out[pos] = pk.x;
   }
 }
 
-// start[k] for every k in [0, K] from sorted keys: each change point i (or
-// the ends) writes the starts of all clusters between the two keys.
-__global__ void k_bounds(const int32_t* __restrict__ sorted, int64_t n, int K, int32_t* __restrict__ start) {
+// start[k] for every k in [0, K] from the sorted pairs: each change point i
+// (or the ends) writes the starts of all clusters between the two keys.
+__global__ void k_bounds(const int2* __restrict__ sorted, int64_t n, int K, int32_t* __restrict__ start) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i > n) return;
-  const int a = i == 0 ? -1 : clamp_key(sorted[i - 1], K);
-  const int c = i == n ? K : clamp_key(sorted[i], K);
+  const int a = i == 0 ? -1 : clamp_key(sorted[i - 1].y, K);
+  const int c = i == n ? K : clamp_key(sorted[i].y, K);
   for (int k = a + 1; k <= c; ++k) start[k] = static_cast<int32_t>(i);
 }
 
-static size_t scatter_smem(int R, int W, int threads) {
-  return (static_cast<size_t>(R) + static_cast<size_t>(W) * R + threads) * 4;
+static size_t scatter_smem(int R, int W, int threads, int T) {
+  return (2 * static_cast<size_t>(T) + 2 * static_cast<size_t>(R) + static_cast<size_t>(W) * R + threads) * 4;
 }
 
 cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
@@ -194,34 +246,43 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
   const int threads = c.W * 32;
   const int64_t nblk = (a.n + c.T - 1) / c.T;
   if (a.n <= 0) return cudaSuccess;
-  const int32_t* kin = a.keys;
-  const int32_t* vin = nullptr;
   for (int ps = 0; ps < c.passes; ++ps) {
     const int R = 1 << c.bits[ps];
     const bool last = ps == c.passes - 1;
+    const bool pairs_in = ps > 0;
     count_launch(3);  // hist, colscan, scatter
-    k_sort_hist<<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(kin, a.n, c.T, c.shift[ps], R, nblk, a.blkhist,
-                                                                a.K);
-    const int cw = 8;
-    k_sort_colscan<<<(R + cw - 1) / cw, cw * 32, 0, s>>>(a.blkhist, R, nblk, a.total);
-    // pass 0 of two writes (keys_tmp, vals_tmp); the last pass writes perm
-    // and the sorted keys (the segment id of every sorted position).
-    int32_t* kout = last ? a.skeys : a.keys_tmp;
-    int32_t* vout = last ? a.perm : a.vals_tmp;
-    const size_t sm = scatter_smem(R, c.W, threads);
+    if (pairs_in)
+      k_sort_hist<true><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps],
+                                                                        R, a.blkhist, a.K);
+    else
+      k_sort_hist<false><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(a.keys, nullptr, a.n, c.T, c.shift[ps], R,
+                                                                         a.blkhist, a.K);
+    k_sort_colscan<<<(R + 31) / 32, 256, 0, s>>>(a.blkhist, R, nblk, a.total);
+    // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
+    // (and perm when asked for).
+    int2* out = last ? a.pairs : a.pairs_tmp;
+    int32_t* perm = last ? a.perm : nullptr;
+    const size_t sm = scatter_smem(R, c.W, threads, c.T);
     int32_t* st = (last && c.passes == 1) ? a.start : nullptr;
-    cudaError_t e = cudaFuncSetAttribute(k_sort_scatter<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sm));
-    if (e != cudaSuccess) return e;
-    k_sort_scatter<16><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
-        kin, vin, a.n, c.T, c.shift[ps], R, nblk, a.blkhist, a.total, kout, vout, st, a.K);
-    kin = kout;
-    vin = vout;
+    cudaError_t e;
+    if (pairs_in) {
+      e = cudaFuncSetAttribute(k_sort_scatter<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sm));
+      if (e != cudaSuccess) return e;
+      k_sort_scatter<16, true><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
+          nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps], R, a.blkhist, a.total, out, perm, st, a.K);
+    } else {
+      e = cudaFuncSetAttribute(k_sort_scatter<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sm));
+      if (e != cudaSuccess) return e;
+      k_sort_scatter<16, false><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
+          a.keys, nullptr, a.n, c.T, c.shift[ps], R, a.blkhist, a.total, out, perm, st, a.K);
+    }
   }
   if (c.passes > 1) {
     const int64_t cnt = a.n + 1;
     count_launch();
-    k_bounds<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(a.skeys, a.n, a.K, a.start);
+    k_bounds<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(a.pairs, a.n, a.K, a.start);
   }
   return cudaGetLastError();
 }

@@ -24,7 +24,7 @@ namespace km {
 template <int LPR>
 struct RowGeom {
   static constexpr int RPS = 32 / LPR;                    // rows per step
-  static constexpr int STEPS = LPR < 16 ? LPR : 16;        // steps per batch
+  static constexpr int STEPS = LPR < 8 ? LPR : 8;          // steps (16-byte loads per lane) per batch
   static constexpr int BATCH = STEPS * RPS;               // rows per batch (<= 32)
 };
 
@@ -142,8 +142,7 @@ __device__ __forceinline__ void warp_range_sums(const uint8_t* X, int row_bytes,
 // -1 when unused, vectors in slot_v[2][D]).
 template <int LPR, bool BF16, class FinalStore>
 __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D,
-                                                      const int32_t* __restrict__ perm,
-                                                      const int32_t* __restrict__ skeys, int64_t n, int64_t q0,
+                                                      const int2* __restrict__ pairs, int64_t n, int64_t q0,
                                                       int64_t q1, int lane, int* slot_k, float* slot_v,
                                                       FinalStore final_store) {
   using G = RowGeom<LPR>;
@@ -152,10 +151,10 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
   const int sub = lane / LPR;
   const int cl = lane % LPR;
   const bool active = cl * 16 < row_bytes;
-  const int kfirst = skeys[q0];
-  const bool left_cont = q0 > 0 && skeys[q0 - 1] == kfirst;
-  const int klast = skeys[q1 - 1];
-  const bool right_cont = q1 < n && skeys[q1] == klast;
+  const int kfirst = pairs[q0].y;
+  const bool left_cont = q0 > 0 && pairs[q0 - 1].y == kfirst;
+  const int klast = pairs[q1 - 1].y;
+  const bool right_cont = q1 < n && pairs[q1].y == klast;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -177,13 +176,11 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   };
   const bool in_batch = lane < G::BATCH;
-  int pv = (in_batch && q0 + lane < q1) ? perm[q0 + lane] : -1;
-  int kv = (in_batch && q0 + lane < q1) ? skeys[q0 + lane] : -1;
+  int2 pv = (in_batch && q0 + lane < q1) ? pairs[q0 + lane] : make_int2(-1, -1);
   for (int64_t p = q0; p < q1; p += G::BATCH) {
-    const int cur_p = pv, cur_k = kv;
+    const int cur_p = pv.x, cur_k = pv.y;
     const int64_t pn = p + G::BATCH;
-    pv = (in_batch && pn + lane < q1) ? perm[pn + lane] : -1;
-    kv = (in_batch && pn + lane < q1) ? skeys[pn + lane] : -1;
+    pv = (in_batch && pn + lane < q1) ? pairs[pn + lane] : make_int2(-1, -1);
     const int nb = q1 - p < G::BATCH ? static_cast<int>(q1 - p) : G::BATCH;
     int prevk = __shfl_up_sync(0xffffffffu, cur_k, 1);
     if (lane == 0) prevk = open_k;
@@ -216,85 +213,77 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
 }
 
 // ------------------------------------------------------------ big path
-// Persistent blocks walk chunks of W*L sorted positions.  Per chunk: each
-// warp sums its L positions, then the block combines the runs cut at warp
-// edges in position order; runs inside the chunk become final sums, a run
-// continuing past the chunk's left edge goes to pl[chunk], one continuing
-// only past its right edge to pr[chunk].
+// One wave of blocks; block c owns sorted positions [c*P, (c+1)*P), split in
+// 8 contiguous warp ranges.  Each warp sums its range; then the block
+// combines the runs cut at warp edges in position order: runs inside the
+// block's range become final sums, a run continuing past its left edge goes
+// to pl[c], one continuing only past its right edge to pr[c].
 template <int LPR, bool BF16>
-__global__ void __launch_bounds__(256) k_segsum(const uint8_t* __restrict__ X, int64_t n, int D, int row_bytes,
-                                                const int32_t* __restrict__ perm, const int32_t* __restrict__ skeys,
-                                                const int32_t* __restrict__ start, int L, int64_t nchunks,
-                                                float* __restrict__ sums, float* __restrict__ pl,
-                                                float* __restrict__ pr) {
+__global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X, int64_t n, int D, int row_bytes,
+                                                   const int2* __restrict__ pairs,
+                                                   const int32_t* __restrict__ start, int64_t P,
+                                                   float* __restrict__ sums, float* __restrict__ pl,
+                                                   float* __restrict__ pr) {
   extern __shared__ float sm[];
   constexpr int W = 8;
   int* slot_k = reinterpret_cast<int*>(sm);          // [W][2]
   float* slot_v = sm + 2 * W;                         // [W][2][D]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
-    const int64_t p0 = c * W * L;
-    const int64_t p1 = p0 + static_cast<int64_t>(W) * L < n ? p0 + static_cast<int64_t>(W) * L : n;
-    const int64_t q0 = p0 + static_cast<int64_t>(warp) * L < p1 ? p0 + static_cast<int64_t>(warp) * L : p1;
-    const int64_t q1 = q0 + L < p1 ? q0 + L : p1;
-    warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, perm, skeys, n, q0, q1, lane, slot_k + 2 * warp,
-                                     slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
-                                       store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane,
-                                                            acc, 1.f);
-                                     });
-    __syncthreads();
-    // Ordered combine of the cut runs, one thread per column.
-    for (int j = threadIdx.x; j < D; j += blockDim.x) {
-      int open = -1;
-      float a = 0.f;
-      auto flush = [&](int k, float v) {
-        const int64_t s0 = start[k], s1 = start[k + 1];
-        if (s0 >= p0 && s1 <= p1) sums[static_cast<int64_t>(k) * D + j] = v;
-        else if (s0 < p0) pl[c * D + j] = v;
-        else pr[c * D + j] = v;
-      };
-      for (int w = 0; w < W; ++w) {
-        for (int sl = 0; sl < 2; ++sl) {
-          const int k = slot_k[2 * w + sl];
-          if (k < 0) continue;
-          const float v = slot_v[(2 * w + sl) * D + j];
-          if (k == open) {
-            a += v;
-          } else {
-            if (open >= 0) flush(open, a);
-            open = k;
-            a = v;
-          }
+  const int64_t c = blockIdx.x;
+  const int64_t p0 = c * P;
+  const int64_t p1 = p0 + P < n ? p0 + P : n;
+  const int64_t Lw = P / W;
+  const int64_t q0 = p0 + warp * Lw < p1 ? p0 + warp * Lw : p1;
+  const int64_t q1 = q0 + Lw < p1 ? q0 + Lw : p1;
+  warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, pairs, n, q0, q1, lane, slot_k + 2 * warp,
+                                   slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
+                                     store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc,
+                                                          1.f);
+                                   });
+  __syncthreads();
+  // Ordered combine of the cut runs, one thread per column.
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+    int open = -1;
+    float a = 0.f;
+    auto flush = [&](int k, float v) {
+      const int64_t s0 = start[k], s1 = start[k + 1];
+      if (s0 >= p0 && s1 <= p1) sums[static_cast<int64_t>(k) * D + j] = v;
+      else if (s0 < p0) pl[c * D + j] = v;
+      else pr[c * D + j] = v;
+    };
+    for (int w = 0; w < W; ++w) {
+      for (int sl = 0; sl < 2; ++sl) {
+        const int k = slot_k[2 * w + sl];
+        if (k < 0) continue;
+        const float v = slot_v[(2 * w + sl) * D + j];
+        if (k == open) {
+          a += v;
+        } else {
+          if (open >= 0) flush(open, a);
+          open = k;
+          a = v;
         }
       }
-      if (open >= 0) flush(open, a);
     }
-    __syncthreads();
+    if (open >= 0) flush(open, a);
   }
 }
 
 template <int LPR>
 static cudaError_t launch_segsum_t(const Plan& p, const SegArgs& a, cudaStream_t s) {
   const int row_bytes = p.D * p.es;
-  const int64_t nch = (a.n + p.gc.BNS - 1) / p.gc.BNS;
+  const int64_t P = seg_block_positions(a.n);
+  const int64_t nch = (a.n + P - 1) / P;
   const size_t sm = (2 * 8 + 2 * 8 * static_cast<size_t>(p.D)) * 4;
-  int dev = 0, nsm = 0, occ = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   count_launch();
-  if (p.dtype == kDtypeBF16) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_segsum<LPR, true>, 256, sm);
-    const int64_t grid = nch < static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1) ? nch : static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1);
-    k_segsum<LPR, true><<<static_cast<unsigned>(grid), 256, sm, s>>>(
-        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.skeys, a.start, p.gc.L, nch, a.sums,
-        a.pl, a.pr);
-  } else {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_segsum<LPR, false>, 256, sm);
-    const int64_t grid = nch < static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1) ? nch : static_cast<int64_t>(nsm) * (occ > 0 ? occ : 1);
-    k_segsum<LPR, false><<<static_cast<unsigned>(grid), 256, sm, s>>>(
-        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.perm, a.skeys, a.start, p.gc.L, nch, a.sums,
-        a.pl, a.pr);
-  }
+  if (p.dtype == kDtypeBF16)
+    k_segsum<LPR, true><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
+                                                                    row_bytes, a.pairs, a.start, P, a.sums, a.pl,
+                                                                    a.pr);
+  else
+    k_segsum<LPR, false><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
+                                                                     row_bytes, a.pairs, a.start, P, a.sums, a.pl,
+                                                                     a.pr);
   return cudaGetLastError();
 }
 
@@ -343,24 +332,79 @@ __device__ __forceinline__ void* op_row(const FinK& f, int k) {
   return reinterpret_cast<float*>(f.c_op) + static_cast<int64_t>(k) * 3 * f.Dp;
 }
 
-// Finalise cluster k given its summed row in `srow` (shared or global), run
-// by one warp: centroid = sum / count (or keep), operand copy, norm, counts.
-__device__ void finish_cluster(const FinK& f, int k, int64_t cnt, const float* srow, int lane) {
+// Operand row (-2c in bf16, or the TF32 split) and ||c||^2 of a centroid held
+// in registers: v[i] = c[lane + 32 i] (D <= 256).
+__device__ __forceinline__ float emit_operand_regs(const float (&v)[8], int D, int Dp, int dtype, void* row,
+                                                   int lane) {
+  float s = 0.f;
+  if (dtype == kDtypeBF16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(row);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = lane + 32 * i;
+      if (j < D) {
+        const float f = __bfloat162float(__float2bfloat16_rn(v[i]));
+        if (o) o[j] = __float2bfloat16_rn(-2.f * f);
+        s = fmaf(f, f, s);
+      }
+    }
+  } else {
+    float* o = reinterpret_cast<float*>(row);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int j = lane + 32 * i;
+      if (j < Dp) {
+        const float val = j < D ? v[i] : 0.f;
+        if (o) {
+          const float hi = tf32_round(val);
+          const float lo = tf32_round(val - hi);
+          o[j] = -2.f * hi;
+          o[Dp + j] = -2.f * lo;
+          o[2 * Dp + j] = -2.f * hi;
+        }
+        s = fmaf(val, val, s);
+      }
+    }
+  }
+  return warp_sum_f(s);
+}
+
+// Finalise cluster k, run by one warp.  sum[i] holds the member sum of column
+// lane + 32 i (ignored when cnt == 0).  Mode 0: centroid = sum / count (or
+// keep the previous one), operand copy, augmentation row, count.  Mode 1:
+// add the sum and count to the float64 accumulators.
+__device__ void finish_cluster(const FinK& f, int k, int64_t cnt, float (&sum)[8], int lane) {
   float* crow = f.C + static_cast<int64_t>(k) * f.D;
   if (f.mode == 0) {
     if (cnt > 0) {
       const float fc = static_cast<float>(cnt);
-      for (int j = lane; j < f.D; j += 32) crow[j] = srow[j] / fc;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = lane + 32 * i;
+        if (j < f.D) {
+          sum[i] = sum[i] / fc;
+          crow[j] = sum[i];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = lane + 32 * i;
+        sum[i] = j < f.D ? crow[j] : 0.f;
+      }
     }
-    __syncwarp();
-    const float s = emit_operand_row([&](int j) { return crow[j]; }, f.D, f.Dp, f.dtype, op_row(f, k), lane);
+    const float s = emit_operand_regs(sum, f.D, f.Dp, f.dtype, op_row(f, k), lane);
     if (lane == 0) {
       if (f.caug) write_aug_row(f.caug + static_cast<int64_t>(k) * kAugBytes, f.dtype, s, 1);
       if (f.counts) f.counts[k] = static_cast<int32_t>(cnt);
     }
   } else if (cnt > 0) {
     double* arow = f.acc64 + static_cast<int64_t>(k) * f.D;
-    for (int j = lane; j < f.D; j += 32) arow[j] += static_cast<double>(srow[j]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = lane + 32 * i;
+      if (j < f.D) arow[j] += static_cast<double>(sum[i]);
+    }
     if (lane == 0) f.cnt64[k] += cnt;
   }
 }
@@ -369,7 +413,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
   extern __shared__ float fsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && f.ntiles > 0) {
-    // objective of this pass: fixed-order reduction of the tile partials
+    // objective of this pass: fixed-order reduction of the assign partials
     double* red = reinterpret_cast<double*>(fsm);
     double s = 0.0;
     for (int64_t i = threadIdx.x; i < f.ntiles * 4; i += blockDim.x) s += f.tobj[i];
@@ -389,24 +433,29 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
     const int k = static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + warp;
     if (k >= f.K) return;
     const int64_t s0 = f.start[k], s1 = f.start[k + 1], cnt = s1 - s0;
+    float v[8];
     if (cnt > 0) {
       const int64_t ca = s0 / f.BNS, cb = (s1 - 1) / f.BNS;
       if (cb - ca > f.big_span) return;  // handled by a whole block below
-      float* srow = fsm + (f.ntiles > 0 && blockIdx.x == 0 ? 1024 : 0) + warp * f.D;
-      if (ca == cb) {
-        for (int j = lane; j < f.D; j += 32) srow[j] = f.sums[static_cast<int64_t>(k) * f.D + j];
-      } else {
-        for (int j = lane; j < f.D; j += 32) {
-          float a = f.pr[ca * f.D + j];
-          for (int64_t c = ca + 1; c <= cb; ++c) a += f.pl[c * f.D + j];
-          srow[j] = a;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = lane + 32 * i;
+        v[i] = 0.f;
+        if (j < f.D) {
+          if (ca == cb) {
+            v[i] = f.sums[static_cast<int64_t>(k) * f.D + j];
+          } else {
+            float a = f.pr[ca * f.D + j];
+            for (int64_t c = ca + 1; c <= cb; ++c) a += f.pl[c * f.D + j];
+            v[i] = a;
+          }
         }
       }
-      __syncwarp();
-      finish_cluster(f, k, cnt, srow, lane);
     } else {
-      finish_cluster(f, k, 0, nullptr, lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
     }
+    finish_cluster(f, k, cnt, v, lane);
     return;
   }
   // Big clusters: block i owns the cluster containing position i*G (G =
@@ -445,7 +494,15 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
     srow[j] = a;
   }
   __syncthreads();
-  if (warp == 0) finish_cluster(f, k, s1 - s0, srow, lane);
+  if (warp == 0) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = lane + 32 * i;
+      v[i] = j < f.D ? srow[j] : 0.f;
+    }
+    finish_cluster(f, k, s1 - s0, v, lane);
+  }
 }
 
 cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s) {
@@ -454,7 +511,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.D = p.D;
   f.Dp = p.Dp;
   f.dtype = p.dtype;
-  f.BNS = p.gc.BNS;
+  f.BNS = static_cast<int>(seg_block_positions(p.rows));
   f.big_span = p.gc.big_span;
   f.n = p.rows;
   f.start = a.start;
@@ -473,7 +530,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.obj = a.obj;
   const int threads = 512;
   f.nwarp_blocks = (p.K + 15) / 16;
-  const int64_t G = static_cast<int64_t>(p.gc.big_span) * p.gc.BNS;
+  const int64_t G = static_cast<int64_t>(p.gc.big_span) * f.BNS;
   const int64_t nbig = (p.rows + G - 1) / G;
   // block 0: 512 doubles of objective reduction (1024 floats) + 16 warp rows;
   // big-cluster blocks: slices x D partial rows + one summed row.

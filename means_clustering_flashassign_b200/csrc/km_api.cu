@@ -218,9 +218,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   sc.nblk = (p.rows + sc.T - 1) / sc.T;
   sc.Rmax = 1 << (sc.bits[0] > sc.bits[1] ? sc.bits[0] : sc.bits[1]);
   SegCfg& gc = p.gc;
-  gc.W = 8;
-  gc.L = p.rows >= int64_t(148) * 8 * 2048 ? 256 : 128;
-  gc.BNS = gc.W * gc.L;
+  gc.BNS = static_cast<int>(seg_block_positions(p.rows));
   gc.nchunks = (p.rows + gc.BNS - 1) / gc.BNS;
   gc.big_span = 8;
   // ---- workspace layout
@@ -235,12 +233,9 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   if (op == KM_OP_ARGSORT) {
     p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
-    if (sc.passes > 1) {
-      p.off_keys = take(sizeof(int32_t) * p.rows);
-      p.off_vals = take(sizeof(int32_t) * p.rows);
-    }
+    if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
+    p.off_pairs = take(sizeof(int2) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));
-    p.off_skeys = take(sizeof(int32_t) * p.rows);
     p.total = off;
     return KM_OK;
   }
@@ -254,12 +249,8 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   if (op != KM_OP_ASSIGN && !p.small_update) {
     p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
-    if (sc.passes > 1) {
-      p.off_keys = take(sizeof(int32_t) * p.rows);
-      p.off_vals = take(sizeof(int32_t) * p.rows);
-    }
-    p.off_perm = take(sizeof(int32_t) * p.rows);
-    p.off_skeys = take(sizeof(int32_t) * p.rows);
+    if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
+    p.off_pairs = take(sizeof(int2) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));
     p.off_sums = take(sizeof(float) * static_cast<size_t>(K) * D);
     p.off_pl = take(sizeof(float) * gc.nchunks * D);
@@ -312,13 +303,12 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
               p.K,
               at<int32_t>(c.ws, p.off_blkhist),
               at<int32_t>(c.ws, p.off_total),
-              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
-              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
-              at<int32_t>(c.ws, p.off_perm),
-              at<int32_t>(c.ws, p.off_start),
-              at<int32_t>(c.ws, p.off_skeys)};
+              p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
+              at<int2>(c.ws, p.off_pairs),
+              nullptr,
+              at<int32_t>(c.ws, p.off_start)};
   KM_CUDA(launch_sort(p, sa, c.s));
-  SegArgs ga{Xb, n, sa.perm, sa.start, sa.skeys, at<float>(c.ws, p.off_sums), at<float>(c.ws, p.off_pl),
+  SegArgs ga{Xb, n, sa.pairs, sa.start, at<float>(c.ws, p.off_sums), at<float>(c.ws, p.off_pl),
              at<float>(c.ws, p.off_pr)};
   KM_CUDA(launch_segsum(p, ga, c.s));
   FinalizeArgs fa{};
@@ -654,11 +644,10 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               K,
               at<int32_t>(c.ws, p.off_blkhist),
               at<int32_t>(c.ws, p.off_total),
-              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_keys) : nullptr,
-              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_vals) : nullptr,
+              p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
+              at<int2>(c.ws, p.off_pairs),
               perm,
-              start ? start : at<int32_t>(c.ws, p.off_start),
-              at<int32_t>(c.ws, p.off_skeys)};
+              start ? start : at<int32_t>(c.ws, p.off_start)};
   KM_CUDA(launch_sort(p, sa, c.s));
   return KM_OK;
 }

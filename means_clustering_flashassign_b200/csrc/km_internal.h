@@ -50,13 +50,19 @@ struct SortCfg {
 };
 
 struct SegCfg {
-  int W = 8;          // warps per block
-  int L = 0;          // sorted positions per warp
-  int BNS = 0;        // sorted positions per block (W * L)
+  int BNS = 0;        // sorted positions per segmented-sum block (seg_block_positions)
   int64_t nchunks = 0;
   int big_span = 8;   // clusters spanning more chunks than this use a whole block in finalize
-  int64_t nbig = 0;   // finalize blocks reserved for such clusters
 };
+
+// Sorted positions per segmented-sum block for n positions: the blocks form
+// one wave (148 SMs x 4 resident blocks), each a multiple of 256 positions.
+constexpr int64_t kSegWaveBlocks = 148 * 4;
+inline int64_t seg_block_positions(int64_t n) {
+  int64_t p = (n + kSegWaveBlocks - 1) / kSegWaveBlocks;
+  p = (p + 255) / 256 * 256;
+  return p < 256 ? 256 : p;
+}
 
 struct Plan {
   int op = 0, B = 1, D = 0, K = 0, dtype = 0;
@@ -74,7 +80,7 @@ struct Plan {
   SegCfg gc;
   // workspace offsets (bytes)
   size_t off_hdr = 0, off_xaug = 0, off_caug = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
-  size_t off_blkhist = 0, off_total = 0, off_keys = 0, off_vals = 0, off_perm = 0, off_start = 0, off_skeys = 0;
+  size_t off_blkhist = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
   size_t total = 0;
@@ -128,16 +134,15 @@ cudaError_t launch_objective(const double* tobj, int B, int64_t groups_per_inst,
 // Stable LSD radix sort of one instance's assignment vector; writes perm and
 // start[K+1] (start[k] = first sorted position of cluster k).
 struct SortArgs {
-  const int32_t* keys;
+  const int32_t* keys;  // the assignment vector
   int64_t n;
   int K;
-  int32_t* blkhist;
-  int32_t* total;
-  int32_t* keys_tmp;
-  int32_t* vals_tmp;
-  int32_t* perm;
-  int32_t* start;
-  int32_t* skeys;  // [n] sorted keys (cluster id of each sorted position)
+  int32_t* blkhist;     // [nblk][Rmax]
+  int32_t* total;       // [Rmax]
+  int2* pairs_tmp;      // [n] (two-pass sorts only)
+  int2* pairs;          // [n] sorted (point index, cluster id)
+  int32_t* perm;        // [n] sorted point indices, or null
+  int32_t* start;       // [K+1]
 };
 cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s);
 
@@ -146,9 +151,8 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s);
 struct SegArgs {
   const void* X;
   int64_t n;
-  const int32_t* perm;
+  const int2* pairs;      // sorted (point index, cluster id)
   const int32_t* start;
-  const int32_t* skeys;
   float* sums;  // [K][D]
   float* pl;    // [nchunks][D]
   float* pr;    // [nchunks][D]
