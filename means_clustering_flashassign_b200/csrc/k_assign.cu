@@ -50,6 +50,8 @@ struct AssignK {
   double* tobj;
   int obj_per_cta;  // 1: tobj[cta][4] sums over the CTA's tiles in order; 0: tobj[tile][4]
   uint32_t zero;    // always 0; keeps the epilogue's column constants in registers
+  int32_t* hist0;   // may be null: sort pass-0 block digit counts, [row / hist_T][digit]
+  int hist_T, hist_R;
   unsigned int* status;
   uint64_t limit_ns;
 };
@@ -359,6 +361,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           md = fmaxf(0.f, best);
           p.idx[o] = bk;
           if (p.mindist) p.mindist[o] = md;
+          if (p.hist0) atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + (bk & (p.hist_R - 1)), 1);
         }
         double ds = static_cast<double>(md);
 #pragma unroll
@@ -396,6 +399,9 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.tobj = a.tobj;
   k.obj_per_cta = a.B == 1 ? 1 : 0;
   k.zero = 0;
+  k.hist0 = a.B == 1 ? a.hist0 : nullptr;
+  k.hist_T = a.hist_T;
+  k.hist_R = a.hist_R;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN>(k.natoms, k.XB, k.CS);

@@ -141,7 +141,7 @@ __device__ void block_exclusive_scan(const int32_t* total, int R, int32_t* base,
 // element, and optionally the bare point index (perm_out) on the last pass.
 template <int IPT, bool PAIRS>
 __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n,
-                               int T, int shift, int R, const int32_t* __restrict__ blkhist,
+                               int T, int shift, int R, int32_t* __restrict__ blkhist,
                                const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
                                int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
   extern __shared__ int32_t sh[];
@@ -202,7 +202,7 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
   }
   __syncthreads();
   block_exclusive_scan(lstart, R, lstart, tmp);
-  const int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
   for (int d = threadIdx.x; d < R; d += blockDim.x) {
     int32_t run = lstart[d];
     for (int w = 0; w < W; ++w) {
@@ -211,6 +211,7 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
       run += c;
     }
     base[d] += boff[d] - lstart[d];  // global position = base[d] + local position
+    boff[d] = 0;  // leave the counts zeroed for the next accumulation
   }
   __syncthreads();
 #pragma unroll
@@ -221,7 +222,10 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
   const int nvalid = static_cast<int>((n - t0) < T ? (n - t0) : T);
   for (int i = threadIdx.x; i < nvalid; i += blockDim.x) {
     const int2 pk = stage[i];
-    const int32_t pos = base[(pk.y >> shift) & (R - 1)] + i;
+    const int64_t pos = static_cast<int64_t>(base[(pk.y >> shift) & (R - 1)]) + i;
+    // Counts accumulated elsewhere (the assignment kernel) agree with these
+    // keys unless that kernel gave up on a bounded wait; stay in bounds then.
+    if (pos < 0 || pos >= n) continue;
     pairs_out[pos] = pk;
     if (perm_out) perm_out[pos] = pk.x;
   }
@@ -250,14 +254,15 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     const int R = 1 << c.bits[ps];
     const bool last = ps == c.passes - 1;
     const bool pairs_in = ps > 0;
-    count_launch(3);  // hist, colscan, scatter
+    int32_t* bh = ps == 0 ? a.blkhist : a.blkhist1;
+    count_launch(ps == 0 && a.hist0_ready ? 2 : 3);  // [hist,] colscan, scatter
     if (pairs_in)
       k_sort_hist<true><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps],
-                                                                        R, a.blkhist, a.K);
-    else
+                                                                        R, bh, a.K);
+    else if (!a.hist0_ready)
       k_sort_hist<false><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(a.keys, nullptr, a.n, c.T, c.shift[ps], R,
-                                                                         a.blkhist, a.K);
-    k_sort_colscan<<<(R + 31) / 32, 256, 0, s>>>(a.blkhist, R, nblk, a.total);
+                                                                         bh, a.K);
+    k_sort_colscan<<<(R + 31) / 32, 256, 0, s>>>(bh, R, nblk, a.total);
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
     int2* out = last ? a.pairs : a.pairs_tmp;
@@ -270,13 +275,13 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
                                static_cast<int>(sm));
       if (e != cudaSuccess) return e;
       k_sort_scatter<16, true><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
-          nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps], R, a.blkhist, a.total, out, perm, st, a.K);
+          nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps], R, bh, a.total, out, perm, st, a.K);
     } else {
       e = cudaFuncSetAttribute(k_sort_scatter<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sm));
       if (e != cudaSuccess) return e;
       k_sort_scatter<16, false><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
-          a.keys, nullptr, a.n, c.T, c.shift[ps], R, a.blkhist, a.total, out, perm, st, a.K);
+          a.keys, nullptr, a.n, c.T, c.shift[ps], R, bh, a.total, out, perm, st, a.K);
     }
   }
   if (c.passes > 1) {

@@ -140,8 +140,12 @@ __device__ __forceinline__ void warp_range_sums(const uint8_t* X, int row_bytes,
 // `final_store(k, acc)`; a run continuing past the left edge goes to slot 0,
 // one continuing only past the right edge to slot 1 (cluster ids in slot_k,
 // -1 when unused, vectors in slot_v[2][D]).
+__device__ __forceinline__ int clamp_id(int v, int64_t hi) {
+  return v < 0 ? 0 : (v >= hi ? static_cast<int>(hi - 1) : v);
+}
+
 template <int LPR, bool BF16, class FinalStore>
-__device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D,
+__device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D, int K,
                                                       const int2* __restrict__ pairs, int64_t n, int64_t q0,
                                                       int64_t q1, int lane, int* slot_k, float* slot_v,
                                                       FinalStore final_store) {
@@ -151,10 +155,11 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
   const int sub = lane / LPR;
   const int cl = lane % LPR;
   const bool active = cl * 16 < row_bytes;
-  const int kfirst = pairs[q0].y;
-  const bool left_cont = q0 > 0 && pairs[q0 - 1].y == kfirst;
-  const int klast = pairs[q1 - 1].y;
-  const bool right_cont = q1 < n && pairs[q1].y == klast;
+  // ids are clamped (memory safety only: valid pairs are always in range)
+  const int kfirst = clamp_id(pairs[q0].y, K);
+  const bool left_cont = q0 > 0 && clamp_id(pairs[q0 - 1].y, K) == kfirst;
+  const int klast = clamp_id(pairs[q1 - 1].y, K);
+  const bool right_cont = q1 < n && clamp_id(pairs[q1].y, K) == klast;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -178,7 +183,9 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
   const bool in_batch = lane < G::BATCH;
   int2 pv = (in_batch && q0 + lane < q1) ? pairs[q0 + lane] : make_int2(-1, -1);
   for (int64_t p = q0; p < q1; p += G::BATCH) {
-    const int cur_p = pv.x, cur_k = pv.y;
+    // ids are clamped into range: memory safety if an aborted kernel left
+    // the pairs incomplete (no effect on valid input)
+    const int cur_p = clamp_id(pv.x, n), cur_k = pv.y < 0 ? -1 : clamp_id(pv.y, K);
     const int64_t pn = p + G::BATCH;
     pv = (in_batch && pn + lane < q1) ? pairs[pn + lane] : make_int2(-1, -1);
     const int nb = q1 - p < G::BATCH ? static_cast<int>(q1 - p) : G::BATCH;
@@ -220,7 +227,7 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
 // to pl[c], one continuing only past its right edge to pr[c].
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X, int64_t n, int D, int row_bytes,
-                                                   const int2* __restrict__ pairs,
+                                                   const int2* __restrict__ pairs, int K,
                                                    const int32_t* __restrict__ start, int64_t P,
                                                    float* __restrict__ sums, float* __restrict__ pl,
                                                    float* __restrict__ pr) {
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X
   const int64_t Lw = P / W;
   const int64_t q0 = p0 + warp * Lw < p1 ? p0 + warp * Lw : p1;
   const int64_t q1 = q0 + Lw < p1 ? q0 + Lw : p1;
-  warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, pairs, n, q0, q1, lane, slot_k + 2 * warp,
+  warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, K, pairs, n, q0, q1, lane, slot_k + 2 * warp,
                                    slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
                                      store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc,
                                                           1.f);
@@ -278,12 +285,12 @@ static cudaError_t launch_segsum_t(const Plan& p, const SegArgs& a, cudaStream_t
   count_launch();
   if (p.dtype == kDtypeBF16)
     k_segsum<LPR, true><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
-                                                                    row_bytes, a.pairs, a.start, P, a.sums, a.pl,
-                                                                    a.pr);
+                                                                    row_bytes, a.pairs, p.K, a.start, P, a.sums,
+                                                                    a.pl, a.pr);
   else
     k_segsum<LPR, false><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
-                                                                     row_bytes, a.pairs, a.start, P, a.sums, a.pl,
-                                                                     a.pr);
+                                                                     row_bytes, a.pairs, p.K, a.start, P, a.sums,
+                                                                     a.pl, a.pr);
   return cudaGetLastError();
 }
 
@@ -311,6 +318,7 @@ struct FinK {
   int K, D, Dp, dtype, BNS, big_span;
   int64_t n, nwarp_blocks;
   const int32_t* start;
+  const int2* pairs;
   const float* sums;
   const float* pl;
   const float* pr;
@@ -463,7 +471,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
   const int64_t G = static_cast<int64_t>(f.big_span) * f.BNS;
   const int64_t P = (static_cast<int64_t>(blockIdx.x) - f.nwarp_blocks) * G;
   if (P >= f.n) return;
-  const int k = find_cluster(f.start, f.K, P);
+  const int k = clamp_id(f.pairs[P].y, f.K);
   const int64_t s0 = f.start[k], s1 = f.start[k + 1];
   const int64_t ca = s0 / f.BNS, cb = (s1 - 1) / f.BNS;
   if (cb - ca <= f.big_span) return;
@@ -515,6 +523,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.big_span = p.gc.big_span;
   f.n = p.rows;
   f.start = a.start;
+  f.pairs = a.pairs;
   f.sums = a.sums;
   f.pl = a.pl;
   f.pr = a.pr;

@@ -231,7 +231,8 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   const int64_t BR = static_cast<int64_t>(B) * p.rows;
   p.off_hdr = take(kAlign);
   if (op == KM_OP_ARGSORT) {
-    p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
+    p.off_blkhist = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[0]) * sc.nblk);
+    if (sc.passes > 1) p.off_blkhist1 = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[1]) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
     if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
     p.off_pairs = take(sizeof(int2) * p.rows);
@@ -247,7 +248,8 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   if (op == KM_OP_FIT || op == KM_OP_FIT_HOST) p.off_idx = take(sizeof(int32_t) * BR);
   p.off_obj = take(sizeof(double) * (op == KM_OP_FIT_HOST ? kMaxHostIters : B));
   if (op != KM_OP_ASSIGN && !p.small_update) {
-    p.off_blkhist = take(sizeof(int32_t) * static_cast<size_t>(sc.Rmax) * sc.nblk);
+    p.off_blkhist = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[0]) * sc.nblk);
+    if (sc.passes > 1) p.off_blkhist1 = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[1]) * sc.nblk);
     p.off_total = take(sizeof(int32_t) * sc.Rmax);
     if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
     p.off_pairs = take(sizeof(int2) * p.rows);
@@ -296,12 +298,15 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
-                    int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode) {
+                    int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
+                    bool hist0_ready = false) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
               p.K,
               at<int32_t>(c.ws, p.off_blkhist),
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
+              hist0_ready,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),
@@ -313,6 +318,7 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
   KM_CUDA(launch_segsum(p, ga, c.s));
   FinalizeArgs fa{};
   fa.start = sa.start;
+  fa.pairs = sa.pairs;
   fa.sums = ga.sums;
   fa.pl = ga.pl;
   fa.pr = ga.pr;
@@ -462,10 +468,16 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
+  // Single-instance fits let the assignment kernel count the sort's first
+  // digit per block; the sort's scatter zeroes the counts again after use.
+  const bool fused_hist = B == 1 && !p.small_update;
+  int32_t* hist0 = fused_hist ? at<int32_t>(c.ws, p.off_blkhist) : nullptr;
+  if (fused_hist)
+    KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
-                 &groups};
+                 &groups, hist0, p.sc.T, 1 << p.sc.bits[0]};
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t], c.s));
     KM_CUDA(launch_assign(p, a, c.s));
     if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
@@ -480,7 +492,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
                             C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
                             caug + static_cast<int64_t>(b) * p.Kp * 32,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
-                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0);
+                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, fused_hist);
         if (r != KM_OK) return r;
       }
     }
@@ -579,6 +591,8 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
     KM_CUDA(cudaMemsetAsync(cnt64, 0, sizeof(long long) * K, c.s));
     KM_CUDA(cudaMemsetAsync(objacc, 0, sizeof(double), c.s));
     KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
+    int32_t* hist0 = at<int32_t>(c.ws, p.off_blkhist);
+    KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
     for (int i = 0; i < 2; ++i) KM_CUDA(cudaEventRecord(ev_free[i], c.s));
     const bool f32 = dtype == KM_F32;
     CUtensorMap cmap, camap;
@@ -609,12 +623,14 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         pc.tiles_per_inst = (nr + kTileM - 1) / kTileM;
         pc.ntiles = pc.tiles_per_inst;
         int64_t groups = 0;
-        AssignArgs a{&xmap, &xamap, &cmap, &camap, 1, nr, K, p.Kp, idxc, nullptr, tobj, c.status(),
-                     wait_limit_ns(), &groups};
+        AssignArgs a{&xmap, &xamap, &cmap, &camap, 1,       nr,      K,           p.Kp,
+                     idxc,  nullptr, tobj,  c.status(), wait_limit_ns(), &groups, hist0, p.sc.T,
+                     1 << p.sc.bits[0]};
         KM_CUDA(launch_assign(pc, a, c.s));
         Ctx cc = c;
         cc.p = pc;
-        rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1);
+        rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1,
+                             true);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
       }
@@ -643,6 +659,8 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               N,
               K,
               at<int32_t>(c.ws, p.off_blkhist),
+              p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
+              false,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),

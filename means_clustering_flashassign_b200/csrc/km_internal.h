@@ -80,7 +80,7 @@ struct Plan {
   SegCfg gc;
   // workspace offsets (bytes)
   size_t off_hdr = 0, off_xaug = 0, off_caug = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
-  size_t off_blkhist = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
+  size_t off_blkhist = 0, off_blkhist1 = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
   size_t total = 0;
@@ -123,6 +123,8 @@ struct AssignArgs {
   unsigned int* status;
   uint64_t limit_ns;
   int64_t* obj_groups;  // host out (may be null): 4-double groups of partials per instance
+  int32_t* hist0;       // may be null: pass-0 block digit counts to accumulate (B == 1 only)
+  int hist_T, hist_R;   // keys per sort block, pass-0 radix
 };
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s);
 
@@ -137,7 +139,9 @@ struct SortArgs {
   const int32_t* keys;  // the assignment vector
   int64_t n;
   int K;
-  int32_t* blkhist;     // [nblk][Rmax]
+  int32_t* blkhist;     // [nblk][R0] pass-0 block digit counts (zeroed again by the pass-0 scatter)
+  int32_t* blkhist1;    // [nblk][R1] pass-1 block digit counts (two-pass sorts only)
+  bool hist0_ready;     // pass-0 counts were accumulated by the assignment kernel
   int32_t* total;       // [Rmax]
   int2* pairs_tmp;      // [n] (two-pass sorts only)
   int2* pairs;          // [n] sorted (point index, cluster id)
@@ -161,6 +165,7 @@ cudaError_t launch_segsum(const Plan& p, const SegArgs& a, cudaStream_t s);
 
 struct FinalizeArgs {
   const int32_t* start;
+  const int2* pairs;  // sorted (point, cluster) pairs
   const float* sums;
   const float* pl;
   const float* pr;
