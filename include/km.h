@@ -46,6 +46,12 @@
  *    calling thread.
  *  - Calls on distinct workspaces may run concurrently; calls sharing one
  *    workspace must be ordered (same stream or synchronised).
+ *  - Environment (read once per process): KM_WAIT_LIMIT_NS sets the bound of
+ *    every in-kernel wait (default 2e9 ns); KM_ASSIGN_FORM=single|pair picks
+ *    the assignment kernel's form: one CTA per 128-point tile (the default)
+ *    or two-SM CTA pairs on 256-point tiles.  Both forms meet the same
+ *    accuracy rules; the objective's float64 summation order follows the
+ *    form's tiling, so its last bits may differ between forms.
  */
 #ifndef KM_H_
 #define KM_H_

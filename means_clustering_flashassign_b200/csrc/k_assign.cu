@@ -31,6 +31,12 @@
 //   warps 2..17  epilogue: 4 warps per TMEM lane quarter, each owning a
 //                quarter of the BN columns; tcgen05.ld, key, min tree; the
 //                four column quarters merge at the end of the point tile.
+// Pair variant (PAIR=true): two CTAs of a cluster on an SM pair cooperate on
+// 256-point tiles with cta_group::2 UMMAs (M=256): each CTA holds its 128
+// points and half of every centroid tile, the lead CTA issues the MMAs, and
+// each CTA's TMEM receives the distances of its own 128 points for the whole
+// centroid tile.  Per SM this halves the centroid bytes streamed from L2 and
+// read from shared memory, which leaves room for 4 centroid stages.
 // Every wait is an mbarrier wait bounded in time (see km_ptx.cuh).
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -44,7 +50,8 @@ struct AssignK {
   int B;
   int64_t rows;
   int K, Kp, natoms, XB, CS, nct;
-  int64_t tiles_per_inst, ntiles;
+  int64_t tiles_per_inst, ntiles;  // tiles of TM points (256 for pairs, else 128)
+  int64_t tiles128_per_inst;       // 128-point tiles per instance (per-tile objective layout)
   int32_t* idx;
   float* mindist;
   double* tobj;
@@ -64,13 +71,14 @@ constexpr int kEpiWarps = 16;
 __host__ __device__ constexpr size_t x_buf_bytes(int natoms) {
   return static_cast<size_t>(natoms) * kXAtomBytes + kTileM * kAugRowBytes;
 }
-__host__ __device__ constexpr size_t c_stage_bytes(int natoms, int BN) {
-  return static_cast<size_t>(natoms) * BN * kAtomBytesPerRow + static_cast<size_t>(BN) * kAugRowBytes;
+__host__ __device__ constexpr size_t c_stage_bytes(int natoms, int rows) {
+  return static_cast<size_t>(natoms) * rows * kAtomBytesPerRow + static_cast<size_t>(rows) * kAugRowBytes;
 }
 
-template <int BN>
+// BN centroids per MMA; a CTA of a pair holds BN/2 of them per stage.
+template <int BN, bool PAIR>
 __host__ __device__ constexpr size_t assign_smem_bytes(int natoms, int XB, int CS) {
-  return 1024 /* alignment slack */ + XB * x_buf_bytes(natoms) + CS * c_stage_bytes(natoms, BN) +
+  return 1024 /* alignment slack */ + XB * x_buf_bytes(natoms) + CS * c_stage_bytes(natoms, PAIR ? BN / 2 : BN) +
          3 * kTileM * 8 /* merge slots */ + 32 * 8 /* barriers */ + 16;
 }
 
@@ -145,15 +153,21 @@ __device__ __forceinline__ uint32_t chunk_min_key(const float (&v)[CW], const ui
   return __float_as_uint(m);
 }
 
-template <int BN, bool TF32>
+template <int BN, bool TF32, bool PAIR>
 __global__ void __launch_bounds__(kAssignThreads, 1)
     k_assign(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap xamap,
              const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap camap, const AssignK p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int HB = PAIR ? BN / 2 : BN;       // centroid rows of a stage held by this CTA
+  constexpr int TM = PAIR ? 2 * kTileM : kTileM;  // points per tile of the (pair of) CTA(s)
   const int natoms = p.natoms;
   const int XB = p.XB, CS = p.CS;
-  const size_t xbb = x_buf_bytes(natoms), csb = c_stage_bytes(natoms, BN);
+  const size_t xbb = x_buf_bytes(natoms), csb = c_stage_bytes(natoms, HB);
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int64_t unit = PAIR ? blockIdx.x / 2 : blockIdx.x;     // this CTA's (pair's) index
+  const int64_t nunits = PAIR ? gridDim.x / 2 : gridDim.x;
   uint8_t* xs = base;
   uint8_t* cs = xs + XB * xbb;
   float* mval = reinterpret_cast<float*>(cs + CS * csb);  // [3][128]
@@ -184,7 +198,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], kEpiWarps);
+      mbar_init(&a_empty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);  // both CTAs' epilogues release the lead's
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&c_full[i], 1);
@@ -198,11 +212,17 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_holder, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // peers' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitGuard g{p.status, abort_flag, p.limit_ns};
@@ -219,48 +239,70 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       uint32_t xph = 0, cph = 0;
       int x_iss[2] = {-1, -1}, c_iss[4] = {-1, -1, -1, -1};
       bool ok = true;
-      for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
+      // Loads of a pair complete on the lead CTA's barriers; only the lead
+      // posts the expected bytes (both CTAs' share).
+      auto load = [&](void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+        if constexpr (PAIR) tma_load_3d_pair(dst, map, x, y, z, mapa_shared(smem_addr(bar), 0));
+        else tma_load_3d(dst, map, x, y, z, bar);
+      };
+      for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
         const int b = static_cast<int>(t / p.tiles_per_inst);
         const int rt = static_cast<int>(t - static_cast<int64_t>(b) * p.tiles_per_inst);
+        const int row0 = rt * TM + static_cast<int>(rank) * kTileM;
         if (!mbar_wait(&x_empty[xb], xph ^ 1u, g)) { ok = false; break; }
         uint8_t* xdst = xs + xb * xbb;
-        mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>(xbb));
-        for (int a = 0; a < natoms; ++a)
-          tma_load_3d(xdst + a * kXAtomBytes, &xmap, a * kElem, rt * kTileM, b, &x_full[xb]);
-        tma_load_3d(xdst + natoms * kXAtomBytes, &xamap, 0, rt * kTileM, b, &x_full[xb]);
+        if (leader) mbar_arrive_expect_tx(&x_full[xb], static_cast<uint32_t>((PAIR ? 2 : 1) * xbb));
+        for (int a = 0; a < natoms; ++a) load(xdst + a * kXAtomBytes, &xmap, a * kElem, row0, b, &x_full[xb]);
+        load(xdst + natoms * kXAtomBytes, &xamap, 0, row0, b, &x_full[xb]);
         x_iss[xb] = static_cast<int>(xph);
         if (++xb == XB) { xb = 0; xph ^= 1u; }
         for (int j = 0; j < nct; ++j) {
           if (!mbar_wait(&c_empty[cst], cph ^ 1u, g)) { ok = false; break; }
           uint8_t* cdst = cs + cst * csb;
-          mbar_arrive_expect_tx(&c_full[cst], static_cast<uint32_t>(csb));
+          const int crow0 = j * BN + static_cast<int>(rank) * HB;
+          if (leader) mbar_arrive_expect_tx(&c_full[cst], static_cast<uint32_t>((PAIR ? 2 : 1) * csb));
           for (int a = 0; a < natoms; ++a)
-            tma_load_3d(cdst + static_cast<size_t>(a) * BN * kAtomBytesPerRow, &cmap, a * kElem, j * BN, b,
-                        &c_full[cst]);
-          tma_load_3d(cdst + static_cast<size_t>(natoms) * BN * kAtomBytesPerRow, &camap, 0, j * BN, b,
-                      &c_full[cst]);
+            load(cdst + static_cast<size_t>(a) * HB * kAtomBytesPerRow, &cmap, a * kElem, crow0, b, &c_full[cst]);
+          load(cdst + static_cast<size_t>(natoms) * HB * kAtomBytesPerRow, &camap, 0, crow0, b, &c_full[cst]);
           c_iss[cst] = static_cast<int>(cph);
           if (++cst == CS) { cst = 0; cph ^= 1u; }
         }
       }
       if (!ok) {
         // Let copies already in flight land before the CTA can exit.
-        WaitGuard g2 = g;
-        volatile int never = 0;
-        g2.abort_flag = &never;
-        for (int i = 0; i < XB; ++i) if (x_iss[i] >= 0) mbar_wait(&x_full[i], static_cast<uint32_t>(x_iss[i]), g2);
-        for (int i = 0; i < CS; ++i) if (c_iss[i] >= 0) mbar_wait(&c_full[i], static_cast<uint32_t>(c_iss[i]), g2);
+        if (PAIR && !leader) {
+          // this CTA's copies complete on the lead's barriers: give them time
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 200000) {
+          }
+        } else {
+          WaitGuard g2 = g;
+          volatile int never = 0;
+          g2.abort_flag = &never;
+          for (int i = 0; i < XB; ++i)
+            if (x_iss[i] >= 0) mbar_wait(&x_full[i], static_cast<uint32_t>(x_iss[i]), g2);
+          for (int i = 0; i < CS; ++i)
+            if (c_iss[i] >= 0) mbar_wait(&c_full[i], static_cast<uint32_t>(c_iss[i]), g2);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = umma_idesc(TF32, kTileM, BN);
+      constexpr uint32_t idesc = umma_idesc(TF32, TM, BN);
       constexpr int kSteps = 4;  // 32-byte K steps per 128-byte atom
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
+        if constexpr (PAIR) umma_ss_pair<TF32>(d, ad, bd, idesc, acc);
+        else umma_ss<TF32>(d, ad, bd, idesc, acc);
+      };
+      auto commit = [&](uint64_t* bar) {  // arrives on the barrier in every CTA of the pair
+        if constexpr (PAIR) umma_commit_pair(bar, 0x3);
+        else umma_commit(bar);
+      };
       int xb = 0, cst = 0, ab = 0;
       uint32_t xph = 0, cph = 0, aph = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
+      for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
         if (!mbar_wait(&x_full[xb], xph, g)) { ok = false; break; }
         const uint32_t xaddr = smem_addr(xs + xb * xbb);
         for (int j = 0; j < nct; ++j) {
@@ -273,23 +315,24 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 #pragma unroll
             for (int s = 0; s < kSteps; ++s) {
               const uint64_t ad = sw128_kmajor_desc(xaddr + a * kXAtomBytes + s * 32);
-              const uint64_t bd = sw128_kmajor_desc(caddr + a * BN * kAtomBytesPerRow + s * 32);
-              umma_ss<TF32>(dtm, ad, bd, idesc, (a | s) != 0 ? 1u : 0u);
+              const uint64_t bd = sw128_kmajor_desc(caddr + a * HB * kAtomBytesPerRow + s * 32);
+              mma(dtm, ad, bd, (a | s) != 0 ? 1u : 0u);
             }
           }
-          umma_ss<TF32>(dtm, sw32_kmajor_desc(xaddr + natoms * kXAtomBytes),
-                        sw32_kmajor_desc(caddr + natoms * BN * kAtomBytesPerRow), idesc, 1u);
-          umma_commit(&c_empty[cst]);
-          umma_commit(&a_full[ab]);
+          mma(dtm, sw32_kmajor_desc(xaddr + natoms * kXAtomBytes),
+              sw32_kmajor_desc(caddr + natoms * HB * kAtomBytesPerRow), 1u);
+          commit(&c_empty[cst]);
+          commit(&a_full[ab]);
           if (++cst == CS) { cst = 0; cph ^= 1u; }
           if (++ab == 2) { ab = 0; aph ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&x_empty[xb]);
+        commit(&x_empty[xb]);
         if (++xb == XB) { xb = 0; xph ^= 1u; }
       }
       // Wait for every MMA this thread issued before TMEM can be released.
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair(drain, 0x1);
+      else umma_commit(drain);
       WaitGuard g2 = g;
       volatile int never = 0;
       g2.abort_flag = &never;
@@ -310,10 +353,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 #pragma unroll
     for (int i = 0; i < CW; ++i) ci[i] = static_cast<uint32_t>(i) + p.zero;
     const uint32_t kmask = ~31u + p.zero;
-    for (int64_t t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x) {
+    const uint32_t a_empty_lead0 = PAIR ? mapa_shared(smem_addr(&a_empty[0]), 0) : 0u;
+    const uint32_t a_empty_lead1 = PAIR ? mapa_shared(smem_addr(&a_empty[1]), 0) : 0u;
+    for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
       const int b = static_cast<int>(t / p.tiles_per_inst);
       const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
-      const int64_t row = rt * kTileM + r_local;
+      const int64_t row = rt * TM + static_cast<int64_t>(rank) * kTileM + r_local;
       const bool valid = row < p.rows;
       float best = CUDART_INF_F;
       int bk = 0;
@@ -333,7 +378,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_empty[ab]);
+        if (lane == 0) {
+          if (PAIR && !leader) mbar_arrive_cluster(ab == 0 ? a_empty_lead0 : a_empty_lead1);
+          else mbar_arrive(&a_empty[ab]);
+        }
         if (++ab == 2) { ab = 0; aph ^= 1u; }
       }
       if (!ok) break;
@@ -366,8 +414,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         double ds = static_cast<double>(md);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-        if (p.obj_per_cta) cta_obj += ds;
-        else if (lane == 0 && p.tobj) p.tobj[t * 4 + q] = ds;
+        if (p.obj_per_cta) {
+          cta_obj += ds;
+        } else if (lane == 0 && p.tobj) {
+          // per 128-point tile of the instance
+          const int64_t tile128 = rt * (TM / kTileM) + rank;
+          if (tile128 * kTileM < p.rows) p.tobj[(static_cast<int64_t>(b) * p.tiles128_per_inst + tile128) * 4 + q] = ds;
+        }
       }
       mph ^= 1u;
     }
@@ -375,14 +428,17 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   }
 
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // the lead's MMAs no longer read this CTA's shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-template <int BN, bool TF32>
+template <int BN, bool TF32, bool PAIR>
 static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s) {
+  constexpr int TM = PAIR ? 2 * kTileM : kTileM;
   AssignK k{};
   k.B = a.B;
   k.rows = a.rows;
@@ -392,7 +448,8 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.XB = pl.ac.XB;
   k.CS = pl.ac.CS;
   k.nct = a.Kp / BN;
-  k.tiles_per_inst = (a.rows + kTileM - 1) / kTileM;
+  k.tiles_per_inst = (a.rows + TM - 1) / TM;
+  k.tiles128_per_inst = (a.rows + kTileM - 1) / kTileM;
   k.ntiles = k.tiles_per_inst * a.B;
   k.idx = a.idx;
   k.mindist = a.mindist;
@@ -404,36 +461,71 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.hist_R = a.hist_R;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
-  const size_t smem = assign_smem_bytes<BN>(k.natoms, k.XB, k.CS);
-  cudaError_t e = cudaFuncSetAttribute(k_assign<BN, TF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = assign_smem_bytes<BN, PAIR>(k.natoms, k.XB, k.CS);
+  cudaError_t e = cudaFuncSetAttribute(k_assign<BN, TF32, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = k.ntiles < nsm ? k.ntiles : nsm;
-  if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles_per_inst;
+  // one CTA (or CTA pair) per SM (pair), never more than there are tiles;
+  // pairs: as many as can be resident at once (clusters must fit in a GPC)
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  int64_t units = nsm;
+  if constexpr (PAIR) {
+    cfg.blockDim = dim3(kAssignThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(nsm / 2 * 2));
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, k_assign<BN, TF32, true>, &cfg) != cudaSuccess || clusters < 1)
+      clusters = nsm / 2;
+    units = clusters;
+  }
+  const int64_t active = k.ntiles < units ? k.ntiles : units;
+  const int64_t grid = PAIR ? 2 * active : active;
+  if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles128_per_inst;
   if (grid <= 0) return cudaSuccess;
   count_launch();
-  k_assign<BN, TF32><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
-                                                                               *a.camap, k);
+  if constexpr (PAIR) {
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    e = cudaLaunchKernelEx(&cfg, k_assign<BN, TF32, true>, *a.xmap, *a.xamap, *a.cmap, *a.camap, k);
+    if (e != cudaSuccess) return e;
+  } else {
+    k_assign<BN, TF32, false><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
+                                                                                        *a.camap, k);
+  }
   return cudaGetLastError();
 }
 
-size_t assign_smem_for(int BN, int natoms, int XB, int CS) {
+size_t assign_smem_for(int BN, int natoms, int XB, int CS, bool pair) {
   switch (BN) {
-    case 256: return assign_smem_bytes<256>(natoms, XB, CS);
-    case 128: return assign_smem_bytes<128>(natoms, XB, CS);
-    default: return assign_smem_bytes<64>(natoms, XB, CS);
+    case 256: return pair ? assign_smem_bytes<256, true>(natoms, XB, CS) : assign_smem_bytes<256, false>(natoms, XB, CS);
+    case 128: return pair ? assign_smem_bytes<128, true>(natoms, XB, CS) : assign_smem_bytes<128, false>(natoms, XB, CS);
+    default: return assign_smem_bytes<64, false>(natoms, XB, CS);
   }
 }
 
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s) {
   const bool tf32 = p.dtype == kDtypeF32;
+  if (p.ac.pair) {
+    switch (p.ac.BN) {
+      case 256: return tf32 ? launch_t<256, true, true>(p, a, s) : launch_t<256, false, true>(p, a, s);
+      case 128: return tf32 ? launch_t<128, true, true>(p, a, s) : launch_t<128, false, true>(p, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.ac.BN) {
-    case 256: return tf32 ? launch_t<256, true>(p, a, s) : launch_t<256, false>(p, a, s);
-    case 128: return tf32 ? launch_t<128, true>(p, a, s) : launch_t<128, false>(p, a, s);
-    case 64: return tf32 ? launch_t<64, true>(p, a, s) : launch_t<64, false>(p, a, s);
+    case 256: return tf32 ? launch_t<256, true, false>(p, a, s) : launch_t<256, false, false>(p, a, s);
+    case 128: return tf32 ? launch_t<128, true, false>(p, a, s) : launch_t<128, false, false>(p, a, s);
+    case 64: return tf32 ? launch_t<64, true, false>(p, a, s) : launch_t<64, false, false>(p, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -19,7 +19,7 @@
 #include "km_internal.h"
 
 namespace km {
-size_t assign_smem_for(int BN, int natoms, int XB, int CS);
+size_t assign_smem_for(int BN, int natoms, int XB, int CS, bool pair);
 size_t small_update_smem(int64_t N, int K, int D);
 }  // namespace km
 
@@ -58,6 +58,18 @@ uint64_t wait_limit_ns() {
     uint64_t d = 2000000000ull;
     if (e && *e) d = strtoull(e, nullptr, 10);
     return d;
+  }();
+  return v;
+}
+
+// Form of the assignment kernel: -1 = default (single), 0 = one CTA per
+// 128-point tile, 1 = CTA pairs.  Set by KM_ASSIGN_FORM=single|pair.
+int assign_form() {
+  static int v = [] {
+    const char* e = getenv("KM_ASSIGN_FORM");
+    if (e && strcmp(e, "single") == 0) return 0;
+    if (e && strcmp(e, "pair") == 0) return 1;
+    return -1;
   }();
   return v;
 }
@@ -179,16 +191,26 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   ac.natoms = (p.Dop * p.es + 127) / 128;
   int bn0 = K <= 64 ? 64 : (K <= 128 ? 128 : 256);
   bool found = false;
-  for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
-    for (int xb = 2; xb >= 1 && !found; --xb) {
-      for (int cs = 4; cs >= 2 && !found; --cs) {
-        const size_t sm = assign_smem_for(bn, ac.natoms, xb, cs);
-        if (sm <= static_cast<size_t>(kSmemLimit)) {
-          ac.BN = bn;
-          ac.XB = xb;
-          ac.CS = cs;
-          ac.smem = sm;
-          found = true;
+  // Single-CTA tiles by default (measured as fast as CTA pairs on
+  // 1M x 1024 x 128: the epilogue, not the centroid stream, sets the pace);
+  // CTA pairs (cta_group::2, centroid tiles of 128 or 256) on request.  The
+  // deepest rings that fit in shared memory are taken.
+  const int form = assign_form();
+  for (int pair = form == 1 ? 1 : 0; pair >= 0 && !found; --pair) {
+    if (form == 1 && !pair && bn0 >= 128) continue;
+    for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
+      if (pair && bn < 128) continue;
+      for (int xb = 2; xb >= 1 && !found; --xb) {
+        for (int cs = 4; cs >= 2 && !found; --cs) {
+          const size_t sm = assign_smem_for(bn, ac.natoms, xb, cs, pair != 0);
+          if (sm <= static_cast<size_t>(kSmemLimit)) {
+            ac.pair = pair != 0;
+            ac.BN = bn;
+            ac.XB = xb;
+            ac.CS = cs;
+            ac.smem = sm;
+            found = true;
+          }
         }
       }
     }
@@ -244,7 +266,8 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   p.off_caug = take(32 * static_cast<size_t>(B) * p.Kp);
   p.off_clp = take(static_cast<size_t>(B) * K * p.Dop * (dtype == KM_BF16 ? 2 : 4));
   if (dtype == KM_F32) p.off_x3 = take(sizeof(float) * BR * 3 * p.Dp);
-  p.off_tobj = take(sizeof(double) * 4 * static_cast<size_t>(p.ntiles));
+  // per-tile partials, or one group per assignment CTA (at most one per SM)
+  p.off_tobj = take(sizeof(double) * 4 * static_cast<size_t>(p.ntiles > 256 ? p.ntiles : 256));
   if (op == KM_OP_FIT || op == KM_OP_FIT_HOST) p.off_idx = take(sizeof(int32_t) * BR);
   p.off_obj = take(sizeof(double) * (op == KM_OP_FIT_HOST ? kMaxHostIters : B));
   if (op != KM_OP_ASSIGN && !p.small_update) {
@@ -338,6 +361,9 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
   return KM_OK;
 }
 
+// Centroid rows per TMA box: a CTA of a pair loads half of each centroid tile.
+int cbox(const Plan& p) { return p.ac.pair ? p.ac.BN / 2 : p.ac.BN; }
+
 size_t op_row_bytes(const Plan& p) { return static_cast<size_t>(p.Dop) * (p.dtype == KM_BF16 ? 2 : 4); }
 
 }  // namespace
@@ -404,8 +430,8 @@ int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int 
   CUtensorMap xmap, xamap, cmap, camap;
   if ((r = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : X, f32, p.Dop, N, B, kTileM)) != KM_OK) return r;
   if ((r = encode_aug_map(&xamap, xaug, f32, N, B, kTileM)) != KM_OK) return r;
-  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
-  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, p.ac.BN)) != KM_OK) return r;
+  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, cbox(p))) != KM_OK) return r;
+  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, cbox(p))) != KM_OK) return r;
   double* tobj = at<double>(c.ws, p.off_tobj);
   int64_t groups = 0;
   AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, mindist, tobj, c.status(), wait_limit_ns(),
@@ -463,8 +489,8 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   CUtensorMap xmap, xamap, cmap, camap;
   if ((r = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : X, f32, p.Dop, N, B, kTileM)) != KM_OK) return r;
   if ((r = encode_aug_map(&xamap, xaug, f32, N, B, kTileM)) != KM_OK) return r;
-  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, p.ac.BN)) != KM_OK) return r;
-  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, p.ac.BN)) != KM_OK) return r;
+  if ((r = encode_map(&cmap, clp, f32, p.Dop, K, B, cbox(p))) != KM_OK) return r;
+  if ((r = encode_aug_map(&camap, caug, f32, p.Kp, B, cbox(p))) != KM_OK) return r;
   KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
@@ -596,9 +622,9 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
     for (int i = 0; i < 2; ++i) KM_CUDA(cudaEventRecord(ev_free[i], c.s));
     const bool f32 = dtype == KM_F32;
     CUtensorMap cmap, camap;
-    int rr = encode_map(&cmap, clp, f32, p.Dop, K, 1, p.ac.BN);
+    int rr = encode_map(&cmap, clp, f32, p.Dop, K, 1, cbox(p));
     if (rr != KM_OK) return rr;
-    if ((rr = encode_aug_map(&camap, caug, f32, p.Kp, 1, p.ac.BN)) != KM_OK) return rr;
+    if ((rr = encode_aug_map(&camap, caug, f32, p.Kp, 1, cbox(p))) != KM_OK) return rr;
     const int64_t nch = (N + p.chunk_rows - 1) / p.chunk_rows;
     const size_t rowb = static_cast<size_t>(D) * p.es;
     int64_t g = 0;

@@ -29,6 +29,7 @@ inline std::atomic<uint64_t>& launch_counter() {
 inline void count_launch(uint64_t n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
 
 struct AssignCfg {
+  bool pair = false;   // CTA pairs with cta_group::2 UMMAs (256-point tiles)
   int BN = 0;          // centroids per UMMA tile (N of the MMA), 64/128/256
   int XB = 0;          // point-tile buffers (1 or 2)
   int CS = 0;          // centroid-tile stages
