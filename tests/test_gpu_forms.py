@@ -55,9 +55,10 @@ def test_assign_forms_match_oracle(form, tmp_path):
     io, d1, _ = oracle.assign(Xi, Ci)
     assert np.array_equal(out["int"][0].numpy(), io)
     assert np.array_equal(out["int"][1].double().numpy(), d1)
-    for key, (X, C, idx, md, obj) in out.items():
+    for key, val in out.items():
         if key == "int":
             continue
+        X, C, idx, md, obj = val
         B = key[3]
         for b in range(B):
             Xb, Cb = (X[b], C[b]) if B > 1 else (X, C)
