@@ -100,39 +100,72 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// Load CW (16 or 32) consecutive TMEM columns of this thread's lane and wait.
+// Start loading CW (16 or 32) consecutive TMEM columns of this thread's lane.
+// The registers are valid only after tmem_ld_wait on the same array.
 template <int CW>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CW]);
+__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t (&r)[CW]);
 
 template <>
-__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
-  tmem_ld32(taddr, v);
+__device__ __forceinline__ void tmem_ld_issue<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
 }
 
 template <>
-__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+__device__ __forceinline__ void tmem_ld_issue<16>(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Wait for this thread's outstanding TMEM loads.  The registers of `r` pass
+// through the statement, so no use of them can be scheduled before it.
+template <int CW>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[CW]);
+
+template <>
+__device__ __forceinline__ void tmem_ld_wait<32>(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_wait<16>(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
 }
 
 // Minimum key of CW scores: key = score bits with the low 5 bits replaced by
-// the column index in [0, CW) (held in registers: ci[i] == i, mask == ~31),
+// the column index i in [0, CW) (mask == ~31 in a register, i an immediate),
 // so each key is one three-input bitwise operation.  Reduced with 3-input
 // minima.
 template <int CW>
-__device__ __forceinline__ uint32_t chunk_min_key(const float (&v)[CW], const uint32_t (&ci)[CW], uint32_t mask) {
+__device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint32_t mask) {
   float k[CW];
 #pragma unroll
-  for (int i = 0; i < CW; ++i) k[i] = __uint_as_float((__float_as_uint(v[i]) & mask) | ci[i]);
+  for (int i = 0; i < CW; ++i) k[i] = __uint_as_float((v[i] & mask) | static_cast<uint32_t>(i));
   constexpr int L1 = CW / 3 + (CW % 3);  // CW=32: 10 triples + 2 singles; CW=16: 5 triples + 1 single
   float a[L1];
 #pragma unroll
@@ -188,9 +221,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr uint32_t kTmemCols = 2 * BN;
-  constexpr int kQ = BN / 4;                 // columns per epilogue warp per tile
-  constexpr int CW = kQ < 32 ? kQ : 32;      // columns per TMEM load
-  constexpr int kChunks = kQ / CW;
+  constexpr int kHalf = BN / 2;                // columns per epilogue warp per tile
+  constexpr int CW = kHalf < 32 ? kHalf : 32;  // columns per TMEM load
+  constexpr int kChunks = kHalf / CW;
   constexpr int kElem = TF32 ? 32 : 64;      // elements per 128-byte atom row
 
   if (threadIdx.x == 0) {
@@ -198,7 +231,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);  // both CTAs' epilogues release the lead's
+      // one epilogue group (half the epilogue warps) reads each accumulator
+      // buffer; for pairs both CTAs' groups release the lead's barrier
+      mbar_init(&a_empty[i], PAIR ? kEpiWarps : kEpiWarps / 2);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&c_full[i], 1);
@@ -340,49 +375,57 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     }
   } else {
     // -------------------------------------------------- epilogue warps
+    // Two groups of 8 warps; group g reads accumulator buffer g, i.e. every
+    // other centroid tile, so each group has two MMA tiles' time per tile and
+    // the groups' bursts of work interleave.  Within a group, 2 warps per TMEM
+    // lane quarter each take half of the tile's columns, in CW-column chunks
+    // whose TMEM loads run one chunk ahead of the reduction.
     const int ew = warp - 2;
-    const int q = warp & 3;   // TMEM lane quarter this warp may access
-    const int h = ew >> 2;    // column quarter of each accumulator tile
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int grp = ew >> 3;           // accumulator buffer this warp reads
+    const int half = (ew >> 2) & 1;    // column half of each accumulator tile
+    const int h = grp * 2 + half;      // partial-result slot of the merge
     const int r_local = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    int ab = 0;
     uint32_t aph = 0, mph = 0;
     bool ok = true;
     double cta_obj = 0.0;
-    uint32_t ci[CW];
-#pragma unroll
-    for (int i = 0; i < CW; ++i) ci[i] = static_cast<uint32_t>(i) + p.zero;
     const uint32_t kmask = ~31u + p.zero;
-    const uint32_t a_empty_lead0 = PAIR ? mapa_shared(smem_addr(&a_empty[0]), 0) : 0u;
-    const uint32_t a_empty_lead1 = PAIR ? mapa_shared(smem_addr(&a_empty[1]), 0) : 0u;
-    for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
+    const uint32_t a_empty_lead = PAIR ? mapa_shared(smem_addr(&a_empty[grp]), 0) : 0u;
+    int64_t ct0 = 0;  // centroid tiles this CTA processed before the current point tile
+    for (int64_t t = unit; ok && t < p.ntiles; t += nunits, ct0 += nct) {
       const int b = static_cast<int>(t / p.tiles_per_inst);
       const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
       const int64_t row = rt * TM + static_cast<int64_t>(rank) * kTileM + r_local;
       const bool valid = row < p.rows;
       float best = CUDART_INF_F;
       int bk = 0;
-      for (int j = 0; j < nct; ++j) {
-        if (!mbar_wait(&a_full[ab], aph, g)) { ok = false; break; }
+      for (int j = static_cast<int>((ct0 + grp) & 1); j < nct; j += 2) {
+        // the MMA issuer alternates buffers per centroid tile: tile ct0 + j uses buffer (ct0 + j) & 1 == grp
+        if (!mbar_wait(&a_full[grp], aph, g)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t col0 = tmem_base + lane_off + static_cast<uint32_t>(grp * BN + half * kHalf);
+        uint32_t v[2][CW];
+        tmem_ld_issue<CW>(col0, v[0]);
+        tmem_ld_wait<CW>(v[0]);
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
-          float v[CW];
-          tmem_ld<CW>(tmem_base + lane_off + static_cast<uint32_t>(ab * BN + h * kQ + c * CW), v);
-          const uint32_t m = chunk_min_key<CW>(v, ci, kmask);
+          if (c + 1 < kChunks) tmem_ld_issue<CW>(col0 + static_cast<uint32_t>((c + 1) * CW), v[(c + 1) & 1]);
+          const uint32_t m = chunk_min_key<CW>(v[c & 1], kmask);
           const float mv = __uint_as_float(m & ~31u);
           if (mv < best) {
             best = mv;
-            bk = j * BN + h * kQ + c * CW + static_cast<int>(m & 31u);
+            bk = j * BN + half * kHalf + c * CW + static_cast<int>(m & 31u);
           }
+          if (c + 1 < kChunks) tmem_ld_wait<CW>(v[(c + 1) & 1]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          if (PAIR && !leader) mbar_arrive_cluster(ab == 0 ? a_empty_lead0 : a_empty_lead1);
-          else mbar_arrive(&a_empty[ab]);
+          if (PAIR && !leader) mbar_arrive_cluster(a_empty_lead);
+          else mbar_arrive(&a_empty[grp]);
         }
-        if (++ab == 2) { ab = 0; aph ^= 1u; }
+        aph ^= 1u;
       }
       if (!ok) break;
       // merge the four column quarters of this point tile
