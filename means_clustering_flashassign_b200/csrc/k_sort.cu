@@ -56,16 +56,18 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
 
 // In-place exclusive scan of blkhist[0..nblk)[d] over the blocks, and the
 // digit totals.  A block takes 32 digits (one per lane, so every load is
-// coalesced) and splits the block range among its 8 warps: each warp sums
+// coalesced) and splits the block range among its 32 warps: each warp sums
 // its part, the parts are scanned in shared memory, and each warp rewrites
-// its part as running prefixes.
-__global__ void __launch_bounds__(256) k_sort_colscan(int32_t* __restrict__ blkhist, int R, int64_t nblk,
-                                                      int32_t* __restrict__ total) {
-  __shared__ int32_t part[8][32];
+// its part as running prefixes.  (Up to 8K blocks the parts are at most 8
+// rows: one batch of loads per warp.)
+constexpr int kColscanWarps = 32;
+__global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
+                                                                     int64_t nblk, int32_t* __restrict__ total) {
+  __shared__ int32_t part[kColscanWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d = blockIdx.x * 32 + lane;
   const bool ok = d < R;
-  const int64_t seg = (nblk + 7) / 8;
+  const int64_t seg = (nblk + kColscanWarps - 1) / kColscanWarps;
   const int64_t b0 = warp * seg < nblk ? warp * seg : nblk;
   const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
   constexpr int CH = 8;
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(256) k_sort_colscan(int32_t* __restrict__ blkh
   __syncthreads();
   int32_t run = 0;
   for (int w = 0; w < warp; ++w) run += part[w][lane];
-  if (warp == 7 && ok) total[d] = run + s;
+  if (warp == kColscanWarps - 1 && ok) total[d] = run + s;
   for (int64_t b = b0; b < b1; b += CH) {
     int32_t v[CH];
 #pragma unroll
@@ -133,8 +135,24 @@ __device__ void block_exclusive_scan(const int32_t* total, int R, int32_t* base,
   __syncthreads();
 }
 
+// Lanes of the warp holding the same digit as this lane (the low `bits` bits
+// compared), among the lanes with `valid` set: one ballot per digit bit, each
+// lane keeping the lanes that agree with it on that bit.  Same result as a
+// match.any over the digits of the valid lanes, at a few cycles per bit.
+__device__ __forceinline__ uint32_t match_digit(int dig, int bits, bool valid) {
+  uint32_t m = __ballot_sync(0xffffffffu, valid);
+#pragma unroll 12
+  for (int b = 0; b < 12; ++b) {
+    if (b >= bits) break;
+    const bool set = (dig >> b) & 1;
+    const uint32_t bb = __ballot_sync(0xffffffffu, set);
+    m &= set ? bb : ~bb;
+  }
+  return m;
+}
+
 // Stable scatter of one pass: per-warp counters rank equal digits in point
-// order (match.any groups equal digits inside a warp step).  The block first
+// order (match_digit groups equal digits inside a warp step).  The block first
 // places its elements in digit order in shared memory, then writes them out
 // in that order, so elements of one digit leave as one contiguous run at
 // base[d] + (earlier blocks' d).  Writes one 8-byte (point, key) pair per
@@ -151,16 +169,11 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
   int32_t* lstart = base + R;                  // [R]  block-local start of each digit
   int32_t* wcnt = lstart + R;                  // [W][R]
   int32_t* tmp = wcnt + W * R;                 // [blockDim.x / 32]
+  int32_t* bo = tmp + (blockDim.x >> 5);       // [R]  earlier blocks' count of each digit
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  block_exclusive_scan(total, R, base, tmp);
-  if (start && blockIdx.x == 0) {
-    // single-pass sorts: the digit is the cluster id, so base[] is start[]
-    for (int k = threadIdx.x; k < K; k += blockDim.x) start[k] = base[k];
-    if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
-  }
-  for (int i = threadIdx.x; i < W * R; i += blockDim.x) wcnt[i] = 0;
-  __syncthreads();
+  int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  int bits = 0;
+  while ((1 << bits) < R) ++bits;
 
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
   const int64_t w0 = t0 + static_cast<int64_t>(warp) * (T / W);
@@ -180,11 +193,25 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
     }
     dig[s] = i < n ? ((key[s] >> shift) & (R - 1)) : -1;
   }
+  // While the keys are in flight: the digit totals and this block's offsets
+  // into shared memory, per-warp counters zeroed; then the digit bases.
+  for (int d = threadIdx.x; d < R; d += blockDim.x) {
+    base[d] = total[d];
+    bo[d] = boff[d];
+  }
+  for (int i = threadIdx.x; i < W * R; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  block_exclusive_scan(base, R, base, tmp);
+  if (start && blockIdx.x == 0) {
+    // single-pass sorts: the digit is the cluster id, so base[] is start[]
+    for (int k = threadIdx.x; k < K; k += blockDim.x) start[k] = base[k];
+    if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
+  }
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int64_t i = w0 + s * 32 + lane;
     const bool v = i < n;
-    const uint32_t peers = __match_any_sync(0xffffffffu, dig[s]);
+    const uint32_t peers = match_digit(dig[s], bits, v);
     int before = 0;
     if (v) before = wcnt[warp * R + dig[s]];
     rank[s] = before + __popc(peers & ltm);
@@ -202,7 +229,6 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
   }
   __syncthreads();
   block_exclusive_scan(lstart, R, lstart, tmp);
-  int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
   for (int d = threadIdx.x; d < R; d += blockDim.x) {
     int32_t run = lstart[d];
     for (int w = 0; w < W; ++w) {
@@ -210,7 +236,7 @@ __global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* 
       wcnt[w * R + d] = run;
       run += c;
     }
-    base[d] += boff[d] - lstart[d];  // global position = base[d] + local position
+    base[d] += bo[d] - lstart[d];  // global position = base[d] + local position
     boff[d] = 0;  // leave the counts zeroed for the next accumulation
   }
   __syncthreads();
@@ -242,7 +268,7 @@ __global__ void k_bounds(const int2* __restrict__ sorted, int64_t n, int K, int3
 }
 
 static size_t scatter_smem(int R, int W, int threads, int T) {
-  return (2 * static_cast<size_t>(T) + 2 * static_cast<size_t>(R) + static_cast<size_t>(W) * R + threads) * 4;
+  return (2 * static_cast<size_t>(T) + 3 * static_cast<size_t>(R) + static_cast<size_t>(W) * R + threads) * 4;
 }
 
 cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
@@ -262,7 +288,7 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     else if (!a.hist0_ready)
       k_sort_hist<false><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(a.keys, nullptr, a.n, c.T, c.shift[ps], R,
                                                                          bh, a.K);
-    k_sort_colscan<<<(R + 31) / 32, 256, 0, s>>>(bh, R, nblk, a.total);
+    k_sort_colscan<<<(R + 31) / 32, kColscanWarps * 32, 0, s>>>(bh, R, nblk, a.total);
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
     int2* out = last ? a.pairs : a.pairs_tmp;

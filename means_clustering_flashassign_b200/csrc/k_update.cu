@@ -440,6 +440,14 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
   if (blockIdx.x < f.nwarp_blocks) {
     const int k = static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + warp;
     if (k >= f.K) return;
+    // The whole-block sum row is loaded together with the segment bounds (it
+    // is the answer for every cluster inside one segmented-sum block).
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = lane + 32 * i;
+      w[i] = j < f.D ? f.sums[static_cast<int64_t>(k) * f.D + j] : 0.f;
+    }
     const int64_t s0 = f.start[k], s1 = f.start[k + 1], cnt = s1 - s0;
     float v[8];
     if (cnt > 0) {
@@ -451,7 +459,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
         v[i] = 0.f;
         if (j < f.D) {
           if (ca == cb) {
-            v[i] = f.sums[static_cast<int64_t>(k) * f.D + j];
+            v[i] = w[i];
           } else {
             float a = f.pr[ca * f.D + j];
             for (int64_t c = ca + 1; c <= cb; ++c) a += f.pl[c * f.D + j];
