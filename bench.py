@@ -46,9 +46,17 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha() -> str:
+# Sources each timed kernel is built from: a recorded ncu traffic figure is
+# used only while these files are unchanged.
+KERNEL_SOURCES = {
+    "k_assign": ("k_assign.cu", "km_ptx.cuh", "km_internal.h"),
+    "update": ("k_update.cu", "k_sort.cu", "km_rows.cuh", "km_internal.h"),
+}
+
+
+def kernel_source_sha(kernel: str = "k_assign") -> str:
     h = hashlib.sha256()
-    for f in ("k_assign.cu", "km_ptx.cuh", "k_update.cu", "k_sort.cu"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "means_clustering_flashassign_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -60,7 +68,7 @@ def recorded_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(path):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     for line in open(path):
         m = re.match(r"\|\s*(\S+)\s*\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
         if m and m.group(1) == kernel and m.group(2) == workload and m.group(4) == sha:
