@@ -67,6 +67,7 @@ constexpr int kAtomBytesPerRow = 128;
 constexpr int kXAtomBytes = kTileM * kAtomBytesPerRow;  // 16 KB per point-tile atom
 constexpr int kAugRowBytes = 32;
 constexpr int kEpiWarps = 16;
+constexpr int kMaxXB = 8;  // point-tile buffers at most
 
 __host__ __device__ constexpr size_t x_buf_bytes(int natoms) {
   return static_cast<size_t>(natoms) * kXAtomBytes + kTileM * kAugRowBytes;
@@ -79,7 +80,7 @@ __host__ __device__ constexpr size_t c_stage_bytes(int natoms, int rows) {
 template <int BN, bool PAIR>
 __host__ __device__ constexpr size_t assign_smem_bytes(int natoms, int XB, int CS) {
   return 1024 /* alignment slack */ + XB * x_buf_bytes(natoms) + CS * c_stage_bytes(natoms, PAIR ? BN / 2 : BN) +
-         3 * kTileM * 8 /* merge slots */ + 32 * 8 /* barriers */ + 16;
+         3 * kTileM * 8 /* merge slots */ + 40 * 8 /* barriers */ + 16;
 }
 
 // Shared-memory descriptor for the 32-byte augmentation slice (K-major,
@@ -186,7 +187,9 @@ __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint3
   return __float_as_uint(m);
 }
 
-template <int BN, bool TF32, bool PAIR>
+// ONE_CT: one centroid tile per point tile (K <= BN), kept resident per
+// instance (see the producer and the MMA issuer).
+template <int BN, bool TF32, bool PAIR, bool ONE_CT>
 __global__ void __launch_bounds__(kAssignThreads, 1)
     k_assign(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap xamap,
              const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap camap, const AssignK p) {
@@ -201,21 +204,33 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   const bool leader = rank == 0;
   const int64_t unit = PAIR ? blockIdx.x / 2 : blockIdx.x;     // this CTA's (pair's) index
   const int64_t nunits = PAIR ? gridDim.x / 2 : gridDim.x;
+  // Tile order of this CTA (pair).  Batched problems with one centroid tile
+  // per point tile take a contiguous run of tiles, so consecutive tiles
+  // belong to the same instance and its centroid tile stays resident (see
+  // below); otherwise tiles are dealt round robin, which keeps the CTAs'
+  // point-tile reads close together in memory (measured faster for one
+  // large instance).
+  const bool contig = ONE_CT && p.B > 1;
+  const int64_t t_first = contig ? unit * p.ntiles / nunits : unit;
+  const int64_t t_end = contig ? (unit + 1) * p.ntiles / nunits : p.ntiles;
+  const int64_t t_step = contig ? 1 : nunits;
   uint8_t* xs = base;
   uint8_t* cs = xs + XB * xbb;
   float* mval = reinterpret_cast<float*>(cs + CS * csb);  // [3][128]
   int* midx = reinterpret_cast<int*>(mval + 3 * kTileM);  // [3][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(midx + 3 * kTileM);
-  uint64_t* x_full = bars + 0;    // [2]
-  uint64_t* x_empty = bars + 2;   // [2]
-  uint64_t* c_full = bars + 4;    // [4]
-  uint64_t* c_empty = bars + 8;   // [4]
-  uint64_t* a_full = bars + 12;   // [2]
-  uint64_t* a_empty = bars + 14;  // [2]
-  uint64_t* m_full = bars + 16;
-  uint64_t* m_empty = bars + 17;
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* x_full = bars + 0;    // [kMaxXB]
+  uint64_t* x_empty = bars + 8;   // [kMaxXB]
+  uint64_t* c_full = bars + 16;   // [4]
+  uint64_t* c_empty = bars + 20;  // [4]
+  uint64_t* a_full = bars + 24;   // [2]
+  uint64_t* a_empty = bars + 26;  // [2]
+  uint64_t* m_full = bars + 28;
+  uint64_t* m_empty = bars + 29;
+  uint64_t* drain = bars + 30;
+  uint64_t* g_full = bars + 31;   // [2] one-tile merge inside epilogue group g
+  uint64_t* g_empty = bars + 33;  // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 36);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -227,9 +242,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   constexpr int kElem = TF32 ? 32 : 64;      // elements per 128-byte atom row
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxXB; ++i) {
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], 1);
       // one epilogue group (half the epilogue warps) reads each accumulator
       // buffer; for pairs both CTAs' groups release the lead's barrier
@@ -241,6 +258,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     }
     mbar_init(m_full, 3 * kTileM);
     mbar_init(m_empty, kTileM);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&g_full[i], kTileM);
+      mbar_init(&g_empty[i], kTileM);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -272,7 +293,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       prefetch_tensormap(&camap);
       int xb = 0, cst = 0;
       uint32_t xph = 0, cph = 0;
-      int x_iss[2] = {-1, -1}, c_iss[4] = {-1, -1, -1, -1};
+      int x_iss[kMaxXB], c_iss[4] = {-1, -1, -1, -1};
+      for (int i = 0; i < kMaxXB; ++i) x_iss[i] = -1;
+      int64_t b_loaded = -1;
       bool ok = true;
       // Loads of a pair complete on the lead CTA's barriers; only the lead
       // posts the expected bytes (both CTAs' share).
@@ -280,7 +303,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if constexpr (PAIR) tma_load_3d_pair(dst, map, x, y, z, mapa_shared(smem_addr(bar), 0));
         else tma_load_3d(dst, map, x, y, z, bar);
       };
-      for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
+      for (int64_t t = t_first; ok && t < t_end; t += t_step) {
         const int b = static_cast<int>(t / p.tiles_per_inst);
         const int rt = static_cast<int>(t - static_cast<int64_t>(b) * p.tiles_per_inst);
         const int row0 = rt * TM + static_cast<int>(rank) * kTileM;
@@ -291,6 +314,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         load(xdst + natoms * kXAtomBytes, &xamap, 0, row0, b, &x_full[xb]);
         x_iss[xb] = static_cast<int>(xph);
         if (++xb == XB) { xb = 0; xph ^= 1u; }
+        // One centroid tile per point tile: it stays resident while the
+        // instance does not change (the MMA issuer releases the stage then).
+        if constexpr (ONE_CT) {
+          if (b == b_loaded) continue;
+          b_loaded = b;
+        }
         for (int j = 0; j < nct; ++j) {
           if (!mbar_wait(&c_empty[cst], cph ^ 1u, g)) { ok = false; break; }
           uint8_t* cdst = cs + cst * csb;
@@ -337,11 +366,22 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       int xb = 0, cst = 0, ab = 0;
       uint32_t xph = 0, cph = 0, aph = 0;
       bool ok = true;
-      for (int64_t t = unit; ok && t < p.ntiles; t += nunits) {
+      int64_t b_cur = -1;
+      for (int64_t t = t_first; ok && t < t_end; t += t_step) {
         if (!mbar_wait(&x_full[xb], xph, g)) { ok = false; break; }
         const uint32_t xaddr = smem_addr(xs + xb * xbb);
+        bool keep = false;  // stage cst already holds this instance's tile
+        if constexpr (ONE_CT) {
+          const int64_t b = t / p.tiles_per_inst;
+          keep = b == b_cur;
+          if (!keep && b_cur >= 0) {  // leave the previous instance's stage
+            commit(&c_empty[cst]);
+            if (++cst == CS) { cst = 0; cph ^= 1u; }
+          }
+          b_cur = b;
+        }
         for (int j = 0; j < nct; ++j) {
-          if (!mbar_wait(&c_full[cst], cph, g)) { ok = false; break; }
+          if (!keep && !mbar_wait(&c_full[cst], cph, g)) { ok = false; break; }
           if (!mbar_wait(&a_empty[ab], aph ^ 1u, g)) { ok = false; break; }
           tc_fence_after();
           const uint32_t caddr = smem_addr(cs + cst * csb);
@@ -356,9 +396,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           }
           mma(dtm, sw32_kmajor_desc(xaddr + natoms * kXAtomBytes),
               sw32_kmajor_desc(caddr + natoms * HB * kAtomBytesPerRow), 1u);
-          commit(&c_empty[cst]);
+          if constexpr (!ONE_CT) {
+            commit(&c_empty[cst]);
+            if (++cst == CS) { cst = 0; cph ^= 1u; }
+          }
           commit(&a_full[ab]);
-          if (++cst == CS) { cst = 0; cph ^= 1u; }
           if (++ab == 2) { ab = 0; aph ^= 1u; }
         }
         if (!ok) break;
@@ -387,13 +429,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const int h = grp * 2 + half;      // partial-result slot of the merge
     const int r_local = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t aph = 0, mph = 0;
+    uint32_t aph = 0, mph = 0, gph = 0;
     bool ok = true;
     double cta_obj = 0.0;
     const uint32_t kmask = ~31u + p.zero;
     const uint32_t a_empty_lead = PAIR ? mapa_shared(smem_addr(&a_empty[grp]), 0) : 0u;
     int64_t ct0 = 0;  // centroid tiles this CTA processed before the current point tile
-    for (int64_t t = unit; ok && t < p.ntiles; t += nunits, ct0 += nct) {
+    for (int64_t t = t_first; ok && t < t_end; t += t_step, ct0 += nct) {
       const int b = static_cast<int>(t / p.tiles_per_inst);
       const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
       const int64_t row = rt * TM + static_cast<int64_t>(rank) * kTileM + r_local;
@@ -428,24 +470,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         aph ^= 1u;
       }
       if (!ok) break;
-      // merge the four column quarters of this point tile
-      if (h != 0) {
-        if (!mbar_wait(m_empty, mph ^ 1u, g)) { ok = false; break; }
-        mval[(h - 1) * kTileM + r_local] = best;
-        midx[(h - 1) * kTileM + r_local] = bk;
-        mbar_arrive(m_full);
-      } else {
-        if (!mbar_wait(m_full, mph, g)) { ok = false; break; }
-#pragma unroll
-        for (int hh = 0; hh < 3; ++hh) {
-          const float ov = mval[hh * kTileM + r_local];
-          const int ok_ = midx[hh * kTileM + r_local];
-          if (ov < best || (ov == best && ok_ < bk)) {
-            best = ov;
-            bk = ok_;
-          }
-        }
-        mbar_arrive(m_empty);
+      // the point tile's result: argmin index, distance, sort counts, objective
+      auto emit = [&]() {
         float md = 0.f;
         if (valid) {
           const int64_t o = static_cast<int64_t>(b) * p.rows + row;
@@ -464,8 +490,54 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           const int64_t tile128 = rt * (TM / kTileM) + rank;
           if (tile128 * kTileM < p.rows) p.tobj[(static_cast<int64_t>(b) * p.tiles128_per_inst + tile128) * 4 + q] = ds;
         }
+      };
+      auto better = [&](float ov, int oi) {
+        if (ov < best || (ov == best && oi < bk)) {
+          best = ov;
+          bk = oi;
+        }
+      };
+      if constexpr (ONE_CT) {
+        // One accumulator tile per point tile: the owning group's two column
+        // halves merge through the group's own slots; the other group skips
+        // the tile, so the two groups never wait for each other.
+        if (((ct0 + grp) & 1) != 0) continue;
+        if (half != 0) {
+          if (!mbar_wait(&g_empty[grp], gph ^ 1u, g)) { ok = false; break; }
+          mval[grp * kTileM + r_local] = best;
+          midx[grp * kTileM + r_local] = bk;
+          mbar_arrive(&g_full[grp]);
+        } else {
+          if (!mbar_wait(&g_full[grp], gph, g)) { ok = false; break; }
+          better(mval[grp * kTileM + r_local], midx[grp * kTileM + r_local]);
+          mbar_arrive(&g_empty[grp]);
+          emit();
+        }
+        gph ^= 1u;
+        continue;
+      }
+      // merge the four column quarters of this point tile
+      if (h != 0) {
+        if (!mbar_wait(m_empty, mph ^ 1u, g)) { ok = false; break; }
+        mval[(h - 1) * kTileM + r_local] = best;
+        midx[(h - 1) * kTileM + r_local] = bk;
+        mbar_arrive(m_full);
+      } else {
+        if (!mbar_wait(m_full, mph, g)) { ok = false; break; }
+#pragma unroll
+        for (int hh = 0; hh < 3; ++hh) better(mval[hh * kTileM + r_local], midx[hh * kTileM + r_local]);
+        mbar_arrive(m_empty);
+        emit();
       }
       mph ^= 1u;
+    }
+    if constexpr (ONE_CT) {
+      // both groups' column-half-0 warps hold objective sums: group 1 hands
+      // its sums to group 0 (fixed order), over the epilogue warps only
+      double* objx = reinterpret_cast<double*>(mval + 2 * kTileM);  // [4], the unused third merge slot
+      if (p.obj_per_cta && h == 2 && lane == 0) objx[q] = cta_obj;
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+      if (p.obj_per_cta && h == 0 && lane == 0) cta_obj += objx[q];
     }
     if (h == 0 && p.obj_per_cta && lane == 0 && p.tobj) p.tobj[static_cast<int64_t>(blockIdx.x) * 4 + q] = cta_obj;
   }
@@ -479,7 +551,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   }
 }
 
-template <int BN, bool TF32, bool PAIR>
+template <int BN, bool TF32, bool PAIR, bool ONE_CT>
 static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s) {
   constexpr int TM = PAIR ? 2 * kTileM : kTileM;
   AssignK k{};
@@ -505,7 +577,7 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN, PAIR>(k.natoms, k.XB, k.CS);
-  cudaError_t e = cudaFuncSetAttribute(k_assign<BN, TF32, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(k_assign<BN, TF32, PAIR, ONE_CT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0;
@@ -528,7 +600,8 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(nsm / 2 * 2));
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, k_assign<BN, TF32, true>, &cfg) != cudaSuccess || clusters < 1)
+    if (cudaOccupancyMaxActiveClusters(&clusters, k_assign<BN, TF32, true, ONE_CT>, &cfg) != cudaSuccess ||
+        clusters < 1)
       clusters = nsm / 2;
     units = clusters;
   }
@@ -539,10 +612,10 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   count_launch();
   if constexpr (PAIR) {
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    e = cudaLaunchKernelEx(&cfg, k_assign<BN, TF32, true>, *a.xmap, *a.xamap, *a.cmap, *a.camap, k);
+    e = cudaLaunchKernelEx(&cfg, k_assign<BN, TF32, true, ONE_CT>, *a.xmap, *a.xamap, *a.cmap, *a.camap, k);
     if (e != cudaSuccess) return e;
   } else {
-    k_assign<BN, TF32, false><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
+    k_assign<BN, TF32, false, ONE_CT><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
                                                                                         *a.camap, k);
   }
   return cudaGetLastError();
@@ -556,19 +629,24 @@ size_t assign_smem_for(int BN, int natoms, int XB, int CS, bool pair) {
   }
 }
 
+template <int BN, bool TF32, bool PAIR>
+static cudaError_t launch_ct(const Plan& p, const AssignArgs& a, cudaStream_t s) {
+  return a.Kp == BN ? launch_t<BN, TF32, PAIR, true>(p, a, s) : launch_t<BN, TF32, PAIR, false>(p, a, s);
+}
+
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s) {
   const bool tf32 = p.dtype == kDtypeF32;
   if (p.ac.pair) {
     switch (p.ac.BN) {
-      case 256: return tf32 ? launch_t<256, true, true>(p, a, s) : launch_t<256, false, true>(p, a, s);
-      case 128: return tf32 ? launch_t<128, true, true>(p, a, s) : launch_t<128, false, true>(p, a, s);
+      case 256: return tf32 ? launch_ct<256, true, true>(p, a, s) : launch_ct<256, false, true>(p, a, s);
+      case 128: return tf32 ? launch_ct<128, true, true>(p, a, s) : launch_ct<128, false, true>(p, a, s);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (p.ac.BN) {
-    case 256: return tf32 ? launch_t<256, true, false>(p, a, s) : launch_t<256, false, false>(p, a, s);
-    case 128: return tf32 ? launch_t<128, true, false>(p, a, s) : launch_t<128, false, false>(p, a, s);
-    case 64: return tf32 ? launch_t<64, true, false>(p, a, s) : launch_t<64, false, false>(p, a, s);
+    case 256: return tf32 ? launch_ct<256, true, false>(p, a, s) : launch_ct<256, false, false>(p, a, s);
+    case 128: return tf32 ? launch_ct<128, true, false>(p, a, s) : launch_ct<128, false, false>(p, a, s);
+    case 64: return tf32 ? launch_ct<64, true, false>(p, a, s) : launch_ct<64, false, false>(p, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -16,6 +16,7 @@
 #include <cstdint>
 
 #include "km_internal.h"
+#include "km_ptx.cuh"
 
 namespace km {
 
@@ -133,22 +134,6 @@ __device__ void block_exclusive_scan(const int32_t* total, int R, int32_t* base,
     run += t;
   }
   __syncthreads();
-}
-
-// Lanes of the warp holding the same digit as this lane (the low `bits` bits
-// compared), among the lanes with `valid` set: one ballot per digit bit, each
-// lane keeping the lanes that agree with it on that bit.  Same result as a
-// match.any over the digits of the valid lanes, at a few cycles per bit.
-__device__ __forceinline__ uint32_t match_digit(int dig, int bits, bool valid) {
-  uint32_t m = __ballot_sync(0xffffffffu, valid);
-#pragma unroll 12
-  for (int b = 0; b < 12; ++b) {
-    if (b >= bits) break;
-    const bool set = (dig >> b) & 1;
-    const uint32_t bb = __ballot_sync(0xffffffffu, set);
-    m &= set ? bb : ~bb;
-  }
-  return m;
 }
 
 // Stable scatter of one pass: per-warp counters rank equal digits in point

@@ -14,6 +14,7 @@
 #include <math_constants.h>
 
 #include "km_internal.h"
+#include "km_ptx.cuh"
 #include "km_rows.cuh"
 
 namespace km {
@@ -192,28 +193,38 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
     int prevk = __shfl_up_sync(0xffffffffu, cur_k, 1);
     if (lane == 0) prevk = open_k;
     const uint32_t starts = __ballot_sync(0xffffffffu, lane < nb && cur_k != prevk);
-    int a = 0;
-    while (a < nb) {
-      if ((starts >> a) & 1u) {
-        flush(false);
-        open_k = __shfl_sync(0xffffffffu, cur_k, a);
-        open_left = false;
-      }
-      const uint32_t later = a + 1 < 32 ? (starts >> (a + 1)) << (a + 1) : 0u;
-      const int e = later ? __ffs(later) - 1 : nb;
-      uint4 buf[G::STEPS];
+    // every row of the batch in one round trip ...
+    uint4 buf[G::STEPS];
 #pragma unroll
-      for (int s = 0; s < G::STEPS; ++s) {
-        const int slot = s * G::RPS + sub;
-        const int r = __shfl_sync(0xffffffffu, cur_p, slot);
-        if (slot >= a && slot < e && active)
-          buf[s] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(r) * row_bytes + cl * 16));
-        else
-          buf[s] = make_uint4(0u, 0u, 0u, 0u);
-      }
+    for (int s = 0; s < G::STEPS; ++s) {
+      const int slot = s * G::RPS + sub;
+      const int r = __shfl_sync(0xffffffffu, cur_p, slot);
+      if (slot < nb && active)
+        buf[s] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(r) * row_bytes + cl * 16));
+      else
+        buf[s] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // ... then the runs inside it are split from registers
+    if (starts == 0u) {
 #pragma unroll
       for (int s = 0; s < G::STEPS; ++s) add16<BF16>(acc, buf[s]);
-      a = e;
+    } else {
+      int a = 0;
+      while (a < nb) {
+        if ((starts >> a) & 1u) {
+          flush(false);
+          open_k = __shfl_sync(0xffffffffu, cur_k, a);
+          open_left = false;
+        }
+        const uint32_t later = a + 1 < 32 ? (starts >> (a + 1)) << (a + 1) : 0u;
+        const int e = later ? __ffs(later) - 1 : nb;
+#pragma unroll
+        for (int s = 0; s < G::STEPS; ++s) {
+          const int slot = s * G::RPS + sub;
+          if (slot >= a && slot < e) add16<BF16>(acc, buf[s]);
+        }
+        a = e;
+      }
     }
   }
   flush(right_cont);
@@ -627,45 +638,74 @@ __device__ __forceinline__ uint32_t lanemask_lt_u() {
   return m;
 }
 
+// Exclusive scan of v[0..256) in place (256 threads): warp shuffles, then
+// the 8 warp totals.
+__device__ __forceinline__ void scan256_exclusive(int32_t* v, int32_t* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t x0 = v[threadIdx.x];
+  int32_t x = x0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t run = 0;
+    for (int w = 0; w < 8; ++w) { const int32_t t = wsum[w]; wsum[w] = run; run += t; }
+  }
+  __syncthreads();
+  v[threadIdx.x] = wsum[warp] + x - x0;
+  __syncthreads();
+}
+
+static_assert(kSmallMaxN <= 65536 && kSmallMaxK <= 65536, "key and rank are packed in 16 bits each");
+
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   extern __shared__ __align__(16) int32_t ssm[];
   constexpr int W = 8;
   const int N = static_cast<int>(p.N), K = p.K, D = p.D;
   // 16-byte aligned pieces first: slot vectors, the double reduction buffer,
-  // then the integer arrays.
+  // the sorted pairs, then the integer arrays.  kr[i] packs point i's key
+  // (low 16 bits; K <= kSmallMaxK) and its rank among equal keys of its warp
+  // range (high 16 bits; N <= kSmallMaxN).
   float* slot_v = reinterpret_cast<float*>(ssm);                      // [W][2][D]
   double* red = reinterpret_cast<double*>(slot_v + 2 * W * D);        // [256]
-  int32_t* keys = reinterpret_cast<int32_t*>(red + 256);              // [N]
-  int32_t* lrank = keys + N;           // [N]
-  int32_t* perm = lrank + N;           // [N]
-  int32_t* wcnt = perm + N;            // [W][K]
+  int2* pairs = reinterpret_cast<int2*>(red + 256);                   // [N] sorted (point, cluster)
+  uint32_t* kr = reinterpret_cast<uint32_t*>(pairs + N);              // [N]
+  int32_t* wcnt = reinterpret_cast<int32_t*>(kr + N);                 // [W][K]
   int32_t* start = wcnt + W * K;       // [K+1]
   int32_t* tmp = start + K + 1;        // [256]
   int* slot_k = tmp + 256;             // [W][2]
+  int32_t* wsum = slot_k + 2 * W;      // [8]
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* gidx = p.idx + static_cast<int64_t>(b) * N;
   const uint8_t* X = p.X + static_cast<int64_t>(b) * N * p.row_bytes;
   float* C = p.C + static_cast<int64_t>(b) * K * D;
+  int bits = 0;
+  while ((1 << bits) < K) ++bits;
 
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const int32_t v = gidx[i];  // ids outside [0, K) are clamped (memory safety only)
-    keys[i] = v < 0 ? 0 : (v >= K ? K - 1 : v);
+    kr[i] = static_cast<uint32_t>(v < 0 ? 0 : (v >= K ? K - 1 : v));
   }
   for (int i = threadIdx.x; i < W * K; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
-  // stable ranks inside each warp's contiguous range
+  // stable ranks inside each warp's contiguous range (equal keys of a warp
+  // step found with one ballot per key bit)
   const int Lw = ((N + W - 1) / W + 31) / 32 * 32;
   const uint32_t ltm = lanemask_lt_u();
   for (int i0 = warp * Lw; i0 < (warp + 1) * Lw && i0 < N; i0 += 32) {
     const int i = i0 + lane;
     const bool v = i < N && i < (warp + 1) * Lw;
-    const int d = v ? keys[i] : -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    const int d = v ? static_cast<int>(kr[i]) : -1;
+    const uint32_t peers = match_digit(d, bits, v);
     int before = 0;
     if (v) before = wcnt[warp * K + d];
-    if (v) lrank[i] = before + __popc(peers & ltm);
+    if (v) kr[i] = static_cast<uint32_t>(d) | (static_cast<uint32_t>(before + __popc(peers & ltm)) << 16);
     __syncwarp();
     if (v && lane == __ffs(peers) - 1) wcnt[warp * K + d] = before + __popc(peers);
     __syncwarp();
@@ -685,38 +725,37 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   {
     const int per = (K + 255) / 256;
     const int lo = threadIdx.x * per;
-    int s = 0;
-    for (int i = lo; i < lo + per && i < K; ++i) s += start[i];
-    tmp[threadIdx.x] = s;
+    int sum = 0;
+    for (int i = lo; i < lo + per && i < K; ++i) sum += start[i];
+    tmp[threadIdx.x] = sum;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int run = 0;
-      for (int i = 0; i < 256; ++i) { const int v = tmp[i]; tmp[i] = run; run += v; }
-    }
-    __syncthreads();
+    scan256_exclusive(tmp, wsum);
     int run = tmp[threadIdx.x];
     for (int i = lo; i < lo + per && i < K; ++i) { const int v = start[i]; start[i] = run; run += v; }
     if (threadIdx.x == 0) start[K] = N;
   }
   __syncthreads();
+  // scatter into sorted (point, cluster) pairs
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const int w = i / Lw;
-    perm[start[keys[i]] + wcnt[w * K + keys[i]] + lrank[i]] = i;
+    const int key = static_cast<int>(kr[i] & 0xffffu), rank = static_cast<int>(kr[i] >> 16);
+    pairs[start[key] + wcnt[(i / Lw) * K + key] + rank] = make_int2(i, key);
   }
   __syncthreads();
-  // segmented sums: runs inside a warp range become centroids directly
+  // segmented sums over the sorted pairs: runs inside a warp range become
+  // centroids directly
   const int L = (N + W - 1) / W;
   const int q0 = warp * L < N ? warp * L : N;
   const int q1 = q0 + L < N ? q0 + L : N;
-  warp_range_sums<LPR, BF16>(X, p.row_bytes, D, perm, start, K, q0, q1, lane, slot_k + 2 * warp,
-                             slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
-                               const float cntf = static_cast<float>(start[k + 1] - start[k]);
-                               // divide (not multiply by a reciprocal) to match sum / count
-                               float q[8];
+  warp_range_sums_keyed<LPR, BF16>(X, p.row_bytes, D, K, pairs, N, q0, q1, lane, slot_k + 2 * warp,
+                                   slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
+                                     const float cntf = static_cast<float>(start[k + 1] - start[k]);
+                                     // divide (not multiply by a reciprocal) to match sum / count
+                                     float q[8];
 #pragma unroll
-                               for (int i = 0; i < 8; ++i) q[i] = acc[i] / cntf;
-                               store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q, 1.f);
-                             });
+                                     for (int i = 0; i < 8; ++i) q[i] = acc[i] / cntf;
+                                     store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q,
+                                                          1.f);
+                                   });
   __syncthreads();
   for (int j = threadIdx.x; j < D; j += blockDim.x) {
     int open = -1;
@@ -749,17 +788,17 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
       orow = p.dtype == kDtypeBF16
                  ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(p.c_op) + grow * D)
                  : static_cast<void*>(reinterpret_cast<float*>(p.c_op) + grow * 3 * p.Dp);
-    const float s = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, orow, lane);
+    const float sq = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, orow, lane);
     if (lane == 0) {
-      if (p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, s, 1);
+      if (p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, sq, 1);
       if (p.counts) p.counts[grow] = start[k + 1] - start[k];
     }
   }
   if (p.tobj && p.obj) {
     const double* t = p.tobj + static_cast<int64_t>(b) * p.tiles_per_inst * 4;
-    double s = 0.0;
-    for (int64_t i = threadIdx.x; i < p.tiles_per_inst * 4; i += blockDim.x) s += t[i];
-    red[threadIdx.x] = s;
+    double sd = 0.0;
+    for (int64_t i = threadIdx.x; i < p.tiles_per_inst * 4; i += blockDim.x) sd += t[i];
+    red[threadIdx.x] = sd;
     __syncthreads();
     for (int w = 128; w > 0; w >>= 1) {
       if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
@@ -771,9 +810,9 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
 
 size_t small_update_smem(int64_t N, int K, int D) {
   const int W = 8;
-  size_t ints = 3 * static_cast<size_t>(N) + static_cast<size_t>(W) * K + K + 1 + 256 + 2 * W;
-  size_t floats = 2 * static_cast<size_t>(W) * D + 1;
-  return (ints + floats) * 4 + 16 + 256 * 8;
+  const size_t floats = 2 * static_cast<size_t>(W) * D;                                   // slot vectors
+  const size_t ints = 3 * static_cast<size_t>(N) + static_cast<size_t>(W) * K + K + 1 + 256 + 2 * W + 8;
+  return floats * 4 + 256 * 8 + ints * 4 + 16;
 }
 
 template <int LPR>

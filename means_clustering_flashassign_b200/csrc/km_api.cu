@@ -200,8 +200,14 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     if (form == 1 && !pair && bn0 >= 128) continue;
     for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
       if (pair && bn < 128) continue;
-      for (int xb = 2; xb >= 1 && !found; --xb) {
-        for (int cs = 4; cs >= 2 && !found; --cs) {
+      // One centroid tile per point tile (K <= BN): it stays resident per
+      // instance, so two stages suffice and the point tiles (one tile of MMA
+      // time each) get the deepest ring that fits.  Otherwise two point
+      // buffers and the deepest centroid ring.
+      const bool one_ct = K <= bn;
+      const int xb_hi = one_ct ? 8 : 2;
+      for (int xb = xb_hi; xb >= 1 && !found; --xb) {
+        for (int cs = one_ct ? 2 : 4; cs >= 2 && !found; --cs) {
           const size_t sm = assign_smem_for(bn, ac.natoms, xb, cs, pair != 0);
           if (sm <= static_cast<size_t>(kSmemLimit)) {
             ac.pair = pair != 0;

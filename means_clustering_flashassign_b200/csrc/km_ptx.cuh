@@ -200,6 +200,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Lanes of the warp holding the same digit as this lane (the low `bits` bits
+// compared), among the lanes with `valid` set: one ballot per digit bit, each
+// lane keeping the lanes that agree with it on that bit.  Same result as a
+// match.any over the digits of the valid lanes, at a few cycles per bit.
+__device__ __forceinline__ uint32_t match_digit(int dig, int bits, bool valid) {
+  uint32_t m = __ballot_sync(0xffffffffu, valid);
+#pragma unroll 12
+  for (int b = 0; b < 12; ++b) {
+    if (b >= bits) break;
+    const bool set = (dig >> b) & 1;
+    const uint32_t bb = __ballot_sync(0xffffffffu, set);
+    m &= set ? bb : ~bb;
+  }
+  return m;
+}
+
 // ------------------------------------------------------ CTA pairs (2 SMs)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
