@@ -632,6 +632,12 @@ struct SmallK {
   int obj_stride;
 };
 
+__device__ __forceinline__ void* op_row_of(const SmallK& p, int64_t grow) {
+  if (!p.c_op) return nullptr;
+  if (p.dtype == kDtypeBF16) return reinterpret_cast<__nv_bfloat16*>(p.c_op) + grow * p.D;
+  return reinterpret_cast<float*>(p.c_op) + grow * 3 * p.Dp;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt_u() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -662,6 +668,50 @@ __device__ __forceinline__ void scan256_exclusive(int32_t* v, int32_t* wsum) {
 
 static_assert(kSmallMaxN <= 65536 && kSmallMaxK <= 65536, "key and rank are packed in 16 bits each");
 
+// Operand row of a centroid held in the row-gather register layout (lane
+// cl = lane % LPR holds the 16-byte column group cl: 8 bf16 or 4 float
+// columns of the mean), and ||c||^2 of the operand values, on every lane.
+// bf16: -2 * bf16(mean); f32: the TF32 split -2 * [hi | lo | hi] of row
+// length 3 * Dp.  Lanes with lane >= LPR only help reduce.
+template <int LPR, bool BF16>
+__device__ __forceinline__ float emit_operand_lpr(const float (&q)[8], int row_bytes, int Dp, void* row, int lane) {
+  const int cl = lane % LPR;
+  const bool active = cl * 16 < row_bytes;
+  const bool writer = active && lane < LPR && row != nullptr;
+  float s = 0.f;
+  if constexpr (BF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(q[2 * i]), h1 = __float2bfloat16_rn(q[2 * i + 1]);
+      const float f0 = __bfloat162float(h0), f1 = __bfloat162float(h1);
+      if (active) s = fmaf(f1, f1, fmaf(f0, f0, s));
+      const __nv_bfloat16 o0 = __float2bfloat16_rn(-2.f * f0), o1 = __float2bfloat16_rn(-2.f * f1);
+      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o1)) << 16);
+    }
+    if (writer) reinterpret_cast<uint4*>(static_cast<uint8_t*>(row) + cl * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    float hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (active) s = fmaf(q[i], q[i], s);
+      hi[i] = tf32_round(q[i]);
+      lo[i] = tf32_round(q[i] - hi[i]);
+    }
+    if (writer) {
+      float* o = static_cast<float*>(row) + cl * 4;
+      reinterpret_cast<float4*>(o)[0] = make_float4(-2.f * hi[0], -2.f * hi[1], -2.f * hi[2], -2.f * hi[3]);
+      reinterpret_cast<float4*>(o + Dp)[0] = make_float4(-2.f * lo[0], -2.f * lo[1], -2.f * lo[2], -2.f * lo[3]);
+      reinterpret_cast<float4*>(o + 2 * Dp)[0] = make_float4(-2.f * hi[0], -2.f * hi[1], -2.f * hi[2], -2.f * hi[3]);
+    }
+  }
+  // the LPR lanes of one row hold its column groups; lanes of other rows
+  // (sub > 0) hold copies: reduce inside groups of LPR lanes
+#pragma unroll
+  for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   extern __shared__ __align__(16) int32_t ssm[];
@@ -688,9 +738,19 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   int bits = 0;
   while ((1 << bits) < K) ++bits;
 
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const int32_t v = gidx[i];  // ids outside [0, K) are clamped (memory safety only)
-    kr[i] = static_cast<uint32_t>(v < 0 ? 0 : (v >= K ? K - 1 : v));
+  for (int i0 = 0; i0 < N; i0 += 8 * 256) {  // eight loads in flight per thread
+    int32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * 256 + threadIdx.x;
+      v[u] = i < N ? gidx[i] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * 256 + threadIdx.x;
+      // ids outside [0, K) are clamped (memory safety only)
+      if (i < N) kr[i] = static_cast<uint32_t>(v[u] < 0 ? 0 : (v[u] >= K ? K - 1 : v[u]));
+    }
   }
   for (int i = threadIdx.x; i < W * K; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
@@ -755,13 +815,24 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
                                      for (int i = 0; i < 8; ++i) q[i] = acc[i] / cntf;
                                      store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q,
                                                           1.f);
+                                     // operand row and norm row straight from the registers
+                                     const int64_t grow = static_cast<int64_t>(b) * K + k;
+                                     void* orow = op_row_of(p, grow);
+                                     const float sq = emit_operand_lpr<LPR, BF16>(q, p.row_bytes, p.Dp, orow, lane);
+                                     if (lane == 0 && p.caug)
+                                       write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes,
+                                                     p.dtype, sq, 1);
                                    });
+  __syncthreads();
+  int* cut_list = tmp;  // clusters finished by the combine below (at most 2W)
+  if (threadIdx.x == 0) tmp[255] = 0;
   __syncthreads();
   for (int j = threadIdx.x; j < D; j += blockDim.x) {
     int open = -1;
     float a = 0.f;
     auto flush = [&](int k, float v) {
       C[static_cast<int64_t>(k) * D + j] = v / static_cast<float>(start[k + 1] - start[k]);
+      if (j == 0) cut_list[tmp[255]++] = k;
     };
     for (int w = 0; w < W; ++w)
       for (int sl = 0; sl < 2; ++sl) {
@@ -779,21 +850,18 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
     if (open >= 0) flush(open, a);
   }
   __syncthreads();
-  // operand copies, norms and counts for every cluster (empty ones keep C)
-  for (int k = warp; k < K; k += W) {
-    float* crow = C + static_cast<int64_t>(k) * D;
+  // operand and norm rows of the clusters the combine finished (the others
+  // were written from registers; empty clusters keep C and their rows)
+  const int ncut = tmp[255];
+  for (int c = warp; c < ncut; c += W) {
+    const int k = cut_list[c];
+    const float* crow = C + static_cast<int64_t>(k) * D;
     const int64_t grow = static_cast<int64_t>(b) * K + k;
-    void* orow = nullptr;
-    if (p.c_op)
-      orow = p.dtype == kDtypeBF16
-                 ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(p.c_op) + grow * D)
-                 : static_cast<void*>(reinterpret_cast<float*>(p.c_op) + grow * 3 * p.Dp);
-    const float sq = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, orow, lane);
-    if (lane == 0) {
-      if (p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, sq, 1);
-      if (p.counts) p.counts[grow] = start[k + 1] - start[k];
-    }
+    const float sq = emit_operand_row([&](int j) { return crow[j]; }, D, p.Dp, p.dtype, op_row_of(p, grow), lane);
+    if (lane == 0 && p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, sq, 1);
   }
+  if (p.counts)
+    for (int k = threadIdx.x; k < K; k += blockDim.x) p.counts[static_cast<int64_t>(b) * K + k] = start[k + 1] - start[k];
   if (p.tobj && p.obj) {
     const double* t = p.tobj + static_cast<int64_t>(b) * p.tiles_per_inst * 4;
     double sd = 0.0;
