@@ -260,11 +260,49 @@ def run_ours(args, world, rank, local):
             "ms_call": round(ms_call, 4),
             "clocks": clk.summary(),
         }
+        if world == 1 and args.ablation and wl.B == 1:
+            res["ablation"] = ablation(wl, X, C0, km, assign_ms, update_ms)
         if world == 1 and not args.no_e2e:
             res["e2e"] = e2e(args, wl, X, C0, km)
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl, X, C0, args.cpu_sample, 2)
     return res
+
+
+def _event_ms(fn, reps=3):
+    """Median CUDA-event time of fn() on the current stream."""
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sorted(ts)[len(ts) // 2]
+
+
+def ablation(wl, X, C0, km, assign_ms, update_ms):
+    """The method against the two strategies it replaces, on the same device
+    and inputs: materialised distances (library GEMM writes the N x K scores,
+    an argmin kernel reads them back; rows chunked so the scores take at most
+    8 GiB) and the atomic-scatter update.  Baseline times are CUDA-event
+    medians of 3 calls after one warm-up; the method's are the bench's phase
+    times (kernel only, norms precomputed once per fit)."""
+    chunk = int(max(1, min(wl.N, (8 << 30) // (4 * wl.K), ((1 << 31) - 1) // wl.K)))
+    km.ablation_assign_materialized(X, C0, chunk_rows=chunk)  # warm-up (loads cuBLAS)
+    torch.cuda.synchronize()
+    mat_ms = _event_ms(lambda: km.ablation_assign_materialized(X, C0, chunk_rows=chunk))
+    idx, _, _ = km.assign(X, C0)
+    C = C0.float().clone()
+    km.ablation_update_atomic(X, idx, C)
+    torch.cuda.synchronize()
+    atom_ms = _event_ms(lambda: km.ablation_update_atomic(X, idx, C))
+    return {"assign_flash_ms": round(assign_ms, 4), "assign_materialized_ms": round(mat_ms, 4),
+            "assign_speedup": round(mat_ms / assign_ms, 2), "materialized_chunk_rows": chunk,
+            "materialized_scores_bytes": int(wl.N) * wl.K * 4,
+            "update_sort_inverse_ms": round(update_ms, 4), "update_atomic_ms": round(atom_ms, 4),
+            "update_speedup": round(atom_ms / update_ms, 2)}
 
 
 def h2d_link_gbs(src: torch.Tensor, dev) -> float:
@@ -399,6 +437,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=1 << 20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ablation", action="store_true",
+                    help="also time the materialised-distance and atomic-scatter baselines")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")

@@ -254,6 +254,31 @@ int km_assign_static(const void* X, const void* C, int B, int64_t N, int D, int 
  */
 int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_ns, void* stream);
 
+/*
+ * Baselines (not used by the fit).  The two strategies "Flash-KMeans" (§1
+ * Problem) says FlashAssign and the Sort-Inverse Update replace, for measuring
+ * the method against them on the same device:
+ *   km_ablation_assign_materialized: the N x K distance matrix goes through
+ *     device memory -- S = X C^T by a library GEMM (cuBLAS, fp32 out) into
+ *     the workspace, chunk_rows rows at a time, then an argmin kernel reads S
+ *     back: idx / mindist as km_assign (lowest index on exact ties).
+ *   km_ablation_update_atomic: every point adds its row to its cluster's sum
+ *     with float atomics and counts itself; C = sum / count (an empty cluster
+ *     keeps C).  The atomics' order varies, so the last bits of C may differ
+ *     from run to run.
+ * One instance (B = 1); X [N][D] and C [K][D] in dtype (bf16 or fp32), D a
+ * multiple of 8, X 16-byte aligned.  Workspace sizes: which = 0 (assign; at
+ * least chunk_rows x K x 4 bytes) or 1 (update).  cuBLAS is loaded at run
+ * time (libcublas.so.12); if it cannot be, the assign baseline returns
+ * KM_ERR_UNSUPPORTED.
+ */
+size_t km_ablation_workspace_size(int which, int64_t N, int D, int K, int dtype, int64_t chunk_rows);
+int km_ablation_assign_materialized(const void* X, const void* C, int64_t N, int D, int K, int dtype,
+                                    int64_t chunk_rows, int32_t* idx, float* mindist, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+int km_ablation_update_atomic(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, float* C,
+                              int32_t* counts, void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

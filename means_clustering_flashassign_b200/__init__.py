@@ -26,7 +26,8 @@ import torch
 from . import build as _build
 
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
-           "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static",
+           "ablation_assign_materialized", "ablation_update_atomic", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -36,7 +37,8 @@ STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_E
           4: "KM_ERR_WORKSPACE", 5: "KM_ERR_TIMEOUT"}
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
-           "km_launch_count", "km_assign_static"]
+           "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
+           "km_ablation_update_atomic"]
 
 _lock = threading.Lock()
 _lib = None
@@ -78,6 +80,10 @@ def library() -> ctypes.CDLL:
             L.km_fit_host.argtypes = [P, P, I64, I, I, I, I, I64, P, P, P, P, P, SZ, P]
             L.km_selftest_timeout.argtypes = [P, SZ, I64, P]
             L.km_argsort.argtypes = [P, I64, I, P, P, P, SZ, P]
+            L.km_ablation_workspace_size.argtypes = [I, I64, I, I, I, I64]
+            L.km_ablation_workspace_size.restype = SZ
+            L.km_ablation_assign_materialized.argtypes = [P, P, I64, I, I, I, I64, P, P, P, SZ, P]
+            L.km_ablation_update_atomic.argtypes = [P, P, I64, I, I, I, P, P, P, SZ, P]
             L.km_fit_profile.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
             L.km_launch_count.restype = ctypes.c_uint64
             L.km_assign_static.argtypes = [P, P, I, I64, I, I, I, P, P, P, P]
@@ -222,6 +228,47 @@ def argsort(idx: torch.Tensor, K: int, *, workspace=None, stream=None):
     ws = _workspace(OP_ARGSORT, 1, N, 0, K, 0, idx.device, workspace)
     _check(library().km_argsort(_ptr(idx), N, K, _ptr(perm), _ptr(start), _ptr(ws), ws.numel(), _stream(stream)))
     return perm, start
+
+
+def ablation_assign_materialized(X: torch.Tensor, C: torch.Tensor, *, chunk_rows: Optional[int] = None,
+                                 mindist: bool = True, stream=None):
+    """Baseline (not the method): the N x K distance matrix through device
+    memory -- a library GEMM writes the scores, an argmin kernel reads them.
+    One instance.  Returns (idx int32 [N], mindist float32 [N] or None)."""
+    _contig_cuda(X, "X"), _contig_cuda(C, "C")
+    if X.dim() != 2 or C.dim() != 2 or C.shape[1] != X.shape[1] or C.dtype != X.dtype:
+        raise ValueError("X [N, D] and C [K, D] of one dtype")
+    N, D = X.shape
+    K = C.shape[0]
+    dt = _dtype_code(X)
+    cr = N if chunk_rows is None else int(chunk_rows)
+    idx = torch.empty(N, dtype=torch.int32, device=X.device)
+    md = torch.empty(N, dtype=torch.float32, device=X.device) if mindist else None
+    wsb = int(library().km_ablation_workspace_size(0, N, D, K, dt, cr))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=X.device)
+    _check(library().km_ablation_assign_materialized(_ptr(X), _ptr(C), N, D, K, dt, cr, _ptr(idx), _ptr(md),
+                                                     _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, md
+
+
+def ablation_update_atomic(X: torch.Tensor, idx: torch.Tensor, C: torch.Tensor, *, stream=None):
+    """Baseline (not the method): every point added to its cluster's sum with
+    float atomics, then C = sum / count (empty clusters keep C).  C float32
+    [K, D] is updated in place.  Returns counts int32 [K]."""
+    _contig_cuda(X, "X"), _contig_cuda(idx, "idx"), _contig_cuda(C, "C")
+    if X.dim() != 2 or C.dim() != 2 or C.shape[1] != X.shape[1] or C.dtype != torch.float32:
+        raise ValueError("X [N, D] and float32 C [K, D]")
+    if idx.dtype != torch.int32 or idx.shape != (X.shape[0],):
+        raise ValueError("idx must be int32 [N]")
+    N, D = X.shape
+    K = C.shape[0]
+    dt = _dtype_code(X)
+    counts = torch.empty(K, dtype=torch.int32, device=X.device)
+    wsb = int(library().km_ablation_workspace_size(1, N, D, K, dt, 0))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=X.device)
+    _check(library().km_ablation_update_atomic(_ptr(X), _ptr(idx), N, D, K, dt, _ptr(C), _ptr(counts), _ptr(ws),
+                                               ws.numel(), _stream(stream)))
+    return counts
 
 
 def fit(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_out=None, counts_out=None,

@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 OBJ_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkm.so")
-SOURCES = ["km_api.cu", "k_prep.cu", "k_assign.cu", "k_sort.cu", "k_update.cu", "km_noalloc.cu"]
+SOURCES = ["km_api.cu", "k_prep.cu", "k_assign.cu", "k_sort.cu", "k_update.cu", "km_noalloc.cu", "k_ablation.cu"]
 HEADERS = ["km_internal.h", "km_ptx.cuh", "km_rows.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -62,7 +62,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(compile_one, SOURCES))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs]
+    cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-ldl"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -20,6 +20,12 @@
 
 namespace km {
 size_t assign_smem_for(int BN, int natoms, int XB, int CS, bool pair);
+size_t ablation_assign_ws(int64_t chunk_rows, int K);
+size_t ablation_update_ws(int D, int K);
+int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int dtype, int64_t chunk_rows,
+                    int32_t* idx, float* mindist, void* ws, cudaStream_t s);
+int ablation_update(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, float* C,
+                    int32_t* counts, void* ws, cudaStream_t s);
 size_t small_update_smem(int64_t N, int K, int D);
 }  // namespace km
 
@@ -699,6 +705,62 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               perm,
               start ? start : at<int32_t>(c.ws, p.off_start)};
   KM_CUDA(launch_sort(p, sa, c.s));
+  return KM_OK;
+}
+
+// ------------------------------------------------------------- baselines
+namespace {
+int ablation_check(const void* X, int64_t N, int D, int K, int dtype) {
+  if (!X) return fail(KM_ERR_INVALID_ARG, "X is required");
+  if (dtype != KM_F32 && dtype != KM_BF16) return fail(KM_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (N < 1 || K < 1 || K > N) return fail(KM_ERR_INVALID_ARG, "need 1 <= K <= N (N=%lld K=%d)", (long long)N, K);
+  if (N >= (int64_t(1) << 31)) return fail(KM_ERR_UNSUPPORTED, "N must be below 2^31");
+  if (D < 8 || D % 8 != 0) return fail(KM_ERR_UNSUPPORTED, "D=%d must be a positive multiple of 8", D);
+  if (!aligned16(X)) return fail(KM_ERR_INVALID_ARG, "X must be 16-byte aligned");
+  return check_device();
+}
+}  // namespace
+
+size_t km_ablation_workspace_size(int which, int64_t N, int D, int K, int dtype, int64_t chunk_rows) {
+  (void)dtype;
+  if (N < 1 || K < 1 || D < 8) return 0;
+  if (which == 0) {
+    if (chunk_rows < 1) return 0;
+    return km::ablation_assign_ws(chunk_rows < N ? chunk_rows : N, K);
+  }
+  if (which == 1) return km::ablation_update_ws(D, K);
+  return 0;
+}
+
+int km_ablation_assign_materialized(const void* X, const void* C, int64_t N, int D, int K, int dtype,
+                                    int64_t chunk_rows, int32_t* idx, float* mindist, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  int r = ablation_check(X, N, D, K, dtype);
+  if (r != KM_OK) return r;
+  if (!C || !idx) return fail(KM_ERR_INVALID_ARG, "C and idx are required");
+  if (chunk_rows < 1) return fail(KM_ERR_INVALID_ARG, "chunk_rows must be >= 1");
+  const int64_t cr = chunk_rows < N ? chunk_rows : N;
+  if (cr * static_cast<int64_t>(K) >= (int64_t(1) << 31))
+    return fail(KM_ERR_UNSUPPORTED, "chunk_rows x K must stay below 2^31 scores");
+  if (!workspace || workspace_bytes < km::ablation_assign_ws(cr, K))
+    return fail(KM_ERR_WORKSPACE, "workspace needs %zu bytes", km::ablation_assign_ws(cr, K));
+  r = km::ablation_assign(X, C, N, D, K, dtype, cr, idx, mindist, workspace, static_cast<cudaStream_t>(stream));
+  if (r == KM_ERR_UNSUPPORTED) return fail(r, "cuBLAS (libcublas.so.12) could not be loaded");
+  if (r != KM_OK) return fail(r, "materialised-distance assignment failed");
+  return KM_OK;
+}
+
+int km_ablation_update_atomic(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, float* C,
+                              int32_t* counts, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  int r = ablation_check(X, N, D, K, dtype);
+  if (r != KM_OK) return r;
+  if (!idx || !C || !counts) return fail(KM_ERR_INVALID_ARG, "idx, C and counts are required");
+  if (!workspace || workspace_bytes < km::ablation_update_ws(D, K))
+    return fail(KM_ERR_WORKSPACE, "workspace needs %zu bytes", km::ablation_update_ws(D, K));
+  r = km::ablation_update(X, idx, N, D, K, dtype, C, counts, workspace, static_cast<cudaStream_t>(stream));
+  if (r != KM_OK) return fail(r, "atomic-scatter update failed");
   return KM_OK;
 }
 
