@@ -260,6 +260,8 @@ def run_ours(args, world, rank, local):
             "ms_call": round(ms_call, 4),
             "clocks": clk.summary(),
         }
+        if world == 1 and args.tile_sweep:
+            res["tile_sweep"] = tile_sweep(wl, X, C0, km)
         if world == 1 and args.ablation and wl.B == 1:
             res["ablation"] = ablation(wl, X, C0, km, assign_ms, update_ms)
         if world == 1 and not args.no_e2e:
@@ -303,6 +305,51 @@ def ablation(wl, X, C0, km, assign_ms, update_ms):
             "materialized_scores_bytes": int(wl.N) * wl.K * 4,
             "update_sort_inverse_ms": round(update_ms, 4), "update_atomic_ms": round(atom_ms, 4),
             "update_speedup": round(atom_ms / update_ms, 2)}
+
+
+def tile_sweep(wl, X, C0, km, iters=5):
+    """The static shape -> tiling chooser against every tiling that fits
+    (forced with KM_ASSIGN_TILE): assignment-kernel time of each (median of
+    the per-iteration phase times of one fit), the chooser's loss against the
+    fastest, and the time to plan vs the time the sweep took."""
+    dt = km.BF16 if wl.dtype == "bf16" else km.F32
+    t0 = time.perf_counter()
+    chosen = km.plan(km.OP_FIT, wl.B, wl.N, wl.D, wl.K, dt)
+    plan_s = time.perf_counter() - t0
+
+    def assign_ms():
+        r = km.fit_profile(X, C0, iters)
+        # the first objective depends only on X and C0: every tiling must agree
+        j0 = r["objective"].reshape(-1, iters)[:, 0].double().sum().item()
+        return float(sorted(float(v) for v in r["phase_ms"][:, 0])[iters // 2]), j0
+
+    os.environ.pop("KM_ASSIGN_TILE", None)
+    static_ms, j_ref = assign_ms()
+    results = []
+    t0 = time.perf_counter()
+    for pair in (0, 1):
+        for bn in (64, 128, 256):
+            for xb in range(1, 9):
+                for cs in (2, 3, 4):
+                    os.environ["KM_ASSIGN_TILE"] = f"{pair},{bn},{xb},{cs}"
+                    try:
+                        km.workspace_size(km.OP_FIT, wl.B, wl.N, wl.D, wl.K, dt)
+                    except km.KMError:
+                        continue  # does not fit, or not a tiling for this shape
+                    ms, j0 = assign_ms()
+                    results.append({"pair": pair, "BN": bn, "XB": xb, "CS": cs, "assign_ms": round(ms, 4),
+                                    "objective_ok": abs(j0 - j_ref) <= 1e-6 * abs(j_ref)})
+    sweep_s = time.perf_counter() - t0
+    os.environ.pop("KM_ASSIGN_TILE", None)
+    best = min(results, key=lambda r: r["assign_ms"])
+    # the chosen tiling's own entry in the sweep (same conditions as the rest)
+    mine = next(r for r in results if all(r[k] == chosen[k] for k in ("pair", "BN", "XB", "CS")))
+    return {"chosen": {k: chosen[k] for k in ("pair", "BN", "XB", "CS")}, "chosen_assign_ms": mine["assign_ms"],
+            "chosen_unforced_assign_ms": round(static_ms, 4), "best": best,
+            "chooser_loss_pct": round(100.0 * (mine["assign_ms"] - best["assign_ms"]) / best["assign_ms"], 2),
+            "tilings_tried": len(results), "all_objectives_agree": all(r["objective_ok"] for r in results),
+            "plan_seconds": plan_s, "sweep_seconds": round(sweep_s, 2),
+            "all": results}
 
 
 def h2d_link_gbs(src: torch.Tensor, dev) -> float:
@@ -437,6 +484,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=1 << 20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tile-sweep", action="store_true",
+                    help="also time every assignment tiling that fits against the static choice")
     ap.add_argument("--ablation", action="store_true",
                     help="also time the materialised-distance and atomic-scatter baselines")
     args = ap.parse_args()

@@ -48,10 +48,13 @@
  *    workspace must be ordered (same stream or synchronised).
  *  - Environment (read once per process): KM_WAIT_LIMIT_NS sets the bound of
  *    every in-kernel wait (default 2e9 ns); KM_ASSIGN_FORM=single|pair picks
- *    the assignment kernel's form: one CTA per 128-point tile (the default)
- *    or two-SM CTA pairs on 256-point tiles.  Both forms meet the same
+ *    the assignment kernel's form: one CTA per 128-point tile or two-SM CTA
+ *    pairs on 256-point tiles (the default wherever the centroid tile is 128
+ *    or 256 wide).  Both forms meet the same
  *    accuracy rules; the objective's float64 summation order follows the
  *    form's tiling, so its last bits may differ between forms.
+ *    KM_ASSIGN_TILE=pair,BN,XB,CS (read at every call) forces the whole
+ *    assignment tiling; see km_plan_describe.
  */
 #ifndef KM_H_
 #define KM_H_
@@ -253,6 +256,17 @@ int km_assign_static(const void* X, const void* C, int B, int64_t N, int D, int 
  * status km_workspace_status() then reports (KM_ERR_TIMEOUT when it works).
  */
 int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_ns, void* stream);
+
+/*
+ * The tiling the library chooses for a shape (no device needed): out[0..8) =
+ * assignment form (0 one CTA per 128-point tile, 1 CTA pairs), centroid tile
+ * width BN, point-tile buffers, centroid stages, shared memory bytes of the
+ * assignment kernel, K padded to BN, sort passes, sort block size.  The
+ * choice is a static function of the shape and the shared-memory limit
+ * (KM_ASSIGN_FORM and KM_ASSIGN_TILE=pair,BN,XB,CS override it; an override
+ * that does not fit is refused).
+ */
+int km_plan_describe(int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, int64_t* out);
 
 /*
  * Baselines (not used by the fit).  The two strategies "Flash-KMeans" (§1

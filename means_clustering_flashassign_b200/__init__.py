@@ -27,7 +27,7 @@ from . import build as _build
 
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
            "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static",
-           "ablation_assign_materialized", "ablation_update_atomic", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "ablation_assign_materialized", "ablation_update_atomic", "plan", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -38,7 +38,7 @@ STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_E
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
            "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
-           "km_ablation_update_atomic"]
+           "km_ablation_update_atomic", "km_plan_describe"]
 
 _lock = threading.Lock()
 _lib = None
@@ -80,6 +80,7 @@ def library() -> ctypes.CDLL:
             L.km_fit_host.argtypes = [P, P, I64, I, I, I, I, I64, P, P, P, P, P, SZ, P]
             L.km_selftest_timeout.argtypes = [P, SZ, I64, P]
             L.km_argsort.argtypes = [P, I64, I, P, P, P, SZ, P]
+            L.km_plan_describe.argtypes = [I, I, I64, I, I, I, I64, P]
             L.km_ablation_workspace_size.argtypes = [I, I64, I, I, I, I64]
             L.km_ablation_workspace_size.restype = SZ
             L.km_ablation_assign_materialized.argtypes = [P, P, I64, I, I, I, I64, P, P, P, SZ, P]
@@ -228,6 +229,14 @@ def argsort(idx: torch.Tensor, K: int, *, workspace=None, stream=None):
     ws = _workspace(OP_ARGSORT, 1, N, 0, K, 0, idx.device, workspace)
     _check(library().km_argsort(_ptr(idx), N, K, _ptr(perm), _ptr(start), _ptr(ws), ws.numel(), _stream(stream)))
     return perm, start
+
+
+def plan(op: int, B: int, N: int, D: int, K: int, dtype: int, chunk_rows: int = 0) -> dict:
+    """The tiling the library would use for this shape (host-only query)."""
+    out = (ctypes.c_int64 * 8)()
+    _check(library().km_plan_describe(op, B, N, D, K, dtype, chunk_rows, ctypes.cast(out, ctypes.c_void_p)))
+    keys = ("pair", "BN", "XB", "CS", "smem", "Kp", "sort_passes", "sort_block")
+    return {k: int(v) for k, v in zip(keys, out)}
 
 
 def ablation_assign_materialized(X: torch.Tensor, C: torch.Tensor, *, chunk_rows: Optional[int] = None,

@@ -68,7 +68,7 @@ uint64_t wait_limit_ns() {
   return v;
 }
 
-// Form of the assignment kernel: -1 = default (single), 0 = one CTA per
+// Form of the assignment kernel: -1 = default (by shape), 0 = one CTA per
 // 128-point tile, 1 = CTA pairs.  Set by KM_ASSIGN_FORM=single|pair.
 int assign_form() {
   static int v = [] {
@@ -78,7 +78,7 @@ int assign_form() {
     return -1;
   }();
   return v;
-}
+}  // -1 = chosen by shape (pairs where BN >= 128)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -197,23 +197,24 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   ac.natoms = (p.Dop * p.es + 127) / 128;
   int bn0 = K <= 64 ? 64 : (K <= 128 ? 128 : 256);
   bool found = false;
-  // Single-CTA tiles by default (measured as fast as CTA pairs on
-  // 1M x 1024 x 128: the epilogue, not the centroid stream, sets the pace);
-  // CTA pairs (cta_group::2, centroid tiles of 128 or 256) on request.  The
-  // deepest rings that fit in shared memory are taken.
+  // CTA pairs (cta_group::2) for centroid tiles of 128 or 256, else one CTA
+  // per 128-point tile; KM_ASSIGN_FORM=single|pair forces the form.  A sweep
+  // of every tiling that fits (bench.py --tile-sweep) measured pairs 1-2 %
+  // ahead on 1M x 1024 x 128 and level or ahead on the batched and Zipf
+  // shapes.
   const int form = assign_form();
-  for (int pair = form == 1 ? 1 : 0; pair >= 0 && !found; --pair) {
+  for (int pair = form == 0 ? 0 : 1; pair >= 0 && !found; --pair) {
     if (form == 1 && !pair && bn0 >= 128) continue;
     for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
       if (pair && bn < 128) continue;
       // One centroid tile per point tile (K <= BN): it stays resident per
-      // instance, so two stages suffice and the point tiles (one tile of MMA
-      // time each) get the deepest ring that fits.  Otherwise two point
-      // buffers and the deepest centroid ring.
+      // instance and the point tiles (one short tile of MMA time each) get a
+      // 4-deep ring with 3 centroid stages (deeper point rings measured
+      // slower).  Otherwise two point buffers and the deepest centroid ring.
       const bool one_ct = K <= bn;
-      const int xb_hi = one_ct ? 8 : 2;
+      const int xb_hi = one_ct ? 4 : 2;
       for (int xb = xb_hi; xb >= 1 && !found; --xb) {
-        for (int cs = one_ct ? 2 : 4; cs >= 2 && !found; --cs) {
+        for (int cs = one_ct ? 3 : 4; cs >= 2 && !found; --cs) {
           const size_t sm = assign_smem_for(bn, ac.natoms, xb, cs, pair != 0);
           if (sm <= static_cast<size_t>(kSmemLimit)) {
             ac.pair = pair != 0;
@@ -228,6 +229,23 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     }
   }
   if (!found) return bad(KM_ERR_UNSUPPORTED, "no FlashAssign tiling fits shared memory for D=%d", D);
+  // Explicit tiling (measurement of the chooser against a sweep):
+  // KM_ASSIGN_TILE=pair,BN,XB,CS, e.g. "0,256,2,2"; refused if it does not fit.
+  if (const char* e = getenv("KM_ASSIGN_TILE")) {
+    int fp = 0, fb = 0, fx = 0, fc = 0;
+    if (sscanf(e, "%d,%d,%d,%d", &fp, &fb, &fx, &fc) != 4)
+      return bad(KM_ERR_INVALID_ARG, "KM_ASSIGN_TILE='%s' is not pair,BN,XB,CS", e);
+    const bool bn_ok = fb == 64 || fb == 128 || fb == 256;
+    if (!bn_ok || (fp && fb < 128) || fx < 1 || fx > 8 || fc < 2 || fc > 4)
+      return bad(KM_ERR_UNSUPPORTED, "KM_ASSIGN_TILE='%s' is not a supported tiling for K=%d", e, K);
+    const size_t sm = assign_smem_for(fb, ac.natoms, fx, fc, fp != 0);
+    if (sm > static_cast<size_t>(kSmemLimit)) return bad(KM_ERR_UNSUPPORTED, "KM_ASSIGN_TILE='%s' needs %zu bytes of shared memory", e, sm);
+    ac.pair = fp != 0;
+    ac.BN = fb;
+    ac.XB = fx;
+    ac.CS = fc;
+    ac.smem = sm;
+  }
   ac.tmem_cols = 2 * ac.BN;
   p.Kp = (K + ac.BN - 1) / ac.BN * ac.BN;
   p.tiles_per_inst = (p.rows + kTileM - 1) / kTileM;
@@ -705,6 +723,24 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               perm,
               start ? start : at<int32_t>(c.ws, p.off_start)};
   KM_CUDA(launch_sort(p, sa, c.s));
+  return KM_OK;
+}
+
+int km_plan_describe(int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, int64_t* out) {
+  g_err.clear();
+  if (!out) return fail(KM_ERR_INVALID_ARG, "out is required");
+  km::Plan p;
+  const char* why = "";
+  const int r = km::make_plan(p, op, B, N, D, K, dtype, chunk_rows, &why);
+  if (r != KM_OK) return fail(r, "%s", why);
+  out[0] = p.ac.pair ? 1 : 0;
+  out[1] = p.ac.BN;
+  out[2] = p.ac.XB;
+  out[3] = p.ac.CS;
+  out[4] = static_cast<int64_t>(p.ac.smem);
+  out[5] = p.Kp;
+  out[6] = p.sc.passes;
+  out[7] = p.sc.T;
   return KM_OK;
 }
 
