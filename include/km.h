@@ -258,6 +258,25 @@ int km_assign_static(const void* X, const void* C, int B, int64_t N, int D, int 
 int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_ns, void* stream);
 
 /*
+ * Data-parallel building blocks (a point set sharded by rows over several
+ * devices or processes, §2 Methodology's Lloyd iteration with one exchange):
+ *   km_update_accumulate: the Sort-Inverse Update of this shard (argsort,
+ *     segmented sums, ordered combine) added into float64 sums [K][D] and
+ *     int64 counts [K] (zeroed first if zero_first); deterministic.  One
+ *     instance; workspace as km_update (op KM_OP_UPDATE, B = 1).
+ *   km_finalize_sums: C = sums / counts where counts > 0, else C is kept
+ *     (C in/out float [K][D]); C_lp [K][D] (dtype; may be NULL) receives the
+ *     copy the next km_assign takes (bf16 round-to-nearest-even, or float);
+ *     counts_out int32 [K] may be NULL.
+ * Between the two, the caller adds the shards' sums and counts (an
+ * all-reduce); every rank then finalises the same sums to the same C.
+ */
+int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, double* sums,
+                         int64_t* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream);
+int km_finalize_sums(const double* sums, const int64_t* counts, int K, int D, int dtype, float* C, void* C_lp,
+                     int32_t* counts_out, void* stream);
+
+/*
  * The tiling the library chooses for a shape (no device needed): out[0..8) =
  * assignment form (0 one CTA per 128-point tile, 1 CTA pairs), centroid tile
  * width BN, point-tile buffers, centroid stages, shared memory bytes of the

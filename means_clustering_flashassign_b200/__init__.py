@@ -27,7 +27,8 @@ from . import build as _build
 
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
            "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static",
-           "ablation_assign_materialized", "ablation_update_atomic", "plan", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "ablation_assign_materialized", "ablation_update_atomic", "plan", "update_accumulate",
+           "finalize_sums", "fit_data_parallel", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -38,7 +39,7 @@ STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_E
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
            "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
-           "km_ablation_update_atomic", "km_plan_describe"]
+           "km_ablation_update_atomic", "km_plan_describe", "km_update_accumulate", "km_finalize_sums"]
 
 _lock = threading.Lock()
 _lib = None
@@ -81,6 +82,8 @@ def library() -> ctypes.CDLL:
             L.km_selftest_timeout.argtypes = [P, SZ, I64, P]
             L.km_argsort.argtypes = [P, I64, I, P, P, P, SZ, P]
             L.km_plan_describe.argtypes = [I, I, I64, I, I, I, I64, P]
+            L.km_update_accumulate.argtypes = [P, P, I64, I, I, I, P, P, I, P, SZ, P]
+            L.km_finalize_sums.argtypes = [P, P, I, I, I, P, P, P, P]
             L.km_ablation_workspace_size.argtypes = [I, I64, I, I, I, I64]
             L.km_ablation_workspace_size.restype = SZ
             L.km_ablation_assign_materialized.argtypes = [P, P, I64, I, I, I, I64, P, P, P, SZ, P]
@@ -229,6 +232,81 @@ def argsort(idx: torch.Tensor, K: int, *, workspace=None, stream=None):
     ws = _workspace(OP_ARGSORT, 1, N, 0, K, 0, idx.device, workspace)
     _check(library().km_argsort(_ptr(idx), N, K, _ptr(perm), _ptr(start), _ptr(ws), ws.numel(), _stream(stream)))
     return perm, start
+
+
+def update_accumulate(X: torch.Tensor, idx: torch.Tensor, sums: torch.Tensor, counts: torch.Tensor, *,
+                      zero_first: bool = True, workspace=None, stream=None) -> None:
+    """Sort-Inverse Update of one shard added into float64 sums [K, D] and
+    int64 counts [K] (zeroed first by default)."""
+    _contig_cuda(X, "X"), _contig_cuda(idx, "idx"), _contig_cuda(sums, "sums"), _contig_cuda(counts, "counts")
+    if X.dim() != 2 or sums.dtype != torch.float64 or counts.dtype != torch.int64 or idx.dtype != torch.int32:
+        raise ValueError("X [N, D], int32 idx [N], float64 sums [K, D], int64 counts [K]")
+    N, D = X.shape
+    K = sums.shape[0]
+    dt = _dtype_code(X)
+    ws = _workspace(OP_UPDATE, 1, N, D, K, dt, X.device, workspace)
+    _check(library().km_update_accumulate(_ptr(X), _ptr(idx), N, D, K, dt, _ptr(sums), _ptr(counts),
+                                          1 if zero_first else 0, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def finalize_sums(sums: torch.Tensor, counts: torch.Tensor, C: torch.Tensor, C_lp: Optional[torch.Tensor] = None,
+                  counts_out: Optional[torch.Tensor] = None, *, stream=None) -> None:
+    """C = sums / counts where counts > 0 (else kept), in place; C_lp gets the
+    dtype copy for the next assign; counts_out the int32 counts."""
+    for t, n in ((sums, "sums"), (counts, "counts"), (C, "C")):
+        _contig_cuda(t, n)
+    K, D = C.shape
+    dt = _dtype_code(C_lp) if C_lp is not None else F32
+    _check(library().km_finalize_sums(_ptr(sums), _ptr(counts), K, D, dt, _ptr(C), _ptr(C_lp), _ptr(counts_out),
+                                      _stream(stream)))
+
+
+def fit_data_parallel(X: torch.Tensor, C0: torch.Tensor, iters: int, *, group=None):
+    """Lloyd iterations over a point set sharded by rows across the ranks of a
+    torch.distributed process group: every rank passes its own rows X and the
+    same C0.  Per iteration each rank assigns its rows and sums them per
+    cluster (float64, deterministic); one all-reduce adds the ranks' sums,
+    counts and objective; every rank finalises the same sums, so C is the
+    same on all ranks.  The exchange runs through torch.distributed (NCCL on
+    device tensors; host copies for gloo).
+    Returns dict(C float32 [K, D], idx (this rank's rows), counts int32 [K],
+    objective float64 [iters] on the host: the whole point set's J_t)."""
+    import torch.distributed as dist
+    _contig_cuda(X, "X"), _contig_cuda(C0, "C0")
+    if X.dim() != 2 or C0.dim() != 2 or C0.shape[1] != X.shape[1] or C0.dtype != X.dtype:
+        raise ValueError("X [N, D] and C0 [K, D] of one dtype")
+    N, D = X.shape
+    K = C0.shape[0]
+    dev = X.device
+    on_host = dist.get_backend(group) == "gloo"
+
+    def all_reduce(t):
+        if on_host:
+            h = t.cpu()
+            dist.all_reduce(h, group=group)
+            t.copy_(h)
+        else:
+            dist.all_reduce(t, group=group)
+
+    C = C0.float().contiguous().clone()
+    C_lp = C0.clone()
+    sums = torch.empty(K, D, dtype=torch.float64, device=dev)
+    cnt = torch.empty(K, dtype=torch.int64, device=dev)
+    counts = torch.empty(K, dtype=torch.int32, device=dev)
+    idx = torch.empty(N, dtype=torch.int32, device=dev)
+    dt = _dtype_code(X)
+    ws_a = _workspace(OP_ASSIGN, 1, N, D, K, dt, dev)
+    ws_u = _workspace(OP_UPDATE, 1, N, D, K, dt, dev)
+    J = torch.empty(iters, dtype=torch.float64)
+    for t in range(iters):
+        _, _, obj = assign(X, C_lp, idx=idx, want_mindist=False, workspace=ws_a)
+        update_accumulate(X, idx, sums, cnt, workspace=ws_u)
+        all_reduce(sums)
+        all_reduce(cnt)
+        all_reduce(obj)
+        finalize_sums(sums, cnt, C, C_lp, counts)
+        J[t] = obj.item()
+    return dict(C=C, idx=idx, counts=counts, objective=J)
 
 
 def plan(op: int, B: int, N: int, D: int, K: int, dtype: int, chunk_rows: int = 0) -> dict:

@@ -602,6 +602,36 @@ __global__ void k_finalize_acc(int K, int D, int Dp, int dtype, double* acc64, l
   }
 }
 
+// Centroids from float64 sums and counts accumulated elsewhere (e.g. added
+// up across the ranks of a data-parallel fit): C = sum / count where count >
+// 0, else C is kept; C_lp is the dtype copy the next assignment takes (bf16
+// round-to-nearest-even or the float values); counts as int32.
+__global__ void k_finalize_sums(const double* __restrict__ sums, const long long* __restrict__ cnt, int K, int D,
+                                int dtype, float* C, void* C_lp, int32_t* counts) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= static_cast<int64_t>(K) * D) return;
+  const int k = static_cast<int>(e / D);
+  const long long n = cnt[k];
+  float c = C[e];
+  if (n > 0) {
+    c = static_cast<float>(sums[e] / static_cast<double>(n));
+    C[e] = c;
+  }
+  if (C_lp) {
+    if (dtype == kDtypeBF16) static_cast<__nv_bfloat16*>(C_lp)[e] = __float2bfloat16_rn(c);
+    else static_cast<float*>(C_lp)[e] = c;
+  }
+  if (counts && e - static_cast<int64_t>(k) * D == 0) counts[k] = static_cast<int32_t>(n);
+}
+
+cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const long long* cnt, float* C,
+                                 void* C_lp, int32_t* counts, cudaStream_t s) {
+  const int64_t e = static_cast<int64_t>(K) * D;
+  count_launch();
+  k_finalize_sums<<<static_cast<unsigned>((e + 255) / 256), 256, 0, s>>>(sums, cnt, K, D, dtype, C, C_lp, counts);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, void* caug,
                                 int32_t* counts, double* objacc, double* obj_out, cudaStream_t s) {
   const int threads = 256;

@@ -352,7 +352,7 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
-                    bool hist0_ready = false) {
+                    bool hist0_ready = false, double* acc_ext = nullptr, long long* cnt_ext = nullptr) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
@@ -380,8 +380,8 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
   fa.c_op = c_opb;
   fa.caug = caugb;
   fa.counts = countsb;
-  fa.acc64 = mode == 1 ? at<double>(c.ws, p.off_acc64) : nullptr;
-  fa.cnt64 = mode == 1 ? at<long long>(c.ws, p.off_cnt64) : nullptr;
+  fa.acc64 = mode == 1 ? (acc_ext ? acc_ext : at<double>(c.ws, p.off_acc64)) : nullptr;
+  fa.cnt64 = mode == 1 ? (cnt_ext ? cnt_ext : at<long long>(c.ws, p.off_cnt64)) : nullptr;
   fa.tobj = tobjb;
   fa.ntiles = obj ? ntiles : 0;
   fa.obj = obj;
@@ -723,6 +723,35 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               perm,
               start ? start : at<int32_t>(c.ws, p.off_start)};
   KM_CUDA(launch_sort(p, sa, c.s));
+  return KM_OK;
+}
+
+int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, double* sums,
+                         int64_t* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!X || !idx || !sums || !counts) return fail(KM_ERR_INVALID_ARG, "X, idx, sums and counts are required");
+  if (!aligned16(X)) return fail(KM_ERR_INVALID_ARG, "X must be 16-byte aligned");
+  Ctx c;
+  int r = prepare(c, KM_OP_UPDATE, 1, N, D, K, dtype, 0, workspace, workspace_bytes, stream);
+  if (r != KM_OK) return r;
+  if (zero_first) {
+    KM_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
+    KM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int64_t) * K, c.s));
+  }
+  return update_instance(c, X, idx, N, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 1, false, sums,
+                         reinterpret_cast<long long*>(counts));
+}
+
+int km_finalize_sums(const double* sums, const int64_t* counts, int K, int D, int dtype, float* C, void* C_lp,
+                     int32_t* counts_out, void* stream) {
+  g_err.clear();
+  if (!sums || !counts || !C) return fail(KM_ERR_INVALID_ARG, "sums, counts and C are required");
+  if (K < 1 || D < 1) return fail(KM_ERR_INVALID_ARG, "need K >= 1 and D >= 1");
+  if (dtype != KM_F32 && dtype != KM_BF16) return fail(KM_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  int r = check_device();
+  if (r != KM_OK) return r;
+  KM_CUDA(km::launch_finalize_sums(K, D, dtype, sums, reinterpret_cast<const long long*>(counts), C, C_lp,
+                                   counts_out, static_cast<cudaStream_t>(stream)));
   return KM_OK;
 }
 

@@ -182,6 +182,8 @@ struct FinalizeArgs {
   double* obj;       // objective output (mode 0) or accumulator (mode 1)
 };
 cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s);
+cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const long long* cnt, float* C,
+                                 void* C_lp, int32_t* counts, cudaStream_t s);
 
 // Final step of the out-of-core update: centroids from float64 accumulators.
 cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, void* caug,
