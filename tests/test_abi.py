@@ -94,3 +94,34 @@ def test_null_arguments_rejected_before_device_use():
     assert L.km_update(None, None, 1, 100, 64, 10, 1, None, None, None, 0, None) == 1
     assert L.km_fit(None, None, 1, 100, 64, 10, 1, 3, None, None, None, None, None, 0, None) == 1
     assert L.km_argsort(None, 100, 10, None, None, None, 0, None) == 1
+
+
+def test_plan_describes_the_chosen_tiling():
+    # CTA pairs with 256-wide centroid tiles at D=128; two point buffers and
+    # four centroid stages for K > BN; a 4 x 3 ring when one tile covers K
+    p = km.plan(km.OP_FIT, 1, 1 << 20, 128, 1024, km.BF16)
+    assert (p["pair"], p["BN"], p["XB"], p["CS"], p["Kp"], p["sort_passes"]) == (1, 256, 2, 4, 1024, 1)
+    assert p["smem"] <= 232448
+    q = km.plan(km.OP_FIT, 512, 4096, 64, 256, km.BF16)
+    assert (q["pair"], q["BN"], q["XB"], q["CS"], q["Kp"]) == (1, 256, 4, 3, 256)
+    r = km.plan(km.OP_FIT, 1, 16384, 32, 64, km.F32)
+    assert (r["pair"], r["BN"]) == (0, 64)  # pairs need 128-wide tiles
+    assert km.plan(km.OP_FIT, 1, 1 << 22, 128, 16384, km.BF16)["sort_passes"] == 2
+
+
+@pytest.mark.parametrize("tile,ok", [("0,256,2,2", True), ("1,128,3,3", True), ("1,64,2,2", False),
+                                     ("0,256,8,4", False), ("0,256,9,2", False), ("junk", False)])
+def test_tiling_override_is_validated(monkeypatch, tile, ok):
+    monkeypatch.setenv("KM_ASSIGN_TILE", tile)
+    if ok:
+        p = km.plan(km.OP_FIT, 1, 1 << 20, 128, 1024, km.BF16)
+        assert f'{p["pair"]},{p["BN"]},{p["XB"]},{p["CS"]}' == tile
+    else:
+        with pytest.raises(km.KMError):
+            km.plan(km.OP_FIT, 1, 1 << 20, 128, 1024, km.BF16)
+
+
+def test_baseline_workspaces():
+    assert km.library().km_ablation_workspace_size(0, 1 << 20, 128, 1024, km.BF16, 1 << 18) >= (1 << 18) * 1024 * 4
+    assert km.library().km_ablation_workspace_size(1, 1 << 20, 128, 1024, km.BF16, 0) >= 1024 * 128 * 4
+    assert km.library().km_ablation_workspace_size(0, 1 << 20, 128, 1024, km.BF16, 0) == 0  # chunk_rows must be >= 1
