@@ -203,7 +203,7 @@ def run_ours(args, world, rank, local):
     X, C0 = X.contiguous(), C0.contiguous()
     torch.cuda.synchronize()
     # warm-up: W iterations through the same entry point
-    km.fit_profile(X, C0, args.warmup)
+    km.fit_timed(X, C0, args.warmup)
     torch.cuda.synchronize()
     barrier(world)
     stream = torch.cuda.current_stream()
@@ -213,7 +213,7 @@ def run_ours(args, world, rank, local):
         barrier(world)
         l0 = km.launch_count()
         e0.record(stream)
-        r = km.fit_profile(X, C0, args.steps)
+        r = km.fit_timed(X, C0, args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
         launches = km.launch_count() - l0
@@ -221,7 +221,10 @@ def run_ours(args, world, rank, local):
     ms_call = e0.elapsed_time(e1)  # whole call incl. one-time prep and host sync
     ms = r["iters_ms"]             # device time of exactly the timed iterations
     ms_max = max_over_ranks(world, ms)
-    phase = r["phase_ms"]
+    # Phase split from a second fit of the same problem, outside the timed
+    # region: its events between the assignment and the update stop those two
+    # kernels from overlapping their launch, so it is taken apart from `value`.
+    phase = km.fit_profile(X, C0, args.steps)["phase_ms"]
     assign_ms = float(phase[:, 0].mean())
     update_ms = float(phase[:, 1].mean())
     pk, pk_kind = peaks()

@@ -198,6 +198,20 @@ int km_fit_profile(const void* X, const void* C0, int B, int64_t N, int D, int K
                    void* workspace, size_t workspace_bytes, void* stream, float* phase_ms);
 
 /*
+ * km_fit with the device time of its iterations: one CUDA event is recorded
+ * on `stream` right before the first assignment and one after the last
+ * update, nothing between them, so consecutive kernels chain exactly as in
+ * km_fit (programmatic dependent launch lets each kernel of an iteration
+ * become resident while the previous one drains).  Synchronous.
+ *   iters_ms  float, HOST, written: milliseconds from the start of the first
+ *             assignment to the end of the last update.
+ * Other arguments as km_fit.
+ */
+int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
+                 float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist,
+                 void* workspace, size_t workspace_bytes, void* stream, float* iters_ms);
+
+/*
  * Number of kernels this library has enqueued in this process since it was
  * loaded (all entry points, all threads).  For accounting in benchmarks.
  */

@@ -37,7 +37,7 @@ F32, BF16 = 0, 1
 STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_ERR_CUDA",
           4: "KM_ERR_WORKSPACE", 5: "KM_ERR_TIMEOUT"}
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
-           "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_host", "km_selftest_timeout",
+           "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_timed", "km_fit_host", "km_selftest_timeout",
            "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
            "km_ablation_update_atomic", "km_plan_describe", "km_update_accumulate", "km_finalize_sums"]
 
@@ -89,6 +89,7 @@ def library() -> ctypes.CDLL:
             L.km_ablation_assign_materialized.argtypes = [P, P, I64, I, I, I, I64, P, P, P, SZ, P]
             L.km_ablation_update_atomic.argtypes = [P, P, I64, I, I, I, P, P, P, SZ, P]
             L.km_fit_profile.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
+            L.km_fit_timed.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
             L.km_launch_count.restype = ctypes.c_uint64
             L.km_assign_static.argtypes = [P, P, I, I64, I, I, I, P, P, P, P]
             for f in EXPORTS:
@@ -408,6 +409,34 @@ def fit_profile(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, id
                                     _ptr(phase)))
     return dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective,
                 phase_ms=phase[:2 * iters].reshape(iters, 2), iters_ms=float(phase[2 * iters]))
+
+
+def fit_timed(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_out=None, counts_out=None,
+              objective=None, workspace=None, stream=None):
+    """fit() with the device time of its iterations, events around the loop only.
+
+    Synchronous.  Returns the fit() dict plus "iters_ms": device time from
+    the first assignment's start to the last update's end.  Unlike
+    fit_profile, no event sits between the kernels, so they chain as in fit().
+    """
+    _contig_cuda(X, "X"), _contig_cuda(C0, "C0")
+    B, N, D, batched = _shape3(X, "X")
+    Bc, K, Dc, _ = _shape3(C0, "C0")
+    if Bc != B or Dc != D or C0.dtype != X.dtype:
+        raise ValueError("C0 must match X in batch, D and dtype")
+    dt = _dtype_code(X)
+    dev = X.device
+    C_out = torch.empty((B, K, D) if batched else (K, D), dtype=torch.float32, device=dev) if C_out is None else C_out
+    counts_out = torch.empty((B, K) if batched else (K,), dtype=torch.int32, device=dev) \
+        if counts_out is None else counts_out
+    objective = torch.empty((B, iters) if batched else (iters,), dtype=torch.float64, device=dev) \
+        if objective is None else objective
+    ms = ctypes.c_float(0.0)
+    ws = _workspace(OP_FIT, B, N, D, K, dt, dev, workspace)
+    _check(library().km_fit_timed(_ptr(X), _ptr(C0), B, N, D, K, dt, iters, _ptr(C_out), _ptr(idx_out),
+                                  _ptr(counts_out), _ptr(objective), _ptr(ws), ws.numel(), _stream(stream),
+                                  ctypes.byref(ms)))
+    return dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective, iters_ms=float(ms.value))
 
 
 def launch_count() -> int:

@@ -180,6 +180,7 @@ size_t ablation_update_ws(int D, int K) { return 256 + static_cast<size_t>(K) * 
 
 int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int dtype, int64_t chunk_rows,
                     int32_t* idx, float* mindist, void* ws, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   int dev = 0;
   cudaGetDevice(&dev);
   void* h = cublas_handle(dev);
@@ -219,6 +220,7 @@ int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int d
 
 int ablation_update(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, float* C,
                     int32_t* counts, void* ws, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   float* sums = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   if (cudaMemsetAsync(sums, 0, static_cast<size_t>(K) * D * 4, s) != cudaSuccess) return KM_ERR_CUDA;
   if (cudaMemsetAsync(counts, 0, static_cast<size_t>(K) * 4, s) != cudaSuccess) return KM_ERR_CUDA;

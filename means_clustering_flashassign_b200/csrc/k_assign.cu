@@ -281,6 +281,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   if constexpr (PAIR) cluster_sync_all();  // peers' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Everything above touched only this CTA's (pair's) shared memory and
+  // TMEM; from here on the centroid operands, the sort counts and the
+  // objective partials are shared with the previous kernels.  (This kernel
+  // does not signal launch_dependents: the next one becomes resident only as
+  // its CTAs exit, which measured faster than letting it in at the start.)
+  pdl_wait();
   const WaitGuard g{p.status, abort_flag, p.limit_ns};
   const int nct = p.nct;
 
@@ -610,15 +616,31 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles128_per_inst;
   if (grid <= 0) return cudaSuccess;
   count_launch();
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = dim3(static_cast<unsigned>(grid));
+  lc.blockDim = dim3(kAssignThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute la[2];
+  int na = 0;
   if constexpr (PAIR) {
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    e = cudaLaunchKernelEx(&cfg, k_assign<BN, TF32, true, ONE_CT>, *a.xmap, *a.xamap, *a.cmap, *a.camap, k);
-    if (e != cudaSuccess) return e;
-  } else {
-    k_assign<BN, TF32, false, ONE_CT><<<static_cast<unsigned>(grid), kAssignThreads, smem, s>>>(*a.xmap, *a.xamap, *a.cmap,
-                                                                                        *a.camap, k);
+    la[na].id = cudaLaunchAttributeClusterDimension;
+    la[na].val.clusterDim.x = 2;
+    la[na].val.clusterDim.y = 1;
+    la[na].val.clusterDim.z = 1;
+    ++na;
   }
-  return cudaGetLastError();
+  if (pdl_enabled() && chain_armed()) {
+    la[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  lc.attrs = la;
+  lc.numAttrs = na;
+  e = cudaLaunchKernelEx(&lc, k_assign<BN, TF32, PAIR, ONE_CT>, *a.xmap, *a.xamap, *a.cmap, *a.camap, k);
+  if (e == cudaSuccess) chain_arm();
+  else chain_break();
+  return e;
 }
 
 size_t assign_smem_for(int BN, int natoms, int XB, int CS, bool pair) {
@@ -669,6 +691,7 @@ __global__ void k_timeout_probe(unsigned int* status, uint64_t limit_ns) {
 }
 
 cudaError_t launch_timeout_probe(unsigned int* status, uint64_t limit_ns, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   count_launch();
   k_timeout_probe<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();

@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(256) k_xnorm_bf16(const uint8_t* __restrict__ 
 
 cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, void* xaug_v, float* x3,
                          cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   uint8_t* xaug = static_cast<uint8_t*>(xaug_v);
   if (rows <= 0) return cudaSuccess;
   if (dtype == kDtypeBF16) {
@@ -133,6 +134,7 @@ __global__ void k_cprep(const void* __restrict__ src, int src_dtype, int B, int 
 
 cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, int D, int Dp, int dtype,
                          float* master, void* c_op, void* caug, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   const int threads = 256;
   const int64_t warps = static_cast<int64_t>(B) * Kp;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
@@ -162,6 +164,7 @@ __global__ void k_objective(const double* __restrict__ tobj, int64_t per_inst, d
 
 cudaError_t launch_objective(const double* tobj, int B, int64_t groups_per_inst, double* out, int out_stride,
                              cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   count_launch();
   k_objective<<<B, 256, 0, s>>>(tobj, groups_per_inst * 4, out, out_stride);
   return cudaGetLastError();

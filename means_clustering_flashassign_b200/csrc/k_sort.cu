@@ -8,9 +8,10 @@
 //   hist     block b counts the digits of its T keys -> blkhist[digit][b]
 //   colscan  one warp per digit: exclusive scan over blocks (digit-major
 //            order makes the concatenation the stable counting-sort offsets)
-//   scatter  each block scans the digit totals, ranks its keys stably with
-//            per-warp counters (match.any groups equal digits inside a warp)
-//            and writes every element to its final position.
+//   scatter  each block ranks its keys stably with per-warp counters
+//            (ballots group equal digits inside a warp step), scans the
+//            digit totals and its own digit counts, and writes every element
+//            to its final position.
 // The sort is deterministic: equal keys keep point order, so the permutation
 // is unique and the later float sums always run in the same order.
 #include <cstdint>
@@ -35,21 +36,17 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
                                                    int64_t n, int T, int shift, int R, int32_t* __restrict__ blkhist,
                                                    int K) {
   extern __shared__ int32_t sh[];
-  constexpr int kPer = 16;  // keys per thread (T == blockDim.x * kPer)
+  pdl_trigger();
   for (int d = threadIdx.x; d < R; d += blockDim.x) sh[d] = 0;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
-  int dig[kPer];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {  // all loads first, then the counting
-    const int64_t i = t0 + static_cast<int64_t>(j) * blockDim.x + threadIdx.x;
-    int key = 0;
-    if (i < n) key = PAIRS ? pairs[i].y : clamp_key(keys[i], K);
-    dig[j] = i < n ? ((key >> shift) & (R - 1)) : -1;
-  }
+  pdl_wait();
   __syncthreads();
-#pragma unroll
-  for (int j = 0; j < kPer; ++j)
-    if (dig[j] >= 0) atomicAdd(&sh[dig[j]], 1);
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
+  for (int j = threadIdx.x; j < T; j += blockDim.x) {
+    const int64_t i = t0 + j;
+    if (i >= n) break;
+    const int key = PAIRS ? pairs[i].y : clamp_key(keys[i], K);
+    atomicAdd(&sh[(key >> shift) & (R - 1)], 1);
+  }
   __syncthreads();
   int32_t* out = blkhist + static_cast<int64_t>(blockIdx.x) * R;
   for (int d = threadIdx.x; d < R; d += blockDim.x) out[d] = sh[d];
@@ -65,6 +62,8 @@ constexpr int kColscanWarps = 32;
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
                                                                      int64_t nblk, int32_t* __restrict__ total) {
   __shared__ int32_t part[kColscanWarps][32];
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d = blockIdx.x * 32 + lane;
   const bool ok = d < R;
@@ -83,7 +82,9 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
   part[warp][lane] = s;
   __syncthreads();
   int32_t run = 0;
-  for (int w = 0; w < warp; ++w) run += part[w][lane];
+#pragma unroll
+  for (int w = 0; w < kColscanWarps; ++w)
+    if (w < warp) run += part[w][lane];
   if (warp == kColscanWarps - 1 && ok) total[d] = run + s;
   for (int64_t b = b0; b < b1; b += CH) {
     int32_t v[CH];
@@ -97,154 +98,229 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
   }
 }
 
-// Block-wide exclusive scan of total[0..R) into base[0..R) (shared memory;
-// base may alias total): contiguous per-thread runs, a warp-shuffle scan of
-// the run sums, then a scan of the warp sums by warp 0.  tmp needs
-// blockDim.x / 32 ints.
-__device__ void block_exclusive_scan(const int32_t* total, int R, int32_t* base, int32_t* tmp) {
-  const int nt = blockDim.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nt >> 5;
-  const int per = (R + nt - 1) / nt;
-  const int lo = threadIdx.x * per;
-  int32_t s = 0;
-  for (int i = lo; i < lo + per && i < R; ++i) s += total[i];
-  int32_t x = s;
+constexpr int kSortThreads = 256;
+constexpr int kSortWarps = kSortThreads / 32;
+
+// RPT consecutive ints (RPT = 1, 2 or a multiple of 4; p aligned to them).
+template <int RPT>
+__device__ __forceinline__ void ld_run(const int32_t* p, int32_t (&v)[RPT]) {
+  if constexpr (RPT % 4 == 0) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) tmp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t w = lane < nw ? tmp[lane] : 0;
-    int32_t v = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += y;
+    for (int q = 0; q < RPT / 4; ++q) {
+      const int4 x = reinterpret_cast<const int4*>(p)[q];
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
     }
-    if (lane < nw) tmp[lane] = v - w;
+  } else if constexpr (RPT == 2) {
+    const int2 x = *reinterpret_cast<const int2*>(p);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+    v[0] = p[0];
   }
-  __syncthreads();
-  int32_t run = tmp[warp] + x - s;
-  for (int i = lo; i < lo + per && i < R; ++i) {
-    const int32_t t = total[i];
-    base[i] = run;
-    run += t;
-  }
-  __syncthreads();
 }
 
-// Stable scatter of one pass: per-warp counters rank equal digits in point
-// order (match_digit groups equal digits inside a warp step).  The block first
-// places its elements in digit order in shared memory, then writes them out
-// in that order, so elements of one digit leave as one contiguous run at
-// base[d] + (earlier blocks' d).  Writes one 8-byte (point, key) pair per
-// element, and optionally the bare point index (perm_out) on the last pass.
-template <int IPT, bool PAIRS>
-__global__ void k_sort_scatter(const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n,
-                               int T, int shift, int R, int32_t* __restrict__ blkhist,
-                               const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
-                               int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
-  extern __shared__ int32_t sh[];
-  const int W = blockDim.x >> 5;
-  int2* stage = reinterpret_cast<int2*>(sh);   // [T]
-  int32_t* base = sh + 2 * T;                  // [R]  global start of each digit in this block
-  int32_t* lstart = base + R;                  // [R]  block-local start of each digit
-  int32_t* wcnt = lstart + R;                  // [W][R]
-  int32_t* tmp = wcnt + W * R;                 // [blockDim.x / 32]
-  int32_t* bo = tmp + (blockDim.x >> 5);       // [R]  earlier blocks' count of each digit
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
-  int bits = 0;
-  while ((1 << bits) < R) ++bits;
+template <int RPT>
+__device__ __forceinline__ void st_run(int32_t* p, const int32_t (&v)[RPT]) {
+  if constexpr (RPT % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < RPT / 4; ++q)
+      reinterpret_cast<int4*>(p)[q] = make_int4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else if constexpr (RPT == 2) {
+    *reinterpret_cast<int2*>(p) = make_int2(v[0], v[1]);
+  } else {
+    p[0] = v[0];
+  }
+}
+
+// Exclusive scan over the block's threads of two values per thread at once;
+// red holds 2 x kSortWarps ints.  Ends with the block synchronised.
+__device__ __forceinline__ void block_scan_pair(int32_t a, int32_t b, int32_t& ea, int32_t& eb, int32_t* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t x = a, y = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xffffffffu, x, o);
+    const int32_t v = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) {
+      x += u;
+      y += v;
+    }
+  }
+  if (lane == 31) {
+    red[warp] = x;
+    red[kSortWarps + warp] = y;
+  }
+  __syncthreads();
+  int32_t pa = 0, pb = 0;
+#pragma unroll
+  for (int w = 0; w < kSortWarps; ++w)
+    if (w < warp) {
+      pa += red[w];
+      pb += red[kSortWarps + w];
+    }
+  ea = pa + x - a;
+  eb = pb + y - b;
+}
+
+// Stable scatter of one pass, one block per T = 256 * IPT keys.  Warp w
+// takes keys [w T/8, (w+1) T/8) of the block in IPT steps of 32; per-warp
+// counters rank equal digits in point order (match_digit groups equal digits
+// of one step; every step's groups are found before the counter chain, so
+// the chain is one shared load and one store per step).  Thread t owns the
+// RPT digits [t RPT, (t+1) RPT): it scans the digit totals and the block's
+// counts of them (one two-value block scan), turns the per-warp counts into
+// warp offsets inside the digit's block-local run, and keeps the digit's
+// global position minus its local start.  The block then places its keys in
+// digit order in shared memory and writes them out in that order, so the
+// elements of one digit leave as one contiguous run.  Writes one 8-byte
+// (point, key) pair per element, and optionally the bare point index
+// (perm_out) on the last pass; zeroes the block's counts (blkhist row) for
+// the next accumulation.
+template <int IPT, int RPT, bool PAIRS>
+__global__ void __launch_bounds__(kSortThreads, IPT <= 8 ? 4 : 2) k_sort_scatter(
+    const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n, int shift, int R, int bits,
+    int32_t* __restrict__ blkhist, const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
+    int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
+  constexpr int W = kSortWarps;
+  constexpr int T = kSortThreads * IPT;
+  extern __shared__ __align__(16) int32_t sh[];
+  int2* stage = reinterpret_cast<int2*>(sh);  // [T]
+  int32_t* wcnt = sh + 2 * T;                 // [W][R]
+  int32_t* gpos = wcnt + W * R;               // [R] global position of the digit's run minus its local start
+  int32_t* red = gpos + R;                    // [2][W]
+  pdl_trigger();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int d0 = tid * RPT;
+  const bool owner = d0 < R;
+  if (owner) {
+    const int32_t z[RPT] = {};
+#pragma unroll
+    for (int w = 0; w < W; ++w) st_run<RPT>(wcnt + w * R + d0, z);
+  }
+  pdl_wait();
 
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
   const int64_t w0 = t0 + static_cast<int64_t>(warp) * (T / W);
-  int dig[IPT], rank[IPT];
-  int32_t key[IPT], val[IPT];
-  const uint32_t ltm = lanemask_lt();
+  // step s of this lane holds point w0 + 32 s + lane (valid while < n); its
+  // digit is computed from the key where needed
+  const int64_t nw = n - w0 - lane;  // steps s with 32 s < nw are valid
+  auto valid = [&](int s) { return 32 * s < nw; };
+  auto digit = [&](int32_t k) { return (k >> shift) & (R - 1); };
+  int32_t key[IPT], val[PAIRS ? IPT : 1];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {  // all loads first
     const int64_t i = w0 + s * 32 + lane;
-    if (PAIRS) {
+    if constexpr (PAIRS) {
       const int2 pk = i < n ? pairs_in[i] : make_int2(0, 0);
       val[s] = pk.x;
       key[s] = pk.y;
     } else {
-      val[s] = static_cast<int32_t>(i);
       key[s] = i < n ? clamp_key(keys_in[i], K) : 0;
     }
-    dig[s] = i < n ? ((key[s] >> shift) & (R - 1)) : -1;
   }
-  // While the keys are in flight: the digit totals and this block's offsets
-  // into shared memory, per-warp counters zeroed; then the digit bases.
-  for (int d = threadIdx.x; d < R; d += blockDim.x) {
-    base[d] = total[d];
-    bo[d] = boff[d];
+  int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  int32_t tot[RPT] = {}, bo[RPT] = {};
+  if (owner) {
+    ld_run<RPT>(total + d0, tot);
+    ld_run<RPT>(boff + d0, bo);
   }
-  for (int i = threadIdx.x; i < W * R; i += blockDim.x) wcnt[i] = 0;
-  __syncthreads();
-  block_exclusive_scan(base, R, base, tmp);
-  if (start && blockIdx.x == 0) {
-    // single-pass sorts: the digit is the cluster id, so base[] is start[]
-    for (int k = threadIdx.x; k < K; k += blockDim.x) start[k] = base[k];
-    if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
-  }
+  uint32_t peers[IPT];
+#pragma unroll
+  for (int s = 0; s < IPT; ++s) peers[s] = match_digit(digit(key[s]), bits, valid(s));
+  __syncthreads();  // counters zeroed
+
+  const uint32_t ltm = lanemask_lt();
+  int32_t rank[IPT];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
-    const int64_t i = w0 + s * 32 + lane;
-    const bool v = i < n;
-    const uint32_t peers = match_digit(dig[s], bits, v);
-    int before = 0;
-    if (v) before = wcnt[warp * R + dig[s]];
-    rank[s] = before + __popc(peers & ltm);
+    const bool v = valid(s);
+    int32_t* cp = wcnt + warp * R + digit(key[s]);
+    const int32_t before = v ? *cp : 0;
+    rank[s] = before + __popc(peers[s] & ltm);
     __syncwarp();
-    if (v && lane == __ffs(peers) - 1) wcnt[warp * R + dig[s]] = before + __popc(peers);
+    if (v && lane == __ffs(peers[s]) - 1) *cp = before + __popc(peers[s]);
     __syncwarp();
   }
   __syncthreads();
-  // per digit: block count -> block-local starts (scan over digits), then
-  // warp offsets inside the digit's local run
-  for (int d = threadIdx.x; d < R; d += blockDim.x) {
-    int32_t c = 0;
-    for (int w = 0; w < W; ++w) c += wcnt[w * R + d];
-    lstart[d] = c;
-  }
-  __syncthreads();
-  block_exclusive_scan(lstart, R, lstart, tmp);
-  for (int d = threadIdx.x; d < R; d += blockDim.x) {
-    int32_t run = lstart[d];
+
+  // block count of each owned digit, then both scans over the digits
+  int32_t cnt[RPT] = {};
+  if (owner) {
+#pragma unroll
     for (int w = 0; w < W; ++w) {
-      const int32_t c = wcnt[w * R + d];
-      wcnt[w * R + d] = run;
-      run += c;
+      int32_t c[RPT];
+      ld_run<RPT>(wcnt + w * R + d0, c);
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) cnt[j] += c[j];
     }
-    base[d] += bo[d] - lstart[d];  // global position = base[d] + local position
-    boff[d] = 0;  // leave the counts zeroed for the next accumulation
   }
+  int32_t sT = 0, sC = 0;
+#pragma unroll
+  for (int j = 0; j < RPT; ++j) {
+    sT += tot[j];
+    sC += cnt[j];
+  }
+  int32_t eT, eC;
+  block_scan_pair(sT, sC, eT, eC, red);
+  if (owner) {
+    int32_t dbase = eT, lstart = eC;
+    int32_t gp[RPT];
+    int32_t run[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+      // single-pass sorts: the digit is the cluster id, so the digit base is start[]
+      if (start && blockIdx.x == 0 && d0 + j < K) start[d0 + j] = dbase;
+      gp[j] = dbase + bo[j] - lstart;
+      run[j] = lstart;
+      dbase += tot[j];
+      lstart += cnt[j];
+    }
+    st_run<RPT>(gpos + d0, gp);
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      int32_t c[RPT];
+      ld_run<RPT>(wcnt + w * R + d0, c);
+      st_run<RPT>(wcnt + w * R + d0, run);
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) run[j] += c[j];
+    }
+    const int32_t z[RPT] = {};
+    st_run<RPT>(boff + d0, z);  // leave the counts zeroed for the next accumulation
+  }
+  if (start && blockIdx.x == 0 && tid == 0) start[K] = static_cast<int32_t>(n);
   __syncthreads();
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
-    if (dig[s] >= 0) stage[wcnt[warp * R + dig[s]] + rank[s]] = make_int2(val[s], key[s]);
+    const int32_t pt = PAIRS ? val[PAIRS ? s : 0] : static_cast<int32_t>(w0 + s * 32 + lane);
+    if (valid(s)) stage[wcnt[warp * R + digit(key[s])] + rank[s]] = make_int2(pt, key[s]);
   }
   __syncthreads();
-  const int nvalid = static_cast<int>((n - t0) < T ? (n - t0) : T);
-  for (int i = threadIdx.x; i < nvalid; i += blockDim.x) {
-    const int2 pk = stage[i];
-    const int64_t pos = static_cast<int64_t>(base[(pk.y >> shift) & (R - 1)]) + i;
-    // Counts accumulated elsewhere (the assignment kernel) agree with these
-    // keys unless that kernel gave up on a bounded wait; stay in bounds then.
-    if (pos < 0 || pos >= n) continue;
-    pairs_out[pos] = pk;
-    if (perm_out) perm_out[pos] = pk.x;
+  const int64_t left = n - t0;
+  const int nvalid = static_cast<int>(left < T ? left : T);
+#pragma unroll
+  for (int s = 0; s < IPT; ++s) {
+    const int i = s * kSortThreads + tid;
+    if (i < nvalid) {
+      const int2 pk = stage[i];
+      const int64_t pos = static_cast<int64_t>(gpos[(pk.y >> shift) & (R - 1)]) + i;
+      // Counts accumulated elsewhere (the assignment kernel) agree with these
+      // keys unless that kernel gave up on a bounded wait; stay in bounds then.
+      if (pos >= 0 && pos < n) {
+        pairs_out[pos] = pk;
+        if (perm_out) perm_out[pos] = pk.x;
+      }
+    }
   }
 }
 
 // start[k] for every k in [0, K] from the sorted pairs: each change point i
 // (or the ends) writes the starts of all clusters between the two keys.
 __global__ void k_bounds(const int2* __restrict__ sorted, int64_t n, int K, int32_t* __restrict__ start) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i > n) return;
   const int a = i == 0 ? -1 : clamp_key(sorted[i - 1].y, K);
@@ -252,53 +328,88 @@ __global__ void k_bounds(const int2* __restrict__ sorted, int64_t n, int K, int3
   for (int k = a + 1; k <= c; ++k) start[k] = static_cast<int32_t>(i);
 }
 
-static size_t scatter_smem(int R, int W, int threads, int T) {
-  return (2 * static_cast<size_t>(T) + 3 * static_cast<size_t>(R) + static_cast<size_t>(W) * R + threads) * 4;
+// Digits per scatter thread for radix R: R / 256, at least 1.
+static int scatter_rpt(int R) { return R <= kSortThreads ? 1 : R / kSortThreads; }
+
+static size_t scatter_smem(int R, int T) {
+  return (2 * static_cast<size_t>(T) + static_cast<size_t>(kSortWarps + 1) * R + 2 * kSortWarps) * 4;
+}
+
+template <int IPT, int RPT, bool PAIRS>
+static cudaError_t launch_scatter_t(int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys, const int2* pin,
+                                    int64_t n, int shift, int R, int bits, int32_t* bh, const int32_t* total,
+                                    int2* out, int32_t* perm, int32_t* st, int K) {
+  auto kern = k_sort_scatter<IPT, RPT, PAIRS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+  if (e != cudaSuccess) return e;
+  return launch_chained(kern, dim3(static_cast<unsigned>(nblk)), dim3(kSortThreads), sm, s, keys, pin, n, shift, R,
+                        bits, bh, total, out, perm, st, K);
+}
+
+template <int IPT, bool PAIRS>
+static cudaError_t launch_scatter_r(int rpt, int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys,
+                                    const int2* pin, int64_t n, int shift, int R, int bits, int32_t* bh,
+                                    const int32_t* total, int2* out, int32_t* perm, int32_t* st, int K) {
+  switch (rpt) {
+    case 1: return launch_scatter_t<IPT, 1, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 2: return launch_scatter_t<IPT, 2, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 4: return launch_scatter_t<IPT, 4, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 8: return launch_scatter_t<IPT, 8, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 16: return launch_scatter_t<IPT, 16, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
   const SortCfg& c = p.sc;
-  const int threads = c.W * 32;
   const int64_t nblk = (a.n + c.T - 1) / c.T;
   if (a.n <= 0) return cudaSuccess;
+  if (c.T != kSortThreads * c.IPT || (c.IPT != 8 && c.IPT != 16)) return cudaErrorInvalidValue;
+  cudaError_t e;
   for (int ps = 0; ps < c.passes; ++ps) {
-    const int R = 1 << c.bits[ps];
+    const int bits = c.bits[ps];
+    const int R = 1 << bits;
     const bool last = ps == c.passes - 1;
     const bool pairs_in = ps > 0;
     int32_t* bh = ps == 0 ? a.blkhist : a.blkhist1;
     count_launch(ps == 0 && a.hist0_ready ? 2 : 3);  // [hist,] colscan, scatter
+    const dim3 hgrid(static_cast<unsigned>(nblk));
     if (pairs_in)
-      k_sort_hist<true><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps],
-                                                                        R, bh, a.K);
+      e = launch_chained(k_sort_hist<true>, hgrid, dim3(256), R * 4, s, nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps],
+                         R, bh, a.K);
     else if (!a.hist0_ready)
-      k_sort_hist<false><<<static_cast<unsigned>(nblk), 256, R * 4, s>>>(a.keys, nullptr, a.n, c.T, c.shift[ps], R,
-                                                                         bh, a.K);
-    k_sort_colscan<<<(R + 31) / 32, kColscanWarps * 32, 0, s>>>(bh, R, nblk, a.total);
+      e = launch_chained(k_sort_hist<false>, hgrid, dim3(256), R * 4, s, a.keys, nullptr, a.n, c.T, c.shift[ps], R,
+                         bh, a.K);
+    else
+      e = cudaSuccess;
+    if (e != cudaSuccess) return e;
+    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32), dim3(kColscanWarps * 32), 0, s, bh, R, nblk, a.total);
+    if (e != cudaSuccess) return e;
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
     int2* out = last ? a.pairs : a.pairs_tmp;
     int32_t* perm = last ? a.perm : nullptr;
-    const size_t sm = scatter_smem(R, c.W, threads, c.T);
+    const size_t sm = scatter_smem(R, c.T);
     int32_t* st = (last && c.passes == 1) ? a.start : nullptr;
-    cudaError_t e;
-    if (pairs_in) {
-      e = cudaFuncSetAttribute(k_sort_scatter<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sm));
-      if (e != cudaSuccess) return e;
-      k_sort_scatter<16, true><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
-          nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps], R, bh, a.total, out, perm, st, a.K);
-    } else {
-      e = cudaFuncSetAttribute(k_sort_scatter<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sm));
-      if (e != cudaSuccess) return e;
-      k_sort_scatter<16, false><<<static_cast<unsigned>(nblk), threads, sm, s>>>(
-          a.keys, nullptr, a.n, c.T, c.shift[ps], R, bh, a.total, out, perm, st, a.K);
-    }
+    const int rpt = scatter_rpt(R);
+    if (pairs_in)
+      e = c.IPT == 16 ? launch_scatter_r<16, true>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R, bits,
+                                                   bh, a.total, out, perm, st, a.K)
+                      : launch_scatter_r<8, true>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R, bits,
+                                                  bh, a.total, out, perm, st, a.K);
+    else
+      e = c.IPT == 16 ? launch_scatter_r<16, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R, bits, bh,
+                                                    a.total, out, perm, st, a.K)
+                      : launch_scatter_r<8, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R, bits, bh,
+                                                   a.total, out, perm, st, a.K);
+    if (e != cudaSuccess) return e;
   }
   if (c.passes > 1) {
     const int64_t cnt = a.n + 1;
     count_launch();
-    k_bounds<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(a.pairs, a.n, a.K, a.start);
+    e = launch_chained(k_bounds, dim3(static_cast<unsigned>((cnt + 255) / 256)), dim3(256), 0, s, a.pairs, a.n, a.K,
+                       a.start);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

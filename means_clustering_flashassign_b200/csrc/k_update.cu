@@ -243,6 +243,8 @@ __global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X
                                                    float* __restrict__ sums, float* __restrict__ pl,
                                                    float* __restrict__ pr) {
   extern __shared__ float sm[];
+  pdl_trigger();
+  pdl_wait();
   constexpr int W = 8;
   int* slot_k = reinterpret_cast<int*>(sm);          // [W][2]
   float* slot_v = sm + 2 * W;                         // [W][2][D]
@@ -294,15 +296,10 @@ static cudaError_t launch_segsum_t(const Plan& p, const SegArgs& a, cudaStream_t
   const int64_t nch = (a.n + P - 1) / P;
   const size_t sm = (2 * 8 + 2 * 8 * static_cast<size_t>(p.D)) * 4;
   count_launch();
-  if (p.dtype == kDtypeBF16)
-    k_segsum<LPR, true><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
-                                                                    row_bytes, a.pairs, p.K, a.start, P, a.sums,
-                                                                    a.pl, a.pr);
-  else
-    k_segsum<LPR, false><<<static_cast<unsigned>(nch), 256, sm, s>>>(static_cast<const uint8_t*>(a.X), a.n, p.D,
-                                                                     row_bytes, a.pairs, p.K, a.start, P, a.sums,
-                                                                     a.pl, a.pr);
-  return cudaGetLastError();
+  auto kern = p.dtype == kDtypeBF16 ? k_segsum<LPR, true> : k_segsum<LPR, false>;
+  return launch_chained(kern, dim3(static_cast<unsigned>(nch)), dim3(256), sm, s,
+                        static_cast<const uint8_t*>(a.X), a.n, p.D, row_bytes, a.pairs, p.K, a.start, P, a.sums,
+                        a.pl, a.pr);
 }
 
 static int lanes_per_row(int row_bytes) {
@@ -430,9 +427,12 @@ __device__ void finish_cluster(const FinK& f, int k, int64_t cnt, float (&sum)[8
 
 __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
   extern __shared__ float fsm[];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && f.ntiles > 0) {
-    // objective of this pass: fixed-order reduction of the assign partials
+  if (blockIdx.x == gridDim.x - 1 && f.ntiles > 0) {
+    // the last block: objective of this pass, a fixed-order reduction of the
+    // assign partials
     double* red = reinterpret_cast<double*>(fsm);
     double s = 0.0;
     for (int64_t i = threadIdx.x; i < f.ntiles * 4; i += blockDim.x) s += f.tobj[i];
@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
       if (f.mode == 0) *f.obj = red[0];
       else *f.obj += red[0];
     }
-    __syncthreads();
+    return;
   }
   if (blockIdx.x < f.nwarp_blocks) {
     const int k = static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + warp;
@@ -560,7 +560,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.nwarp_blocks = (p.K + 15) / 16;
   const int64_t G = static_cast<int64_t>(p.gc.big_span) * f.BNS;
   const int64_t nbig = (p.rows + G - 1) / G;
-  // block 0: 512 doubles of objective reduction (1024 floats) + 16 warp rows;
+  // objective block: 512 doubles (1024 floats); warp blocks: 16 warp rows;
   // big-cluster blocks: slices x D partial rows + one summed row.
   const size_t fl_warp = 1024 + 16 * static_cast<size_t>(p.D);
   const size_t fl_big = 2048 + 2 * static_cast<size_t>(p.D);
@@ -569,8 +569,9 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
                                        static_cast<int>(sm));
   if (e != cudaSuccess) return e;
   count_launch();
-  k_finalize<<<static_cast<unsigned>(f.nwarp_blocks + nbig), threads, sm, s>>>(f);
-  return cudaGetLastError();
+  const int64_t nobj = f.ntiles > 0 ? 1 : 0;
+  return launch_chained(k_finalize, dim3(static_cast<unsigned>(f.nwarp_blocks + nbig + nobj)), dim3(threads), sm, s,
+                        f);
 }
 
 // Out-of-core: float64 accumulators -> centroids; resets the accumulators.
@@ -626,6 +627,7 @@ __global__ void k_finalize_sums(const double* __restrict__ sums, const long long
 
 cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const long long* cnt, float* C,
                                  void* C_lp, int32_t* counts, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   const int64_t e = static_cast<int64_t>(K) * D;
   count_launch();
   k_finalize_sums<<<static_cast<unsigned>((e + 255) / 256), 256, 0, s>>>(sums, cnt, K, D, dtype, C, C_lp, counts);
@@ -634,6 +636,7 @@ cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, co
 
 cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, float* C, void* c_op, void* caug,
                                 int32_t* counts, double* objacc, double* obj_out, cudaStream_t s) {
+  chain_break();  // plain launch: the next kernel must not chain to it
   const int threads = 256;
   const int blocks = (p.K + 7) / 8;
   count_launch();
@@ -745,6 +748,8 @@ __device__ __forceinline__ float emit_operand_lpr(const float (&q)[8], int row_b
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   extern __shared__ __align__(16) int32_t ssm[];
+  pdl_trigger();
+  pdl_wait();
   constexpr int W = 8;
   const int N = static_cast<int>(p.N), K = p.K, D = p.D;
   // 16-byte aligned pieces first: slot vectors, the double reduction buffer,
@@ -941,14 +946,14 @@ static cudaError_t launch_small_t(const Plan& p, const SmallUpdateArgs& a, cudaS
     e = cudaFuncSetAttribute(k_small_update<LPR, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sm));
     if (e != cudaSuccess) return e;
-    k_small_update<LPR, true><<<p.B, 256, sm, s>>>(k);
+    e = launch_chained(k_small_update<LPR, true>, dim3(p.B), dim3(256), sm, s, k);
   } else {
     e = cudaFuncSetAttribute(k_small_update<LPR, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sm));
     if (e != cudaSuccess) return e;
-    k_small_update<LPR, false><<<p.B, 256, sm, s>>>(k);
+    e = launch_chained(k_small_update<LPR, false>, dim3(p.B), dim3(256), sm, s, k);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_small_update(const Plan& p, const SmallUpdateArgs& a, cudaStream_t s) {

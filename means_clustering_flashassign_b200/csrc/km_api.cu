@@ -27,6 +27,16 @@ int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int d
 int ablation_update(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, float* C,
                     int32_t* counts, void* ws, cudaStream_t s);
 size_t small_update_smem(int64_t N, int K, int D);
+
+bool pdl_enabled() {
+  const char* e = getenv("KM_PDL");
+  return !(e && strcmp(e, "0") == 0);
+}
+
+static thread_local bool t_chain = false;
+void chain_break() { t_chain = false; }
+bool chain_armed() { return t_chain; }
+void chain_arm() { t_chain = true; }
 }  // namespace km
 
 using namespace km;
@@ -265,7 +275,13 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     sc.shift[1] = sc.bits[0];
   }
   sc.W = 8;
-  sc.IPT = 16;
+  // Keys per scatter block: 4096 when those blocks fill the 148 SMs with one
+  // to two resident blocks each (one wave at 2 per SM), else 2048 (4 per SM):
+  // measured faster for 16K and 4M points, slower for 1M.
+  {
+    const int64_t b4k = (p.rows + 4095) / 4096;
+    sc.IPT = b4k >= 148 && b4k <= 2 * 148 ? 16 : 8;
+  }
   sc.T = sc.W * 32 * sc.IPT;
   sc.nblk = (p.rows + sc.T - 1) / sc.T;
   sc.Rmax = 1 << (sc.bits[0] > sc.bits[1] ? sc.bits[0] : sc.bits[1]);
@@ -346,6 +362,7 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
   if (r != KM_OK) return r;
   c.ws = ws;
   c.s = static_cast<cudaStream_t>(stream);
+  chain_break();
   return KM_OK;
 }
 
@@ -433,8 +450,10 @@ int km_workspace_status(void* workspace, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int v = 0;
   KM_CUDA(cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s));
+  chain_break();
   KM_CUDA(cudaStreamSynchronize(s));
   KM_CUDA(cudaMemsetAsync(workspace, 0, sizeof(v), s));
+  chain_break();
   KM_CUDA(cudaStreamSynchronize(s));
   if (v) return fail(KM_ERR_TIMEOUT, "a kernel gave up on a bounded wait (status 0x%x)", v);
   return KM_OK;
@@ -454,6 +473,7 @@ int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int 
   void* clp = at<void>(c.ws, p.off_clp);
   const bool f32 = dtype == KM_F32;
   KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+  chain_break();
   float* x3 = f32 ? at<float>(c.ws, p.off_x3) : nullptr;
   KM_CUDA(launch_xprep(X, dtype, static_cast<int64_t>(B) * N, D, p.Dp, xaug, x3, c.s));
   KM_CUDA(launch_cprep(C, dtype, B, K, p.Kp, D, p.Dp, dtype, nullptr, clp, caug, c.s));
@@ -497,7 +517,7 @@ int km_update(const void* X, const int32_t* idx, int B, int64_t N, int D, int K,
 
 static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
                     float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
-                    size_t workspace_bytes, void* stream, cudaEvent_t* ev) {
+                    size_t workspace_bytes, void* stream, cudaEvent_t* ev, bool per_phase = true) {
   if (!X || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X, C0 and C_out are required");
   if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
   if (!aligned16(X) || !aligned16(C0) || !aligned16(C_out))
@@ -514,6 +534,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   double* objs = at<double>(c.ws, p.off_obj);
   const bool f32 = dtype == KM_F32;
   KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+  chain_break();
   float* x3 = f32 ? at<float>(c.ws, p.off_x3) : nullptr;
   KM_CUDA(launch_xprep(X, dtype, static_cast<int64_t>(B) * N, D, p.Dp, xaug, x3, c.s));
   CUtensorMap xmap, xamap, cmap, camap;
@@ -530,13 +551,20 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   int32_t* hist0 = fused_hist ? at<int32_t>(c.ws, p.off_blkhist) : nullptr;
   if (fused_hist)
     KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
+  chain_break();
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
                  &groups, hist0, p.sc.T, 1 << p.sc.bits[0]};
-    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t], c.s));
+    if (ev && (per_phase || t == 0)) {
+      KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t : 0], c.s));
+      chain_break();
+    }
     KM_CUDA(launch_assign(p, a, c.s));
-    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
+    if (ev && per_phase) {
+      KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
+      chain_break();
+    }
     if (p.small_update) {
       SmallUpdateArgs u{X,    idx,       C_out, clp, caug, counts_out, tobj, p.tiles_per_inst,
                         objective_hist ? objective_hist + t : objs, objective_hist ? iters : 1};
@@ -552,7 +580,10 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
         if (r != KM_OK) return r;
       }
     }
-    if (ev) KM_CUDA(cudaEventRecord(ev[3 * t + 2], c.s));
+    if (ev && (per_phase || t == iters - 1)) {
+      KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t + 2 : 1], c.s));
+      chain_break();
+    }
   }
   return KM_OK;
 }
@@ -601,6 +632,30 @@ int km_fit_profile(const void* X, const void* C0, int B, int64_t N, int D, int K
   return r;
 }
 
+int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters, float* C_out,
+                 int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
+                 size_t workspace_bytes, void* stream, float* iters_ms) {
+  g_err.clear();
+  if (!iters_ms) return fail(KM_ERR_INVALID_ARG, "iters_ms is required");
+  if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  cudaEvent_t ev[2] = {nullptr, nullptr};
+  for (auto& e : ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (auto x : ev)
+        if (x) cudaEventDestroy(x);
+      return fail(KM_ERR_CUDA, "cudaEventCreate failed");
+    }
+  int r = fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
+                   workspace_bytes, stream, iters > 0 ? ev : nullptr, false);
+  if (r == KM_OK && cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    r = fail(KM_ERR_CUDA, "stream synchronisation failed");
+  *iters_ms = 0.f;
+  if (r == KM_OK && iters > 0 && cudaEventElapsedTime(iters_ms, ev[0], ev[1]) != cudaSuccess)
+    r = fail(KM_ERR_CUDA, "cudaEventElapsedTime failed");
+  for (auto e : ev) cudaEventDestroy(e);
+  return r;
+}
+
 int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int dtype, int iters, int64_t chunk_rows,
                 float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
                 size_t workspace_bytes, void* stream) {
@@ -643,13 +698,21 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
       KM_CUDA(cudaEventCreateWithFlags(&ev_free[i], cudaEventDisableTiming));
     }
     KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+    chain_break();
     KM_CUDA(cudaMemsetAsync(acc64, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
+    chain_break();
     KM_CUDA(cudaMemsetAsync(cnt64, 0, sizeof(long long) * K, c.s));
+    chain_break();
     KM_CUDA(cudaMemsetAsync(objacc, 0, sizeof(double), c.s));
+    chain_break();
     KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
     int32_t* hist0 = at<int32_t>(c.ws, p.off_blkhist);
     KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
-    for (int i = 0; i < 2; ++i) KM_CUDA(cudaEventRecord(ev_free[i], c.s));
+    chain_break();
+    for (int i = 0; i < 2; ++i) {
+      KM_CUDA(cudaEventRecord(ev_free[i], c.s));
+      chain_break();
+    }
     const bool f32 = dtype == KM_F32;
     CUtensorMap cmap, camap;
     int rr = encode_map(&cmap, clp, f32, p.Dop, K, 1, cbox(p));
@@ -664,10 +727,14 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         const int64_t r0 = ch * p.chunk_rows;
         const int64_t nr = N - r0 < p.chunk_rows ? N - r0 : p.chunk_rows;
         KM_CUDA(cudaStreamWaitEvent(cs, ev_free[bi], 0));
+        chain_break();
         KM_CUDA(cudaMemcpyAsync(dbuf[bi], static_cast<const uint8_t*>(X_host) + r0 * rowb, nr * rowb,
                                 cudaMemcpyHostToDevice, cs));
+        chain_break();
         KM_CUDA(cudaEventRecord(ev_copied[bi], cs));
+        chain_break();
         KM_CUDA(cudaStreamWaitEvent(c.s, ev_copied[bi], 0));
+        chain_break();
         CUtensorMap xmap, xamap;
         KM_CUDA(launch_xprep(dbuf[bi], dtype, nr, D, p.Dp, xaug, x3, c.s));
         rr = encode_map(&xmap, f32 ? static_cast<const void*>(x3) : dbuf[bi], f32, p.Dop, nr, 1, kTileM);
@@ -689,6 +756,7 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
                              true);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
+        chain_break();
       }
       KM_CUDA(launch_finalize_acc(p, acc64, cnt64, C_out, clp, caug, counts_out, objacc, objs + t, c.s));
     }
@@ -736,7 +804,9 @@ int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, in
   if (r != KM_OK) return r;
   if (zero_first) {
     KM_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
+    chain_break();
     KM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int64_t) * K, c.s));
+    chain_break();
   }
   return update_instance(c, X, idx, N, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 1, false, sums,
                          reinterpret_cast<long long*>(counts));
@@ -837,6 +907,7 @@ int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_n
   if (r != KM_OK) return r;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   KM_CUDA(cudaMemsetAsync(workspace, 0, sizeof(unsigned int), s));
+  chain_break();
   KM_CUDA(launch_timeout_probe(static_cast<unsigned int*>(workspace), static_cast<uint64_t>(limit_ns), s));
   return km_workspace_status(workspace, s);
 }

@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -55,6 +56,42 @@ struct SegCfg {
   int64_t nchunks = 0;
   int big_span = 8;   // clusters spanning more chunks than this use a whole block in finalize
 };
+
+// Programmatic dependent launch for the kernels of one Lloyd iteration: a
+// kernel launched this way may become resident while the previous kernel of
+// the stream drains, and runs griddepcontrol.wait (pdl_wait) in every thread
+// before it reads or writes anything an earlier kernel touches.  KM_PDL=0 in
+// the environment launches them with plain stream order instead.
+bool pdl_enabled();
+
+// Chaining state of the calling thread's stream.  Only a kernel whose
+// immediate predecessor on the stream is one of this library's chained
+// kernels gets the programmatic attribute: launch_chained (and the
+// assignment launcher) arm the state after enqueueing, and every other
+// stream operation -- entry into the library, a memset, a copy, an event, a
+// plain kernel launch -- breaks it.
+void chain_break();
+bool chain_armed();
+void chain_arm();
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() && chain_armed() ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e == cudaSuccess) chain_arm();
+  else chain_break();
+  return e;
+}
 
 // Sorted positions per segmented-sum block for n positions: the blocks form
 // one wave (148 SMs x 4 resident blocks), each a multiple of 256 positions.
