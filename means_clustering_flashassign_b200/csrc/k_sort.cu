@@ -56,8 +56,7 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
 // digit totals.  A block takes 32 digits (one per lane, so every load is
 // coalesced) and splits the block range among its 32 warps: each warp sums
 // its part, the parts are scanned in shared memory, and each warp rewrites
-// its part as running prefixes.  (Up to 8K blocks the parts are at most 8
-// rows: one batch of loads per warp.)
+// its part as running prefixes.
 constexpr int kColscanWarps = 32;
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
                                                                      int64_t nblk, int32_t* __restrict__ total) {
@@ -70,15 +69,22 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
   const int64_t seg = (nblk + kColscanWarps - 1) / kColscanWarps;
   const int64_t b0 = warp * seg < nblk ? warp * seg : nblk;
   const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
-  constexpr int CH = 8;
+  // The first KEEP rows of the warp's part stay in registers for the second
+  // pass (all of it up to 512 blocks); rows beyond are read again.
+  constexpr int KEEP = 16, CH = 8;
+  int32_t keep[KEEP];
+#pragma unroll
+  for (int u = 0; u < KEEP; ++u) keep[u] = (ok && b0 + u < b1) ? blkhist[(b0 + u) * R + d] : 0;
   int32_t s = 0;
-  for (int64_t b = b0; b < b1; b += CH) {
+  for (int64_t b = b0 + KEEP; b < b1; b += CH) {
     int32_t v[CH];
 #pragma unroll
     for (int u = 0; u < CH; ++u) v[u] = (ok && b + u < b1) ? blkhist[(b + u) * R + d] : 0;
 #pragma unroll
     for (int u = 0; u < CH; ++u) s += v[u];
   }
+#pragma unroll
+  for (int u = 0; u < KEEP; ++u) s += keep[u];
   part[warp][lane] = s;
   __syncthreads();
   int32_t run = 0;
@@ -86,7 +92,12 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
   for (int w = 0; w < kColscanWarps; ++w)
     if (w < warp) run += part[w][lane];
   if (warp == kColscanWarps - 1 && ok) total[d] = run + s;
-  for (int64_t b = b0; b < b1; b += CH) {
+#pragma unroll
+  for (int u = 0; u < KEEP; ++u) {
+    if (ok && b0 + u < b1) blkhist[(b0 + u) * R + d] = run;
+    run += keep[u];
+  }
+  for (int64_t b = b0 + KEEP; b < b1; b += CH) {
     int32_t v[CH];
 #pragma unroll
     for (int u = 0; u < CH; ++u) v[u] = (ok && b + u < b1) ? blkhist[(b + u) * R + d] : 0;
@@ -179,8 +190,10 @@ __device__ __forceinline__ void block_scan_pair(int32_t a, int32_t b, int32_t& e
 // (point, key) pair per element, and optionally the bare point index
 // (perm_out) on the last pass; zeroes the block's counts (blkhist row) for
 // the next accumulation.
+// Resident blocks per SM the register budget is sized for: what the shared
+// memory (2T + 9R ints) admits, 1 to 4.
 template <int IPT, int RPT, bool PAIRS>
-__global__ void __launch_bounds__(kSortThreads, IPT <= 8 ? 4 : 2) k_sort_scatter(
+__global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT < 8 ? 4 : 2)) k_sort_scatter(
     const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n, int shift, int R, int bits,
     int32_t* __restrict__ blkhist, const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
     int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
@@ -199,6 +212,17 @@ __global__ void __launch_bounds__(kSortThreads, IPT <= 8 ? 4 : 2) k_sort_scatter
     const int32_t z[RPT] = {};
 #pragma unroll
     for (int w = 0; w < W; ++w) st_run<RPT>(wcnt + w * R + d0, z);
+  }
+  {
+    // While the previous kernel drains: pull this block's keys into L2 (the
+    // assignment vector is written early in the assignment kernel and partly
+    // evicted by the point stream that follows).
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * T;
+    const int64_t line = first + static_cast<int64_t>(tid) * (PAIRS ? 16 : 32);
+    if (tid < T / (PAIRS ? 16 : 32) && line < n) {
+      if (PAIRS) prefetch_l2(pairs_in + line);
+      else prefetch_l2(keys_in + line);
+    }
   }
   pdl_wait();
 
@@ -227,9 +251,11 @@ __global__ void __launch_bounds__(kSortThreads, IPT <= 8 ? 4 : 2) k_sort_scatter
     ld_run<RPT>(total + d0, tot);
     ld_run<RPT>(boff + d0, bo);
   }
+  // digit bits: R = 256 RPT exactly when RPT > 1; at most 8 when RPT == 1
+  constexpr int NB = RPT == 1 ? 8 : RPT == 2 ? 9 : RPT == 4 ? 10 : RPT == 8 ? 11 : 12;
   uint32_t peers[IPT];
 #pragma unroll
-  for (int s = 0; s < IPT; ++s) peers[s] = match_digit(digit(key[s]), bits, valid(s));
+  for (int s = 0; s < IPT; ++s) peers[s] = match_digit<NB>(digit(key[s]), bits, valid(s));
   __syncthreads();  // counters zeroed
 
   const uint32_t ltm = lanemask_lt();
@@ -292,26 +318,33 @@ __global__ void __launch_bounds__(kSortThreads, IPT <= 8 ? 4 : 2) k_sort_scatter
   }
   if (start && blockIdx.x == 0 && tid == 0) start[K] = static_cast<int32_t>(n);
   __syncthreads();
+  // all slot lookups, then all stores (they do not wait on each other)
+#pragma unroll
+  for (int s = 0; s < IPT; ++s) rank[s] = valid(s) ? wcnt[warp * R + digit(key[s])] + rank[s] : -1;
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int32_t pt = PAIRS ? val[PAIRS ? s : 0] : static_cast<int32_t>(w0 + s * 32 + lane);
-    if (valid(s)) stage[wcnt[warp * R + digit(key[s])] + rank[s]] = make_int2(pt, key[s]);
+    if (rank[s] >= 0) stage[rank[s]] = make_int2(pt, key[s]);
   }
   __syncthreads();
   const int64_t left = n - t0;
   const int nvalid = static_cast<int>(left < T ? left : T);
+  // staged elements in order, then their run positions, then the stores
+  int2 pk[IPT];
+  int32_t gp[IPT];
+#pragma unroll
+  for (int s = 0; s < IPT; ++s) pk[s] = s * kSortThreads + tid < nvalid ? stage[s * kSortThreads + tid] : make_int2(0, 0);
+#pragma unroll
+  for (int s = 0; s < IPT; ++s) gp[s] = gpos[digit(pk[s].y)];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int i = s * kSortThreads + tid;
-    if (i < nvalid) {
-      const int2 pk = stage[i];
-      const int64_t pos = static_cast<int64_t>(gpos[(pk.y >> shift) & (R - 1)]) + i;
-      // Counts accumulated elsewhere (the assignment kernel) agree with these
-      // keys unless that kernel gave up on a bounded wait; stay in bounds then.
-      if (pos >= 0 && pos < n) {
-        pairs_out[pos] = pk;
-        if (perm_out) perm_out[pos] = pk.x;
-      }
+    const int64_t pos = static_cast<int64_t>(gp[s]) + i;
+    // Counts accumulated elsewhere (the assignment kernel) agree with these
+    // keys unless that kernel gave up on a bounded wait; stay in bounds then.
+    if (i < nvalid && pos >= 0 && pos < n) {
+      pairs_out[pos] = pk[s];
+      if (perm_out) perm_out[pos] = pk[s].x;
     }
   }
 }

@@ -322,6 +322,10 @@ cudaError_t launch_segsum(const Plan& p, const SegArgs& a, cudaStream_t s) {
 }
 
 // --------------------------------------------------------------- finalize
+// Largest number of segmented-sum chunk boundaries a cluster may cross and
+// still be finalised by one warp (more: a whole block).
+constexpr int kBigSpan = 8;
+
 struct FinK {
   int K, D, Dp, dtype, BNS, big_span;
   int64_t n, nwarp_blocks;
@@ -472,8 +476,16 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
           if (ca == cb) {
             v[i] = w[i];
           } else {
-            float a = f.pr[ca * f.D + j];
-            for (int64_t c = ca + 1; c <= cb; ++c) a += f.pl[c * f.D + j];
+            // the pieces (right end of chunk ca, left ends of ca+1..cb) are
+            // loaded together, then added in chunk order
+            float pc[kBigSpan + 1];
+#pragma unroll
+            for (int q = 0; q <= kBigSpan; ++q)
+              pc[q] = ca + q <= cb ? (q == 0 ? f.pr : f.pl)[(ca + q) * f.D + j] : 0.f;
+            float a = pc[0];
+#pragma unroll
+            for (int q = 1; q <= kBigSpan; ++q)
+              if (ca + q <= cb) a += pc[q];
             v[i] = a;
           }
         }
@@ -539,7 +551,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.Dp = p.Dp;
   f.dtype = p.dtype;
   f.BNS = static_cast<int>(seg_block_positions(p.rows));
-  f.big_span = p.gc.big_span;
+  f.big_span = p.gc.big_span < kBigSpan ? p.gc.big_span : kBigSpan;
   f.n = p.rows;
   f.start = a.start;
   f.pairs = a.pairs;
@@ -797,7 +809,7 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
     const int i = i0 + lane;
     const bool v = i < N && i < (warp + 1) * Lw;
     const int d = v ? static_cast<int>(kr[i]) : -1;
-    const uint32_t peers = match_digit(d, bits, v);
+    const uint32_t peers = match_digit<10>(d, bits, v);  // K <= kSmallMaxK = 1024
     int before = 0;
     if (v) before = wcnt[warp * K + d];
     if (v) kr[i] = static_cast<uint32_t>(d) | (static_cast<uint32_t>(before + __popc(peers & ltm)) << 16);

@@ -25,6 +25,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Lets the next kernel of the stream be scheduled (it still waits in
 // pdl_wait for this grid to finish).
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Brings the 128-byte line holding p into L2.  A hint only: no data comes
+// back, so it may be issued before pdl_wait for data an earlier kernel of the
+// chain finished writing (the later loads still follow the wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
 // Blocks until the grids this one depends on have completed and their
 // memory is visible; returns at once for a kernel launched without the
 // programmatic-serialization attribute.
@@ -210,17 +216,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // Lanes of the warp holding the same digit as this lane (the low `bits` bits
-// compared), among the lanes with `valid` set: one ballot per digit bit, each
-// lane keeping the lanes that agree with it on that bit.  Same result as a
-// match.any over the digits of the valid lanes, at a few cycles per bit.
+// compared, bits <= NB), among the lanes with `valid` set: one ballot per
+// possible digit bit, each lane keeping the lanes that agree with it on that
+// bit.  Bits at or above `bits` are masked out by a select, not a branch, so
+// the NB ballots do not depend on each other and issue back to back (and
+// those of several calls interleave).  Same result as a match.any over the
+// digits of the valid lanes.
+template <int NB>
 __device__ __forceinline__ uint32_t match_digit(int dig, int bits, bool valid) {
   uint32_t m = __ballot_sync(0xffffffffu, valid);
-#pragma unroll 12
-  for (int b = 0; b < 12; ++b) {
-    if (b >= bits) break;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
     const bool set = (dig >> b) & 1;
     const uint32_t bb = __ballot_sync(0xffffffffu, set);
-    m &= set ? bb : ~bb;
+    const uint32_t agree = set ? bb : ~bb;
+    m &= b < bits ? agree : 0xffffffffu;
   }
   return m;
 }
