@@ -50,7 +50,7 @@ def peaks():
 # used only while these files are unchanged.
 KERNEL_SOURCES = {
     "k_assign": ("k_assign.cu", "km_ptx.cuh", "km_internal.h"),
-    "update": ("k_update.cu", "k_sort.cu", "km_rows.cuh", "km_internal.h"),
+    "update": ("k_update.cu", "k_sort.cu", "km_rows.cuh", "km_ptx.cuh", "km_internal.h"),
 }
 
 
