@@ -55,6 +55,14 @@
  *    form's tiling, so its last bits may differ between forms.
  *    KM_ASSIGN_TILE=pair,BN,XB,CS (read at every call) forces the whole
  *    assignment tiling; see km_plan_describe.
+ *  - Launch chaining: within one call, a kernel that directly follows another
+ *    of this library's kernels on the stream is launched with programmatic
+ *    stream serialization (it may become resident while its predecessor
+ *    drains and waits on the device, griddepcontrol.wait, before touching
+ *    shared data).  The first kernel of every call, and any kernel after a
+ *    memset, copy, event or plain launch, is stream-ordered as usual, so
+ *    calls compose with any other work on the stream.  Results do not depend
+ *    on it; KM_PDL=0 in the environment (read at every launch) turns it off.
  */
 #ifndef KM_H_
 #define KM_H_
