@@ -5,9 +5,11 @@
 //
 // A stable least-significant-digit radix sort of (key = cluster id, value =
 // point index), one or two passes of at most 12 bits.  Per pass:
-//   hist     block b counts the digits of its T keys -> blkhist[digit][b]
-//   colscan  one warp per digit: exclusive scan over blocks (digit-major
-//            order makes the concatenation the stable counting-sort offsets)
+//   hist     block b counts the digits of its T keys -> blkhist[b][digit]
+//            (on the first pass of a fit, the assignment kernel counts them)
+//   colscan  one lane per digit: exclusive scan over the blocks of each
+//            digit's counts, plus the digit totals (digit-major order of the
+//            runs makes the concatenation the stable counting-sort offsets)
 //   scatter  each block ranks its keys stably with per-warp counters
 //            (ballots group equal digits inside a warp step), scans the
 //            digit totals and its own digit counts, and writes every element
