@@ -52,7 +52,9 @@
  *    pairs on 256-point tiles (the default wherever the centroid tile is 128
  *    or 256 wide).  Both forms meet the same
  *    accuracy rules; the objective's float64 summation order follows the
- *    form's tiling, so its last bits may differ between forms.
+ *    form's tiling and the number of assignment CTAs the device holds at
+ *    once, so its last bits may differ between forms and between GPUs
+ *    (assignments and centroids do not).
  *    KM_ASSIGN_TILE=pair,BN,XB,CS (read at every call) forces the whole
  *    assignment tiling; see km_plan_describe.
  *  - Launch chaining: within one call, a kernel that directly follows another
