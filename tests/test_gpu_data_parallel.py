@@ -40,7 +40,11 @@ def _rank(rank, world, port, q):
         rows = slice(rank * N // world, (rank + 1) * N // world)
         r1 = km.fit_data_parallel(X[rows].contiguous(), C0, 1)
         r = km.fit_data_parallel(X[rows].contiguous(), C0, ITERS)
-        q.put((rank, r["C"].cpu(), r["counts"].cpu(), r["objective"].numpy(), r["idx"].cpu(), r1["C"].cpu()))
+        # numpy arrays travel by value (a torch CPU tensor would be shared by
+        # file descriptor, which the parent can only pick up while this
+        # process is still alive)
+        q.put((rank, r["C"].cpu().numpy(), r["counts"].cpu().numpy(), np.asarray(r["objective"]),
+               r["idx"].cpu().numpy(), r1["C"].cpu().numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -62,7 +66,7 @@ def test_two_ranks_match_the_single_device_fit():
         assert p.exitcode == 0
     (_, C_a, n_a, J_a, i_a, C1_a), (_, C_b, n_b, J_b, i_b, _) = out
     # every rank finalises the same sums: identical centroids, counts, objective
-    assert torch.equal(C_a, C_b) and torch.equal(n_a, n_b) and np.array_equal(J_a, J_b)
+    assert np.array_equal(C_a, C_b) and np.array_equal(n_a, n_b) and np.array_equal(J_a, J_b)
     assert int(n_a.sum()) == N
     X, C0 = _problem()
     # the whole point set's objective at t = 1 (same C0 everywhere) equals the oracle's
@@ -70,9 +74,9 @@ def test_two_ranks_match_the_single_device_fit():
     assert abs(J_a[0] - d1.sum()) <= JTOL * d1.sum()
     # after the last iteration: the centroids are the member means of the
     # assignment the ranks made (their rows concatenated)
-    idx = torch.cat([i_a, i_b]).numpy()
-    Cref, cref = oracle.update(X, idx, C_a)
-    assert np.array_equal(n_a.numpy(), cref)
+    idx = np.concatenate([i_a, i_b])
+    Cref, cref = oracle.update(X, idx, torch.from_numpy(C_a))
+    assert np.array_equal(n_a, cref)
     assert centroid_rel_err(C_a, Cref) <= CTOL["bf16"]
     # the single-device fit agrees: after one iteration (same assignments
     # from C0; float64 sums across ranks here, float32 segments there) the
