@@ -109,6 +109,14 @@ def test_plan_describes_the_chosen_tiling():
     assert km.plan(km.OP_FIT, 1, 1 << 22, 128, 16384, km.BF16)["sort_passes"] == 2
 
 
+@pytest.mark.parametrize("N,block", [(16384, 2048), (147 * 4096, 2048), (147 * 4096 + 1, 4096), (1 << 20, 4096),
+                                     (296 * 4096, 4096), (296 * 4096 + 1, 2048), (1 << 22, 2048)])
+def test_sort_block_fills_one_wave(N, block):
+    # 4096-key scatter blocks only when they fill the 148 SMs with one to two
+    # resident blocks each; 2048-key blocks (4 per SM) otherwise
+    assert km.plan(km.OP_FIT, 1, N, 128, 1024, km.BF16)["sort_block"] == block
+
+
 @pytest.mark.parametrize("tile,ok", [("0,256,2,2", True), ("1,128,3,3", True), ("1,64,2,2", False),
                                      ("0,256,8,4", False), ("0,256,9,2", False), ("junk", False)])
 def test_tiling_override_is_validated(monkeypatch, tile, ok):
