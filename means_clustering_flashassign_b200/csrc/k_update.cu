@@ -94,46 +94,6 @@ __device__ __forceinline__ void store_row(float* dst, int row_bytes, int lane, c
   }
 }
 
-__device__ __forceinline__ int find_cluster(const int32_t* start, int K, int64_t pos) {
-  int lo = 0, hi = K;  // start[lo] <= pos < start[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (start[mid] <= pos) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
-// One warp sums the runs of sorted positions [q0, q1).  Runs inside the range
-// are written with `final_store(k, acc)`; a run crossing the left edge goes to
-// slot 0, one crossing only the right edge to slot 1 (cluster ids in slot_k,
-// -1 when unused, vectors in slot_v[2][D]).
-template <int LPR, bool BF16, class FinalStore>
-__device__ __forceinline__ void warp_range_sums(const uint8_t* X, int row_bytes, int D, const int32_t* perm,
-                                                const int32_t* start, int K, int64_t q0, int64_t q1, int lane,
-                                                int* slot_k, float* slot_v, FinalStore final_store) {
-  if (lane == 0) { slot_k[0] = -1; slot_k[1] = -1; }
-  if (q0 >= q1) return;
-  int k = find_cluster(start, K, q0);
-  int64_t pos = q0;
-  while (pos < q1) {
-    while (start[k + 1] <= pos) ++k;
-    const int64_t s0 = start[k], s1 = start[k + 1];
-    const int64_t hi = s1 < q1 ? s1 : q1;
-    float acc[8];
-    seg_rows_sum<LPR, BF16>(X, row_bytes, perm, pos, hi, lane, acc);
-    const bool cl = s0 < q0, cr = s1 > q1;
-    if (!cl && !cr) {
-      final_store(k, acc);
-    } else {
-      const int slot = cl ? 0 : 1;
-      store_row<LPR, BF16>(slot_v + slot * D, row_bytes, lane, acc, 1.f);
-      if (lane == 0) slot_k[slot] = k;
-    }
-    pos = hi;
-    ++k;
-  }
-}
-
 // One warp sums the runs of sorted positions [q0, q1) using the sorted keys:
 // the cluster of every position is known, so run starts are found with a
 // warp ballot on key changes and the row ids / keys of the next batch are

@@ -28,12 +28,6 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 // One warp writes the assignment operand for centroid row k of an instance
 // from float values supplied by `get(j)` (j < D), and returns ||c||^2 of the
 // values the MMA uses (bf16-rounded in bf16 mode, the float32 values in f32
