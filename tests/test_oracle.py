@@ -164,6 +164,36 @@ def check_bf16_rounding():
     assert np.array_equal(oracle.round_bf16(a), want)
 
 
+def check_f32_rounding(seed=7):
+    """float32 round-to-nearest-even of doubles (the oracle's f32 mirror mode)
+    against numpy's float32 cast, bit for bit, and hand cases derived from the
+    format: 23 stored mantissa bits, subnormal spacing 2^-149, largest finite
+    value (2 - 2^-23) * 2^127."""
+    cases = {1 + 2**-24: 1.0,                      # halfway, ties to even (down)
+             1 + 3 * 2**-24: 1 + 2**-22,           # halfway, ties to even (up)
+             1 + 2**-24 + 2**-40: 1 + 2**-23,      # just above halfway
+             -(1 + 3 * 2**-24): -(1 + 2**-22),
+             2.0**-150: 0.0,                       # half the smallest subnormal
+             3 * 2.0**-150: 2.0**-148,             # subnormal halfway, to even
+             2.0**-149: 2.0**-149,
+             (2 - 2**-24) * 2.0**127: np.inf,      # halfway above the largest finite
+             (2 - 2**-24 - 2**-40) * 2.0**127: (2 - 2**-23) * 2.0**127,
+             0.1: 0.100000001490116119384765625, 0.0: 0.0}
+    for v, want in cases.items():
+        got = oracle.round_f32([v])[0]
+        assert got == want, (v, got, want)
+    rng = np.random.default_rng(seed)
+    a = np.concatenate([rng.normal(size=20000) * 10.0 ** rng.integers(-45, 39, 20000),
+                        rng.normal(size=2000),
+                        # exact float32 halfway points: a float32 value plus half its ulp
+                        (lambda f: f + np.spacing(f.astype(np.float32)).astype(np.float64) / 2)(
+                            rng.normal(size=2000).astype(np.float32).astype(np.float64))])
+    with np.errstate(over="ignore"):
+        want = a.astype(np.float32).astype(np.float64)
+    got = oracle.round_f32(a)
+    assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
+
+
 def check_argsort(seed=5):
     rng = np.random.default_rng(seed)
     for N, K in [(1000, 7), (4096, 256), (10, 40), (1, 1)]:
@@ -175,7 +205,7 @@ def check_argsort(seed=5):
 
 ALL_CHECKS = [check_golden_1d, check_golden_tie, check_assign_vs_cdist, check_bruteforce_integer,
               check_closed_forms, check_separated_mixture, check_invariants_and_sklearn,
-              check_bf16_rounding, check_argsort]
+              check_bf16_rounding, check_f32_rounding, check_argsort]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -207,6 +237,11 @@ MUTATIONS = {
     "second_best_not_updated": ("      } else if (d < second) {\n        second = d;", "      } else if (d < second) {\n        second = best;"),
     "transposed_centroid_index": ("sqdist(x, C + (int64_t)k * D, D)", "sqdist(x, C + (int64_t)k, D)"),
     "bf16_ties_away": ("(frac == 0.5 && fmod(r, 2.0) != 0.0)", "(frac == 0.5)"),
+    "f32_truncates": ("for (int64_t i = 0; i < n; ++i) out[i] = (double)(float)in[i];",
+                      "for (int64_t i = 0; i < n; ++i) { float f = (float)in[i]; "
+                      "if (fabs((double)f) > fabs(in[i])) f = nextafterf(f, 0.0f); out[i] = (double)f; }"),
+    "f32_not_rounded": ("for (int64_t i = 0; i < n; ++i) out[i] = (double)(float)in[i];",
+                        "for (int64_t i = 0; i < n; ++i) out[i] = in[i];"),
     "argsort_unstable": ("for (int64_t i = 0; i < N; ++i) perm[cursor[idx[i]]++] = (int32_t)i;",
                          "for (int64_t i = N - 1; i >= 0; --i) perm[cursor[idx[i]]++] = (int32_t)i;"),
     "objective_after_update": ("    J[t] = kmo_objective(d1, N);\n    kmo_update(X, idx, N, D, K, C, counts);",
