@@ -57,6 +57,16 @@
  *    (assignments and centroids do not).
  *    KM_ASSIGN_TILE=pair,BN,XB,CS (read at every call) forces the whole
  *    assignment tiling; see km_plan_describe.
+ *  - Fault injection (testing the error paths; nothing is done to the GPU):
+ *    KM_FAULT=<point>[:<n>] in the environment, read at the entry of every
+ *    call, makes the n-th occurrence (default 1) of that point inside the
+ *    call fail before it is issued: "alloc" (creating the copy stream or an
+ *    event of km_fit_host, or an event of km_fit_profile / km_fit_timed),
+ *    "h2d" (a host-to-device chunk copy of km_fit_host) or "launch" (a
+ *    kernel launch).  The call returns KM_ERR_INJECTED after the clean-up a
+ *    real failure of that step gets: work already enqueued completes, the
+ *    call's own streams and events are released (km_fit_host synchronises
+ *    first), and the context stays usable.
  *  - Launch chaining: within one call, a kernel that directly follows another
  *    of this library's kernels on the stream is launched with programmatic
  *    stream serialization (it may become resident while its predecessor
@@ -84,7 +94,8 @@ typedef enum km_status {
   KM_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve (shape, device) */
   KM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
   KM_ERR_WORKSPACE = 4,   /* workspace null or smaller than km_workspace_size() */
-  KM_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out */
+  KM_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait ran out */
+  KM_ERR_INJECTED = 6     /* a failure made on purpose by KM_FAULT (testing only) */
 } km_status;
 
 typedef enum km_dtype { KM_F32 = 0, KM_BF16 = 1 } km_dtype;
@@ -260,9 +271,13 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
  *     KM_ERR_UNSUPPORTED before anything is launched (bf16 with D=128 and
  *     K=1024 fits up to about 500 thousand points per call).
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
- *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress, with the device current) and caches it;
- *     make that first call before any stream capture.
+ *   - Every call made outside stream capture looks up the array's device
+ *     address on the current device (cudaGetSymbolAddress, with that device
+ *     current), so a device reset or a re-created context is followed.  A
+ *     call made while its stream is capturing uses the address cached by the
+ *     last uncaptured call on that device: make the first call on a device
+ *     before any stream capture (a captured call with no cached address is
+ *     refused with KM_ERR_UNSUPPORTED).
  *   - All calls on one device share the array and it keeps the last call's
  *     contents; each call clears what must start at zero.  Calls that may
  *     overlap on the GPU (different streams, other threads) race on it: order
@@ -283,11 +298,15 @@ int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_n
 
 /*
  * Data-parallel building blocks (a point set sharded by rows over several
- * devices or processes, §2 Methodology's Lloyd iteration with one exchange):
+ * devices or processes; the Lloyd iteration of Flash-KMeans §2 Methodology
+ * with one exchange per iteration):
  *   km_update_accumulate: the Sort-Inverse Update of this shard (argsort,
  *     segmented sums, ordered combine) added into float64 sums [K][D] and
- *     int64 counts [K] (zeroed first if zero_first); deterministic.  One
- *     instance; workspace as km_update (op KM_OP_UPDATE, B = 1).
+ *     float64 counts [K] (both zeroed first if zero_first); deterministic.
+ *     Counts are float64 so that sums, counts and the objective can sit in
+ *     one float64 buffer and be added across ranks by one all-reduce; they
+ *     are exact integers below 2^53.  One instance; workspace as km_update
+ *     (op KM_OP_UPDATE, B = 1).
  *   km_finalize_sums: C = sums / counts where counts > 0, else C is kept
  *     (C in/out float [K][D]); C_lp [K][D] (dtype; may be NULL) receives the
  *     copy the next km_assign takes (bf16 round-to-nearest-even, or float);
@@ -296,8 +315,8 @@ int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_n
  * all-reduce); every rank then finalises the same sums to the same C.
  */
 int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, double* sums,
-                         int64_t* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream);
-int km_finalize_sums(const double* sums, const int64_t* counts, int K, int D, int dtype, float* C, void* C_lp,
+                         double* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream);
+int km_finalize_sums(const double* sums, const double* counts, int K, int D, int dtype, float* C, void* C_lp,
                      int32_t* counts_out, void* stream);
 
 /*

@@ -187,6 +187,7 @@ int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int d
   if (!h) return KM_ERR_UNSUPPORTED;
   float* cn = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   float* S = cn + ((K + 63) / 64) * 64;
+  if (fault_hit(kFaultLaunch)) return KM_ERR_CUDA;
   count_launch();
   k_ab_cnorm<<<(K * 32 + 255) / 256, 256, 0, s>>>(C, K, D, dtype, cn);
   if (cudaGetLastError() != cudaSuccess) return KM_ERR_CUDA;
@@ -209,6 +210,7 @@ int ablation_assign(const void* X, const void* C, int64_t N, int D, int K, int d
                          &beta, S, CUDA_R_32F, K, kCublasCompute32F, kCublasGemmDefault);
     }
     if (st != 0) return KM_ERR_CUDA;
+    if (fault_hit(kFaultLaunch)) return KM_ERR_CUDA;
     count_launch();
     const int64_t threads = nr * 32;
     k_ab_argmin<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(X, S, cn, nr, r0, D, K, dtype, idx,
@@ -225,6 +227,7 @@ int ablation_update(const void* X, const int32_t* idx, int64_t N, int D, int K, 
   if (cudaMemsetAsync(sums, 0, static_cast<size_t>(K) * D * 4, s) != cudaSuccess) return KM_ERR_CUDA;
   if (cudaMemsetAsync(counts, 0, static_cast<size_t>(K) * 4, s) != cudaSuccess) return KM_ERR_CUDA;
   const int64_t threads = N * (D / 4);
+  if (fault_hit(kFaultLaunch)) return KM_ERR_CUDA;
   count_launch(2);
   k_ab_scatter<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(X, idx, N, D, K, dtype, sums, counts);
   const int64_t e = static_cast<int64_t>(K) * D;

@@ -15,11 +15,14 @@
 //     ||x||^2 + ||c||^2 - 2 x.c        (centroid operand holds -2c)
 // and the epilogue is a pure argmin.  Per score it forms a key -- the float
 // bits with the 5 low mantissa bits replaced by the column inside its
-// 32-column chunk -- and reduces keys with 3-input float minimum; equal
-// distances therefore resolve to the lowest column, and a chunk's winner is
-// merged into the running best only on a strictly smaller distance, so the
-// lowest index wins exact ties.  (Distances closer than 2^-18 relative also
-// compare equal; that is far inside the parity rule's near-tie band.)
+// 32-column chunk -- and reduces keys with 3-input float minimum.  A score
+// below zero (a point on a centroid, where the expanded form rounds to a few
+// ulps either side of 0) is clamped to +0 first: among negative floats a
+// larger column would make a more negative key and win the tie.  So equal
+// distances resolve to the lowest column, and a chunk's winner is merged
+// into the running best only on a strictly smaller distance: the lowest
+// index wins exact ties.  (Distances closer than 2^-18 relative also compare
+// equal; that is far inside the parity rule's near-tie band.)
 //
 // Structure: persistent CTAs (one per SM), warp-specialised:
 //   warp 0       TMA producer: point tile + its augmentation (resident for the
@@ -54,8 +57,7 @@ struct AssignK {
   int64_t tiles128_per_inst;       // 128-point tiles per instance (per-tile objective layout)
   int32_t* idx;
   float* mindist;
-  double* tobj;
-  int obj_per_cta;  // 1: tobj[cta][4] sums over the CTA's tiles in order; 0: tobj[tile][4]
+  double* tobj;     // [B * tiles128_per_inst][4]: per 128-point tile, one sum per 32-row quarter
   uint32_t zero;    // always 0; keeps the epilogue's column constants in registers
   int32_t* hist0;   // may be null: sort pass-0 block digit counts, [row / hist_T][digit]
   int hist_T, hist_R;
@@ -158,15 +160,20 @@ __device__ __forceinline__ void tmem_ld_wait<16>(uint32_t (&r)[16]) {
                : "memory");
 }
 
-// Minimum key of CW scores: key = score bits with the low 5 bits replaced by
-// the column index i in [0, CW) (mask == ~31 in a register, i an immediate),
-// so each key is one three-input bitwise operation.  Reduced with 3-input
-// minima.
+// Minimum key of CW scores: key = max(score, +0) bits with the low 5 bits
+// replaced by the column index i in [0, CW) (mask == ~31 in a register, i an
+// immediate): an integer maximum with 0 (a negative float is a negative
+// signed integer) and one three-input bitwise operation.  Clamping keeps the
+// key order of exact ties: for +0 and positive scores a lower column gives a
+// smaller key.  Reduced with 3-input minima.
 template <int CW>
 __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint32_t mask) {
   float k[CW];
 #pragma unroll
-  for (int i = 0; i < CW; ++i) k[i] = __uint_as_float((v[i] & mask) | static_cast<uint32_t>(i));
+  for (int i = 0; i < CW; ++i) {
+    const uint32_t nonneg = static_cast<uint32_t>(max(static_cast<int32_t>(v[i]), 0));
+    k[i] = __uint_as_float((nonneg & mask) | static_cast<uint32_t>(i));
+  }
   constexpr int L1 = CW / 3 + (CW % 3);  // CW=32: 10 triples + 2 singles; CW=16: 5 triples + 1 single
   float a[L1];
 #pragma unroll
@@ -437,7 +444,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     uint32_t aph = 0, mph = 0, gph = 0;
     bool ok = true;
-    double cta_obj = 0.0;
     const uint32_t kmask = ~31u + p.zero;
     const uint32_t a_empty_lead = PAIR ? mapa_shared(smem_addr(&a_empty[grp]), 0) : 0u;
     int64_t ct0 = 0;  // centroid tiles this CTA processed before the current point tile
@@ -484,15 +490,24 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           md = fmaxf(0.f, best);
           p.idx[o] = bk;
           if (p.mindist) p.mindist[o] = md;
-          if (p.hist0) atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + (bk & (p.hist_R - 1)), 1);
+        }
+        if (p.hist0) {
+          // sort pass-0 digit counts: the warp's 32 rows share one sort block
+          // (hist_T is a multiple of 32), so equal digits are added once per
+          // warp, by their lowest lane (a hot cluster costs one atomic per
+          // warp, not one per point)
+          const int dig = valid ? (bk & (p.hist_R - 1)) : -1;
+          const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+          if (valid && lane == __ffs(peers) - 1)
+            atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + dig, __popc(peers));
         }
         double ds = static_cast<double>(md);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-        if (p.obj_per_cta) {
-          cta_obj += ds;
-        } else if (lane == 0 && p.tobj) {
-          // per 128-point tile of the instance
+        // objective partial of this 32-row quarter of the 128-point tile: the
+        // slot depends on the tile index only, so the later fixed-order
+        // reduction does not depend on how tiles were dealt to CTAs
+        if (lane == 0 && p.tobj) {
           const int64_t tile128 = rt * (TM / kTileM) + rank;
           if (tile128 * kTileM < p.rows) p.tobj[(static_cast<int64_t>(b) * p.tiles128_per_inst + tile128) * 4 + q] = ds;
         }
@@ -537,15 +552,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       }
       mph ^= 1u;
     }
-    if constexpr (ONE_CT) {
-      // both groups' column-half-0 warps hold objective sums: group 1 hands
-      // its sums to group 0 (fixed order), over the epilogue warps only
-      double* objx = reinterpret_cast<double*>(mval + 2 * kTileM);  // [4], the unused third merge slot
-      if (p.obj_per_cta && h == 2 && lane == 0) objx[q] = cta_obj;
-      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-      if (p.obj_per_cta && h == 0 && lane == 0) cta_obj += objx[q];
-    }
-    if (h == 0 && p.obj_per_cta && lane == 0 && p.tobj) p.tobj[static_cast<int64_t>(blockIdx.x) * 4 + q] = cta_obj;
   }
 
   __syncthreads();
@@ -575,7 +581,6 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.idx = a.idx;
   k.mindist = a.mindist;
   k.tobj = a.tobj;
-  k.obj_per_cta = a.B == 1 ? 1 : 0;
   k.zero = 0;
   k.hist0 = a.B == 1 ? a.hist0 : nullptr;
   k.hist_T = a.hist_T;
@@ -613,8 +618,12 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   }
   const int64_t active = k.ntiles < units ? k.ntiles : units;
   const int64_t grid = PAIR ? 2 * active : active;
-  if (a.obj_groups) *a.obj_groups = k.obj_per_cta ? grid : k.tiles128_per_inst;
+  if (a.obj_groups) *a.obj_groups = k.tiles128_per_inst;
   if (grid <= 0) return cudaSuccess;
+  if (fault_hit(kFaultLaunch)) {
+    chain_break();
+    return cudaErrorLaunchFailure;
+  }
   count_launch();
   cudaLaunchConfig_t lc{};
   lc.gridDim = dim3(static_cast<unsigned>(grid));
@@ -692,6 +701,7 @@ __global__ void k_timeout_probe(unsigned int* status, uint64_t limit_ns) {
 
 cudaError_t launch_timeout_probe(unsigned int* status, uint64_t limit_ns, cudaStream_t s) {
   chain_break();  // plain launch: the next kernel must not chain to it
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_timeout_probe<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();

@@ -87,6 +87,7 @@ cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, 
     const int64_t need = (rows * lpr + 255) / 256;
     const unsigned grid = static_cast<unsigned>(need < int64_t(nsm) * 8 ? need : int64_t(nsm) * 8);
     const uint8_t* Xb = static_cast<const uint8_t*>(X);
+    if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
     count_launch();
     switch (lpr) {
       case 1: k_xnorm_bf16<1><<<grid, 256, 0, s>>>(Xb, rows, row_bytes, xaug); break;
@@ -100,6 +101,7 @@ cudaError_t launch_xprep(const void* X, int dtype, int64_t rows, int D, int Dp, 
   }
   const int threads = 256;
   const int64_t blocks = (rows * 32 + threads - 1) / threads;
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_xprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(X, dtype, rows, D, Dp, xaug, x3);
   return cudaGetLastError();
@@ -138,6 +140,7 @@ cudaError_t launch_cprep(const void* src, int src_dtype, int B, int K, int Kp, i
   const int threads = 256;
   const int64_t warps = static_cast<int64_t>(B) * Kp;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_cprep<<<static_cast<unsigned>(blocks), threads, 0, s>>>(src, src_dtype, B, K, Kp, D, Dp, dtype, master, c_op,
                                                            static_cast<uint8_t*>(caug));
@@ -165,6 +168,7 @@ __global__ void k_objective(const double* __restrict__ tobj, int64_t per_inst, d
 cudaError_t launch_objective(const double* tobj, int B, int64_t groups_per_inst, double* out, int out_stride,
                              cudaStream_t s) {
   chain_break();  // plain launch: the next kernel must not chain to it
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_objective<<<B, 256, 0, s>>>(tobj, groups_per_inst * 4, out, out_stride);
   return cudaGetLastError();

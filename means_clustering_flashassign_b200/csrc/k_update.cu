@@ -301,10 +301,61 @@ struct FinK {
   int32_t* counts;
   double* acc64;
   long long* cnt64;
+  double* cntf;  // mode 1: float64 counts instead of cnt64 (data-parallel sums), or null
   const double* tobj;
   int64_t ntiles;
   double* obj;
+  int nobj;                // objective blocks (the grid's last nobj blocks; 0: no objective)
+  double* objpart;         // [nobj] block sums
+  unsigned int* objcnt;    // blocks done (zero at entry; the last block resets it)
 };
+
+// Objective partials per block of the finalise kernel: each block sums a
+// fixed range of this many assignment partials.
+constexpr int kObjPerBlock = 4096;
+
+// Block j of nobj: the objective of this pass from the assignment's
+// per-tile partials in a fixed order -- block j sums partials
+// [j*kObjPerBlock, (j+1)*kObjPerBlock) (thread-strided, then a fixed tree),
+// and the last block to finish sums the nobj block sums the same way.  The
+// order depends only on the number of partials, never on which CTA computed
+// which tile, so the objective is bitwise reproducible across grids.
+__device__ void objective_block(const FinK& f, int j, double* red) {
+  const int tid = threadIdx.x;
+  const int64_t total = f.ntiles * 4;
+  const int64_t lo = static_cast<int64_t>(j) * kObjPerBlock;
+  const int64_t hi = lo + kObjPerBlock < total ? lo + kObjPerBlock : total;
+  __shared__ int is_last;
+  auto block_sum = [&](double v) {
+    red[tid] = v;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (tid < w) red[tid] += red[tid + w];
+      __syncthreads();
+    }
+    return red[0];
+  };
+  double s = 0.0;
+  for (int64_t i = lo + tid; i < hi; i += blockDim.x) s += f.tobj[i];
+  const double bs = block_sum(s);
+  if (tid == 0) {
+    f.objpart[j] = bs;
+    __threadfence();
+    is_last = atomicAdd(f.objcnt, 1u) == static_cast<unsigned>(f.nobj - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  s = 0.0;
+  for (int i = tid; i < f.nobj; i += blockDim.x) s += __ldcg(f.objpart + i);
+  __syncthreads();  // red is reused
+  const double tot = block_sum(s);
+  if (tid == 0) {
+    if (f.mode == 0) *f.obj = tot;
+    else *f.obj += tot;
+    *f.objcnt = 0u;
+  }
+}
 
 __device__ __forceinline__ void* op_row(const FinK& f, int k) {
   if (!f.c_op) return nullptr;
@@ -385,7 +436,10 @@ __device__ void finish_cluster(const FinK& f, int k, int64_t cnt, float (&sum)[8
       const int j = lane + 32 * i;
       if (j < f.D) arow[j] += static_cast<double>(sum[i]);
     }
-    if (lane == 0) f.cnt64[k] += cnt;
+    if (lane == 0) {
+      if (f.cntf) f.cntf[k] += static_cast<double>(cnt);
+      else f.cnt64[k] += cnt;
+    }
   }
 }
 
@@ -394,22 +448,10 @@ __global__ void __launch_bounds__(512) k_finalize(const FinK f) {
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (blockIdx.x == gridDim.x - 1 && f.ntiles > 0) {
-    // the last block: objective of this pass, a fixed-order reduction of the
-    // assign partials
-    double* red = reinterpret_cast<double*>(fsm);
-    double s = 0.0;
-    for (int64_t i = threadIdx.x; i < f.ntiles * 4; i += blockDim.x) s += f.tobj[i];
-    red[threadIdx.x] = s;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-      if (f.mode == 0) *f.obj = red[0];
-      else *f.obj += red[0];
-    }
+  if (static_cast<int>(blockIdx.x) >= static_cast<int>(gridDim.x) - f.nobj) {
+    // the last nobj blocks: objective of this pass (fixed-order reduction)
+    objective_block(f, static_cast<int>(blockIdx.x) - (static_cast<int>(gridDim.x) - f.nobj),
+                    reinterpret_cast<double*>(fsm));
     return;
   }
   if (blockIdx.x < f.nwarp_blocks) {
@@ -525,14 +567,18 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
   f.counts = a.counts;
   f.acc64 = a.acc64;
   f.cnt64 = a.cnt64;
+  f.cntf = a.cntf;
   f.tobj = a.tobj;
   f.ntiles = a.ntiles;
   f.obj = a.obj;
+  f.nobj = a.ntiles > 0 ? static_cast<int>((a.ntiles * 4 + kObjPerBlock - 1) / kObjPerBlock) : 0;
+  f.objpart = a.objpart;
+  f.objcnt = a.objcnt;
   const int threads = 512;
   f.nwarp_blocks = (p.K + 15) / 16;
   const int64_t G = static_cast<int64_t>(p.gc.big_span) * f.BNS;
   const int64_t nbig = (p.rows + G - 1) / G;
-  // objective block: 512 doubles (1024 floats); warp blocks: 16 warp rows;
+  // objective blocks: 512 doubles (1024 floats); warp blocks: 16 warp rows;
   // big-cluster blocks: slices x D partial rows + one summed row.
   const size_t fl_warp = 1024 + 16 * static_cast<size_t>(p.D);
   const size_t fl_big = 2048 + 2 * static_cast<size_t>(p.D);
@@ -541,8 +587,7 @@ cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s
                                        static_cast<int>(sm));
   if (e != cudaSuccess) return e;
   count_launch();
-  const int64_t nobj = f.ntiles > 0 ? 1 : 0;
-  return launch_chained(k_finalize, dim3(static_cast<unsigned>(f.nwarp_blocks + nbig + nobj)), dim3(threads), sm, s,
+  return launch_chained(k_finalize, dim3(static_cast<unsigned>(f.nwarp_blocks + nbig + f.nobj)), dim3(threads), sm, s,
                         f);
 }
 
@@ -576,18 +621,19 @@ __global__ void k_finalize_acc(int K, int D, int Dp, int dtype, double* acc64, l
 }
 
 // Centroids from float64 sums and counts accumulated elsewhere (e.g. added
-// up across the ranks of a data-parallel fit): C = sum / count where count >
-// 0, else C is kept; C_lp is the dtype copy the next assignment takes (bf16
+// up across the ranks of a data-parallel fit; counts are float64, exact
+// integers below 2^53): C = sum / count where count > 0, else C is kept;
+// C_lp is the dtype copy the next assignment takes (bf16
 // round-to-nearest-even or the float values); counts as int32.
-__global__ void k_finalize_sums(const double* __restrict__ sums, const long long* __restrict__ cnt, int K, int D,
+__global__ void k_finalize_sums(const double* __restrict__ sums, const double* __restrict__ cnt, int K, int D,
                                 int dtype, float* C, void* C_lp, int32_t* counts) {
   const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= static_cast<int64_t>(K) * D) return;
   const int k = static_cast<int>(e / D);
-  const long long n = cnt[k];
+  const double n = cnt[k];
   float c = C[e];
-  if (n > 0) {
-    c = static_cast<float>(sums[e] / static_cast<double>(n));
+  if (n > 0.0) {
+    c = static_cast<float>(sums[e] / n);
     C[e] = c;
   }
   if (C_lp) {
@@ -597,10 +643,11 @@ __global__ void k_finalize_sums(const double* __restrict__ sums, const long long
   if (counts && e - static_cast<int64_t>(k) * D == 0) counts[k] = static_cast<int32_t>(n);
 }
 
-cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const long long* cnt, float* C,
+cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const double* cnt, float* C,
                                  void* C_lp, int32_t* counts, cudaStream_t s) {
   chain_break();  // plain launch: the next kernel must not chain to it
   const int64_t e = static_cast<int64_t>(K) * D;
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_finalize_sums<<<static_cast<unsigned>((e + 255) / 256), 256, 0, s>>>(sums, cnt, K, D, dtype, C, C_lp, counts);
   return cudaGetLastError();
@@ -611,6 +658,7 @@ cudaError_t launch_finalize_acc(const Plan& p, double* acc64, long long* cnt64, 
   chain_break();  // plain launch: the next kernel must not chain to it
   const int threads = 256;
   const int blocks = (p.K + 7) / 8;
+  if (fault_hit(kFaultLaunch)) return cudaErrorLaunchFailure;
   count_launch();
   k_finalize_acc<<<blocks, threads, 0, s>>>(p.K, p.D, p.Dp, p.dtype, acc64, cnt64, C, c_op, static_cast<uint8_t*>(caug), counts, objacc,
                                             obj_out);

@@ -37,6 +37,39 @@ static thread_local bool t_chain = false;
 void chain_break() { t_chain = false; }
 bool chain_armed() { return t_chain; }
 void chain_arm() { t_chain = true; }
+
+// Fault injection state of the calling thread (one call at a time).
+struct FaultState {
+  int point = -1;      // FaultPoint to fail, -1 = none
+  int64_t at = 0;      // 1-based occurrence that fails
+  int64_t seen[3] = {0, 0, 0};
+  bool fired = false;
+};
+static thread_local FaultState t_fault;
+
+void fault_arm_from_env() {
+  t_fault = FaultState{};
+  const char* e = getenv("KM_FAULT");
+  if (!e || !*e) return;
+  static const char* names[3] = {"alloc", "h2d", "launch"};
+  for (int i = 0; i < 3; ++i) {
+    const size_t n = strlen(names[i]);
+    if (strncmp(e, names[i], n) == 0 && (e[n] == 0 || e[n] == ':')) {
+      t_fault.point = i;
+      t_fault.at = e[n] == ':' ? strtoll(e + n + 1, nullptr, 10) : 1;
+      if (t_fault.at < 1) t_fault.point = -1;
+    }
+  }
+}
+
+bool fault_hit(int point) {
+  if (t_fault.point != point) return false;
+  if (++t_fault.seen[point] != t_fault.at) return false;
+  t_fault.fired = true;
+  return true;
+}
+
+bool fault_fired() { return t_fault.fired; }
 }  // namespace km
 
 using namespace km;
@@ -52,6 +85,11 @@ int fail(int code, const char* fmt, ...) {
   vsnprintf(buf, sizeof(buf), fmt, ap);
   va_end(ap);
   g_err = buf;
+  // a failure that the host-side injector caused (KM_FAULT) reports as such
+  if (code == KM_ERR_CUDA && fault_fired()) {
+    code = KM_ERR_INJECTED;
+    g_err = std::string("injected fault (KM_FAULT): ") + buf;
+  }
   return code;
 }
 
@@ -316,6 +354,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   p.off_tobj = take(sizeof(double) * 4 * static_cast<size_t>(p.ntiles > 256 ? p.ntiles : 256));
   if (op == KM_OP_FIT || op == KM_OP_FIT_HOST) p.off_idx = take(sizeof(int32_t) * BR);
   p.off_obj = take(sizeof(double) * (op == KM_OP_FIT_HOST ? kMaxHostIters : B));
+  p.off_objpart = take(sizeof(double) * static_cast<size_t>(objective_blocks(p.tiles_per_inst) + 1));
   if (op != KM_OP_ASSIGN && !p.small_update) {
     p.off_blkhist = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[0]) * sc.nblk);
     if (sc.passes > 1) p.off_blkhist1 = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[1]) * sc.nblk);
@@ -342,16 +381,23 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
 
 namespace {
 
+// Set while an entry point that already armed the injector (and may have
+// counted occurrences, e.g. its event creation) calls a shared helper.
+thread_local bool t_fault_keep = false;
+
 struct Ctx {
   Plan p;
   void* ws;
   cudaStream_t s;
   unsigned int* status() const { return at<unsigned int>(ws, p.off_hdr); }
+  // header word 1: blocks done of the finalise kernel's objective reduction
+  unsigned int* objcnt() const { return at<unsigned int>(ws, p.off_hdr) + 1; }
 };
 
 int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t chunk_rows, void* ws,
             size_t ws_bytes, void* stream) {
   const char* why = "";
+  if (!t_fault_keep) fault_arm_from_env();
   int r = make_plan(c.p, op, B, N, D, K, dtype, chunk_rows, &why);
   if (r != KM_OK) return fail(r, "%s", why);
   if (!ws) return fail(KM_ERR_WORKSPACE, "workspace is NULL");
@@ -369,7 +415,7 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
-                    bool hist0_ready = false, double* acc_ext = nullptr, long long* cnt_ext = nullptr) {
+                    bool hist0_ready = false, double* acc_ext = nullptr, double* cnt_ext = nullptr) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
@@ -398,10 +444,13 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
   fa.caug = caugb;
   fa.counts = countsb;
   fa.acc64 = mode == 1 ? (acc_ext ? acc_ext : at<double>(c.ws, p.off_acc64)) : nullptr;
-  fa.cnt64 = mode == 1 ? (cnt_ext ? cnt_ext : at<long long>(c.ws, p.off_cnt64)) : nullptr;
+  fa.cnt64 = mode == 1 && !cnt_ext ? at<long long>(c.ws, p.off_cnt64) : nullptr;
+  fa.cntf = mode == 1 ? cnt_ext : nullptr;
   fa.tobj = tobjb;
   fa.ntiles = obj ? ntiles : 0;
   fa.obj = obj;
+  fa.objpart = at<double>(c.ws, p.off_objpart);
+  fa.objcnt = c.objcnt();
   Plan pp = p;
   pp.rows = n;
   KM_CUDA(launch_finalize(pp, fa, c.s));
@@ -429,6 +478,7 @@ const char* km_status_string(int status) {
     case KM_ERR_CUDA: return "cuda error";
     case KM_ERR_WORKSPACE: return "workspace too small or misaligned";
     case KM_ERR_TIMEOUT: return "bounded in-kernel wait ran out";
+    case KM_ERR_INJECTED: return "injected fault";
     default: return "unknown status";
   }
 }
@@ -533,7 +583,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   int32_t* idx = idx_out ? idx_out : at<int32_t>(c.ws, p.off_idx);
   double* objs = at<double>(c.ws, p.off_obj);
   const bool f32 = dtype == KM_F32;
-  KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+  KM_CUDA(cudaMemsetAsync(c.status(), 0, 2 * sizeof(unsigned int), c.s));  // status, objective counter
   chain_break();
   float* x3 = f32 ? at<float>(c.ws, p.off_x3) : nullptr;
   KM_CUDA(launch_xprep(X, dtype, static_cast<int64_t>(B) * N, D, p.Dp, xaug, x3, c.s));
@@ -602,19 +652,22 @@ int km_fit_profile(const void* X, const void* C0, int B, int64_t N, int D, int K
   g_err.clear();
   if (!phase_ms) return fail(KM_ERR_INVALID_ARG, "phase_ms is required");
   if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  fault_arm_from_env();
   std::vector<cudaEvent_t> ev(3 * static_cast<size_t>(iters), nullptr);
   auto destroy = [&]() {
     for (auto e : ev)
       if (e) cudaEventDestroy(e);
   };
   for (auto& e : ev) {
-    if (cudaEventCreate(&e) != cudaSuccess) {
+    if (fault_hit(kFaultAlloc) || cudaEventCreate(&e) != cudaSuccess) {
       destroy();
       return fail(KM_ERR_CUDA, "cudaEventCreate failed");
     }
   }
+  t_fault_keep = true;
   int r = fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
                    workspace_bytes, stream, iters > 0 ? ev.data() : nullptr);
+  t_fault_keep = false;
   if (r == KM_OK && cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     r = fail(KM_ERR_CUDA, "stream synchronisation failed");
   for (int t = 0; r == KM_OK && t < iters; ++t) {
@@ -638,15 +691,18 @@ int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, 
   g_err.clear();
   if (!iters_ms) return fail(KM_ERR_INVALID_ARG, "iters_ms is required");
   if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  fault_arm_from_env();
   cudaEvent_t ev[2] = {nullptr, nullptr};
   for (auto& e : ev)
-    if (cudaEventCreate(&e) != cudaSuccess) {
+    if (fault_hit(kFaultAlloc) || cudaEventCreate(&e) != cudaSuccess) {
       for (auto x : ev)
         if (x) cudaEventDestroy(x);
       return fail(KM_ERR_CUDA, "cudaEventCreate failed");
     }
+  t_fault_keep = true;
   int r = fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
                    workspace_bytes, stream, iters > 0 ? ev : nullptr, false);
+  t_fault_keep = false;
   if (r == KM_OK && cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     r = fail(KM_ERR_CUDA, "stream synchronisation failed");
   *iters_ms = 0.f;
@@ -692,12 +748,15 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
     if (cs) cudaStreamDestroy(cs);
   };
   auto run = [&]() -> int {
+    if (fault_hit(kFaultAlloc)) return fail(KM_ERR_CUDA, "cudaStreamCreateWithFlags failed");
     KM_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
     for (int i = 0; i < 2; ++i) {
+      if (fault_hit(kFaultAlloc)) return fail(KM_ERR_CUDA, "cudaEventCreateWithFlags failed");
       KM_CUDA(cudaEventCreateWithFlags(&ev_copied[i], cudaEventDisableTiming));
+      if (fault_hit(kFaultAlloc)) return fail(KM_ERR_CUDA, "cudaEventCreateWithFlags failed");
       KM_CUDA(cudaEventCreateWithFlags(&ev_free[i], cudaEventDisableTiming));
     }
-    KM_CUDA(cudaMemsetAsync(c.status(), 0, sizeof(unsigned int), c.s));
+    KM_CUDA(cudaMemsetAsync(c.status(), 0, 2 * sizeof(unsigned int), c.s));  // status, objective counter
     chain_break();
     KM_CUDA(cudaMemsetAsync(acc64, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
     chain_break();
@@ -728,6 +787,7 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         const int64_t nr = N - r0 < p.chunk_rows ? N - r0 : p.chunk_rows;
         KM_CUDA(cudaStreamWaitEvent(cs, ev_free[bi], 0));
         chain_break();
+        if (fault_hit(kFaultH2D)) return fail(KM_ERR_CUDA, "cudaMemcpyAsync of chunk %lld failed", (long long)ch);
         KM_CUDA(cudaMemcpyAsync(dbuf[bi], static_cast<const uint8_t*>(X_host) + r0 * rowb, nr * rowb,
                                 cudaMemcpyHostToDevice, cs));
         chain_break();
@@ -795,7 +855,7 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
 }
 
 int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, int K, int dtype, double* sums,
-                         int64_t* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream) {
+                         double* counts, int zero_first, void* workspace, size_t workspace_bytes, void* stream) {
   g_err.clear();
   if (!X || !idx || !sums || !counts) return fail(KM_ERR_INVALID_ARG, "X, idx, sums and counts are required");
   if (!aligned16(X)) return fail(KM_ERR_INVALID_ARG, "X must be 16-byte aligned");
@@ -805,23 +865,24 @@ int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, in
   if (zero_first) {
     KM_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * static_cast<size_t>(K) * D, c.s));
     chain_break();
-    KM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int64_t) * K, c.s));
+    KM_CUDA(cudaMemsetAsync(counts, 0, sizeof(double) * K, c.s));
     chain_break();
   }
   return update_instance(c, X, idx, N, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 1, false, sums,
-                         reinterpret_cast<long long*>(counts));
+                         counts);
 }
 
-int km_finalize_sums(const double* sums, const int64_t* counts, int K, int D, int dtype, float* C, void* C_lp,
+int km_finalize_sums(const double* sums, const double* counts, int K, int D, int dtype, float* C, void* C_lp,
                      int32_t* counts_out, void* stream) {
   g_err.clear();
   if (!sums || !counts || !C) return fail(KM_ERR_INVALID_ARG, "sums, counts and C are required");
   if (K < 1 || D < 1) return fail(KM_ERR_INVALID_ARG, "need K >= 1 and D >= 1");
   if (dtype != KM_F32 && dtype != KM_BF16) return fail(KM_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  fault_arm_from_env();
   int r = check_device();
   if (r != KM_OK) return r;
-  KM_CUDA(km::launch_finalize_sums(K, D, dtype, sums, reinterpret_cast<const long long*>(counts), C, C_lp,
-                                   counts_out, static_cast<cudaStream_t>(stream)));
+  KM_CUDA(km::launch_finalize_sums(K, D, dtype, sums, counts, C, C_lp, counts_out,
+                                   static_cast<cudaStream_t>(stream)));
   return KM_OK;
 }
 
@@ -846,6 +907,7 @@ int km_plan_describe(int op, int B, int64_t N, int D, int K, int dtype, int64_t 
 // ------------------------------------------------------------- baselines
 namespace {
 int ablation_check(const void* X, int64_t N, int D, int K, int dtype) {
+  fault_arm_from_env();
   if (!X) return fail(KM_ERR_INVALID_ARG, "X is required");
   if (dtype != KM_F32 && dtype != KM_BF16) return fail(KM_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (N < 1 || K < 1 || K > N) return fail(KM_ERR_INVALID_ARG, "need 1 <= K <= N (N=%lld K=%d)", (long long)N, K);
@@ -903,6 +965,7 @@ int km_selftest_timeout(void* workspace, size_t workspace_bytes, int64_t limit_n
   g_err.clear();
   if (!workspace || workspace_bytes < kAlign) return fail(KM_ERR_WORKSPACE, "need at least 256 bytes of workspace");
   if (limit_ns < 1 || limit_ns > 1000000000) return fail(KM_ERR_INVALID_ARG, "limit_ns must be in [1, 1e9]");
+  fault_arm_from_env();
   int r = check_device();
   if (r != KM_OK) return r;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -29,6 +29,18 @@ inline std::atomic<uint64_t>& launch_counter() {
 }
 inline void count_launch(uint64_t n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
 
+// Host-side fault injection, for testing the error paths without faulting a
+// GPU.  KM_FAULT=<point>[:<n>] in the environment (read at the entry of every
+// call) makes the n-th occurrence (default 1) of that point inside the call
+// fail before it is issued: "alloc" (creating a library-owned stream or
+// event), "h2d" (a host-to-device chunk copy of the out-of-core fit) or
+// "launch" (a kernel launch).  The call then returns KM_ERR_INJECTED after
+// the same clean-up as for a real failure of that call.
+enum FaultPoint { kFaultAlloc = 0, kFaultH2D = 1, kFaultLaunch = 2 };
+void fault_arm_from_env();   // at call entry: parse KM_FAULT, reset the counters
+bool fault_hit(int point);   // count one occurrence; true if it must fail
+bool fault_fired();          // the current call failed by injection
+
 struct AssignCfg {
   bool pair = false;   // CTA pairs with cta_group::2 UMMAs (256-point tiles)
   int BN = 0;          // centroids per UMMA tile (N of the MMA), 64/128/256
@@ -87,6 +99,10 @@ inline cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block,
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = pdl_enabled() && chain_armed() ? 1 : 0;
+  if (fault_hit(kFaultLaunch)) {
+    chain_break();
+    return cudaErrorLaunchFailure;
+  }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   if (e == cudaSuccess) chain_arm();
   else chain_break();
@@ -119,7 +135,7 @@ struct Plan {
   // workspace offsets (bytes)
   size_t off_hdr = 0, off_xaug = 0, off_caug = 0, off_clp = 0, off_x3 = 0, off_tobj = 0, off_idx = 0;
   size_t off_blkhist = 0, off_blkhist1 = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
-  size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0;
+  size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0, off_objpart = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
   size_t total = 0;
 };
@@ -157,7 +173,7 @@ struct AssignArgs {
   int K, Kp;
   int32_t* idx;
   float* mindist;
-  double* tobj;  // B == 1: [assign CTAs][4]; else [B * tiles_per_inst][4]
+  double* tobj;  // [B * tiles_per_inst][4]: objective partials per 128-point tile and 32-row quarter
   unsigned int* status;
   uint64_t limit_ns;
   int64_t* obj_groups;  // host out (may be null): 4-double groups of partials per instance
@@ -213,13 +229,19 @@ struct FinalizeArgs {
   void* caug;        // [Kp] augmentation rows
   int32_t* counts;   // [K] or null
   double* acc64;     // [K][D] (mode 1)
-  long long* cnt64;  // [K] (mode 1)
+  long long* cnt64;  // [K] (mode 1, unless cntf)
+  double* cntf;      // [K] (mode 1): float64 counts instead of cnt64, or null
   const double* tobj;
   int64_t ntiles;    // tile partials to reduce into *obj (0: none)
   double* obj;       // objective output (mode 0) or accumulator (mode 1)
+  double* objpart;   // [objective_blocks(ntiles)] scratch of the reduction
+  unsigned int* objcnt;  // zero on entry; left zero
 };
+// Blocks of the finalise kernel's objective reduction for `ntiles` 128-point
+// tiles (4 partials each, 4096 partials per block).
+inline int64_t objective_blocks(int64_t ntiles) { return (ntiles * 4 + 4095) / 4096; }
 cudaError_t launch_finalize(const Plan& p, const FinalizeArgs& a, cudaStream_t s);
-cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const long long* cnt, float* C,
+cudaError_t launch_finalize_sums(int K, int D, int dtype, const double* sums, const double* cnt, float* C,
                                  void* C_lp, int32_t* counts, cudaStream_t s);
 
 // Final step of the out-of-core update: centroids from float64 accumulators.

@@ -38,14 +38,25 @@ int static_fail(int code, const char* msg) {
   return code;
 }
 
-// Device address of g_static_scratch on the current device, looked up once
-// per device (with that device current) and cached.
-int scratch_address(void** out, int* dev_out) {
+// Device address of g_static_scratch on the current device.  Outside stream
+// capture it is looked up again on every call (with that device current), so
+// a device reset or a re-created context, which reloads the module at a new
+// address, is followed.  During capture the address cached by the last
+// uncaptured call on the device is used (a lookup may not be legal while a
+// capture is open); with no such call the request is refused.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return static_fail(KM_ERR_CUDA, "cudaGetDevice failed");
   if (dev < 0 || dev >= kMaxDevices) return static_fail(KM_ERR_UNSUPPORTED, "device ordinal out of range");
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const cudaError_t ce = cudaStreamIsCapturing(stream, &cap);
+  if (ce != cudaSuccess) {
+    char buf[256];
+    snprintf(buf, sizeof(buf), "cudaStreamIsCapturing failed: %s", cudaGetErrorString(ce));
+    return static_fail(KM_ERR_CUDA, buf);
+  }
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || !p) {
@@ -54,9 +65,11 @@ int scratch_address(void** out, int* dev_out) {
       return static_fail(KM_ERR_CUDA, buf);
     }
     g_scratch_addr[dev] = p;
+  } else if (!g_scratch_addr[dev]) {
+    return static_fail(KM_ERR_UNSUPPORTED,
+                       "km_assign_static: the first call on a device must come before any stream capture");
   }
   *out = g_scratch_addr[dev];
-  *dev_out = dev;
   return KM_OK;
 }
 
@@ -80,8 +93,7 @@ int km_assign_static(const void* X, const void* C, int B, int64_t N, int D, int 
     return static_fail(KM_ERR_UNSUPPORTED, buf);
   }
   void* scratch = nullptr;
-  int dev = 0;
-  const int r = scratch_address(&scratch, &dev);
+  const int r = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (r != KM_OK) return r;
   // km_assign clears the status word at the start of the area and fully
   // writes every other scratch value before reading it.

@@ -37,9 +37,21 @@ def test_library_loads_and_exports_header_symbols():
 
 def test_status_strings():
     L = km.library()
-    for code in range(6):
-        assert L.km_status_string(code)
+    for code in range(7):
+        assert L.km_status_string(code) != b"unknown status"
+    assert L.km_status_string(6) == b"injected fault"
     assert L.km_status_string(99) == b"unknown status"
+    assert km.STATUS[6] == "KM_ERR_INJECTED"
+
+
+@pytest.mark.parametrize("spec", ["launch", "launch:3", "h2d:2", "alloc", "bogus", "launch:0", ""])
+def test_fault_spec_does_not_change_host_side_refusals(monkeypatch, spec):
+    """KM_FAULT only acts on device work: argument checks still come first,
+    so an invalid call is refused with its own code whatever the spec."""
+    monkeypatch.setenv("KM_FAULT", spec)
+    L = km.library()
+    assert L.km_fit(None, None, 1, 100, 64, 10, 1, 3, None, None, None, None, None, 0, None) == 1
+    assert L.km_workspace_size(km.OP_FIT, 1, 100, 12, 10, km.BF16, 0) == 0
 
 
 @pytest.mark.parametrize("op", [km.OP_ASSIGN, km.OP_UPDATE, km.OP_FIT])
