@@ -10,7 +10,8 @@ Every function follows "Flash-KMeans: Fast and Memory-Efficient Exact K-Means",
   assign   -- argmin of squared Euclidean distance, lowest index on ties;
   update   -- per-cluster mean, empty clusters keep their centroid;
   argsort  -- stable ordering of point indices by cluster id (§2.2's inverse map);
-  fit      -- T assign/update rounds, objective recorded under the centroids used.
+  fit      -- T assign/update rounds, objective recorded under the centroids used;
+  objective_assigned_bf16 -- the objective of a given assignment of bfloat16 points.
 """
 
 from __future__ import annotations
@@ -63,6 +64,8 @@ def _configure(L):
     L.kmo_update.argtypes = [P, P, i64, i32, i32, P, P]
     L.kmo_objective.argtypes = [P, i64]
     L.kmo_objective.restype = ctypes.c_double
+    L.kmo_objective_assigned_bf16.argtypes = [P, P, P, i64, i32]
+    L.kmo_objective_assigned_bf16.restype = ctypes.c_double
     L.kmo_round_bf16.argtypes = [P, P, i64]
     L.kmo_round_f32.argtypes = [P, P, i64]
     L.kmo_round_bf16_one.argtypes = [ctypes.c_double]
@@ -148,6 +151,20 @@ def update(X, idx, C_prev):
 def objective(d1) -> float:
     d1 = _f64(d1)
     return float(lib().kmo_objective(_p(d1), d1.shape[0]))
+
+
+def objective_assigned_bf16(X, C, idx) -> float:
+    """sum_i ||x_i - c_{idx[i]}||^2 in float64 (direct form) for bfloat16
+    points X (a torch bfloat16 tensor on the CPU, or its raw uint16 bits as a
+    numpy array), float64-widened centroids C and an assignment idx."""
+    if hasattr(X, "detach"):
+        import torch
+        X = X.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+    Xb = np.ascontiguousarray(X, dtype=np.uint16)
+    Cd, ii = _f64(C), _i32(idx)
+    N, D = Xb.shape
+    assert Cd.shape[1] == D and ii.shape[0] == N
+    return float(lib().kmo_objective_assigned_bf16(_p(Xb), _p(Cd), _p(ii), N, D))
 
 
 def round_bf16(a) -> np.ndarray:

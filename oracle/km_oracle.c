@@ -19,8 +19,9 @@
  * Readings where the pages are silent (tie rule, empty clusters, objective
  * timing) are the plainest ones and are listed in the design notes.
  * Distances use the direct form sum_j (x_ij - c_kj)^2, never the expanded
- * ||x||^2 - 2 x.c + ||c||^2 form the GPU uses.  OpenMP splits only the loop
- * over points of the assignment; every per-cluster sum runs in point order.
+ * ||x||^2 - 2 x.c + ||c||^2 form the GPU uses.  OpenMP splits only loops
+ * over points (the assignment, and the objective of a given assignment in
+ * fixed blocks); every per-cluster sum runs in point order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -123,6 +124,49 @@ double kmo_objective(const double* d1, int64_t N) {
   double s = 0.0;
   for (int64_t i = 0; i < N; ++i) s += d1[i];
   return s;
+}
+
+/*
+ * Objective of a given assignment, for point sets too large to convert to
+ * float64 at once: J = sum_i ||x_i - c_{idx[i]}||^2 (direct form), with X
+ * given as raw bfloat16 bit patterns.  A bfloat16 value is the upper 16 bits
+ * of a float32, so it widens exactly: place the bits in the top half of a
+ * 32-bit word, read it as a float, widen to double.  Points are summed in
+ * blocks of 4096, each block sequentially, and the block sums sequentially
+ * in block order (the order does not depend on the thread count).
+ *   Xbits: N x D uint16, C: K x D float64, idx: N entries in [0, K).
+ */
+static double bf16_bits_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+double kmo_objective_assigned_bf16(const uint16_t* Xbits, const double* C, const int32_t* idx,
+                                   int64_t N, int D) {
+  const int64_t blk = 4096;
+  const int64_t nb = (N + blk - 1) / blk;
+  double* part = (double*)calloc((size_t)(nb > 0 ? nb : 1), sizeof(double));
+  int64_t b;
+#pragma omp parallel for schedule(static)
+  for (b = 0; b < nb; ++b) {
+    double s = 0.0;
+    const int64_t i1 = (b + 1) * blk < N ? (b + 1) * blk : N;
+    for (int64_t i = b * blk; i < i1; ++i) {
+      const uint16_t* x = Xbits + i * (int64_t)D;
+      const double* c = C + (int64_t)idx[i] * D;
+      for (int j = 0; j < D; ++j) {
+        double t = bf16_bits_to_double(x[j]) - c[j];
+        s += t * t;
+      }
+    }
+    part[b] = s;
+  }
+  double J = 0.0;
+  for (b = 0; b < nb; ++b) J += part[b];
+  free(part);
+  return J;
 }
 
 /*

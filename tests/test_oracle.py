@@ -194,6 +194,25 @@ def check_f32_rounding(seed=7):
     assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
 
 
+def check_objective_of_assignment(seed=8):
+    """The objective of a given assignment of bfloat16 points: for the
+    oracle's own argmin it equals the sum of the minimal distances (cdist),
+    for another assignment the direct sum written out in numpy; the bf16
+    points widen exactly (torch's cast to float64)."""
+    rng = np.random.default_rng(seed)
+    for N, D, K in [(5000, 16, 7), (4097, 64, 40), (1, 8, 1)]:
+        Xt = torch.from_numpy(rng.normal(size=(N, D)) * 3).to(torch.bfloat16)
+        Xd = Xt.double().numpy()
+        C = rng.normal(size=(K, D)) * 3
+        Dm = cdist(Xd, C, "sqeuclidean")
+        best = np.argmin(Dm, axis=1).astype(np.int32)
+        want = Dm.min(1).sum()
+        assert abs(oracle.objective_assigned_bf16(Xt, C, best) - want) <= 1e-12 * max(want, 1.0)
+        other = rng.integers(0, K, N).astype(np.int32)
+        want2 = ((Xd - C[other]) ** 2).sum()
+        assert abs(oracle.objective_assigned_bf16(Xt, C, other) - want2) <= 1e-12 * max(want2, 1.0)
+
+
 def check_argsort(seed=5):
     rng = np.random.default_rng(seed)
     for N, K in [(1000, 7), (4096, 256), (10, 40), (1, 1)]:
@@ -205,7 +224,7 @@ def check_argsort(seed=5):
 
 ALL_CHECKS = [check_golden_1d, check_golden_tie, check_assign_vs_cdist, check_bruteforce_integer,
               check_closed_forms, check_separated_mixture, check_invariants_and_sklearn,
-              check_bf16_rounding, check_f32_rounding, check_argsort]
+              check_bf16_rounding, check_f32_rounding, check_objective_of_assignment, check_argsort]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -242,6 +261,9 @@ MUTATIONS = {
                       "if (fabs((double)f) > fabs(in[i])) f = nextafterf(f, 0.0f); out[i] = (double)f; }"),
     "f32_not_rounded": ("for (int64_t i = 0; i < n; ++i) out[i] = (double)(float)in[i];",
                         "for (int64_t i = 0; i < n; ++i) out[i] = in[i];"),
+    "assigned_objective_wrong_row": ("const double* c = C + (int64_t)idx[i] * D;",
+                                     "const double* c = C + (int64_t)idx[i > 0 ? i - 1 : 0] * D;"),
+    "bf16_widened_as_low_half": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b;"),
     "argsort_unstable": ("for (int64_t i = 0; i < N; ++i) perm[cursor[idx[i]]++] = (int32_t)i;",
                          "for (int64_t i = N - 1; i >= 0; --i) perm[cursor[idx[i]]++] = (int32_t)i;"),
     "objective_after_update": ("    J[t] = kmo_objective(d1, N);\n    kmo_update(X, idx, N, D, K, C, counts);",
