@@ -40,7 +40,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, init_rows, make_points, make_problem  # noqa: E402
+from synth import WORKLOADS, init_rows, make_points, make_problem, pool_workload  # noqa: E402
 
 METRIC = "Lloyd iters/sec and assign GFLOP/s (% bf16 tensor peak), update GB/s (% HBM)"
 UNIT = "iters/s"
@@ -251,6 +251,9 @@ def workload_config(wl, world: int, parallelism: str) -> dict:
            "parallelism": parallelism, "ranks": world}
     if wl.host_resident:
         cfg["x"] = "pinned host memory, streamed in 16M-row chunks every iteration"
+    if wl.pool_rows:
+        cfg["x"] = (f"{wl.N} rows never held whole: streamed in 16M-row chunks from a {wl.pool_rows}-row pinned "
+                    f"pool, row i = pool row i mod {wl.pool_rows}")
     return cfg
 
 
@@ -292,11 +295,18 @@ def oracle_rows(wl, X, C0, target_s: float, iters: int, seed: int = 1234):
     g = torch.Generator().manual_seed(seed)
     perm = torch.randperm(n_all, generator=g)
     Cs = (C0 if C0.dim() == 2 else C0[0]).cpu()
-    probe = min(n_all, max(64, min(4096, (1 << 22) // max(1, wl.K))))
-    Xp = Xf[perm[:probe].to(Xf.device)].cpu()
-    t0 = time.perf_counter()
-    oracle.fit(Xp, Cs, 1, mirror=wl.dtype)
-    per_row = (time.perf_counter() - t0) / probe
+    # probe: double the rows until one iteration takes 0.3 s (or all rows),
+    # so thread start-up does not dominate the per-row estimate
+    probe = min(n_all, 64)
+    while True:
+        Xp = Xf[perm[:probe].to(Xf.device)].cpu()
+        t0 = time.perf_counter()
+        oracle.fit(Xp, Cs, 1, mirror=wl.dtype)
+        el = time.perf_counter() - t0
+        if el >= 0.3 or probe >= n_all:
+            break
+        probe = min(n_all, probe * 2)
+    per_row = el / probe
     n = int(min(n_all, max(probe, target_s / max(per_row * iters, 1e-12))))
     return Xf[perm[:n].to(Xf.device)].cpu(), Cs
 
@@ -543,27 +553,42 @@ def h2d_link_gbs(src: torch.Tensor, dev) -> float:
 
 
 def run_host_resident(args, wl, km):
-    """The out-of-core workload: X lives in pinned host memory and every
+    """The out-of-core workloads: X lives in pinned host memory and every
     iteration streams it to the device in chunks (copies overlapped with the
     assignment and update of the previous chunk).  The step is one Lloyd
-    iteration over all N points through km_fit_host; the host link, not a
-    kernel, bounds it, so the roofline reports host->device bytes against the
-    pinned copy bandwidth measured here."""
+    iteration over all N points, through km_fit_host (ooc_268m_k4096) or,
+    for a set never held whole (ooc_1b_k4096: 2^30 rows, row i = pool row
+    i mod 2^28), through km_fit_source with a source that points into the
+    pool.  The host link, not a kernel, bounds these, so the roofline
+    reports host->device bytes against the pinned copy bandwidth measured
+    here."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     chunk = 16 << 20
-    Xh = torch.empty((wl.N, wl.D), dtype=wl.torch_dtype, pin_memory=True)
-    make_points(wl, seed=args.seed, device=dev, out=Xh)
+    pw = pool_workload(wl)
+    Xh = torch.empty((pw.N, wl.D), dtype=wl.torch_dtype, pin_memory=True)
+    make_points(pw, seed=args.seed, device=dev, out=Xh)
     sel = init_rows(wl, args.seed, dev).cpu()
     C0 = Xh[sel].to(dev).contiguous()
     torch.cuda.synchronize()
     link = h2d_link_gbs(Xh[:chunk], dev)
-    km.fit_host(Xh, C0, args.warmup, chunk)
+    P = pw.N
+
+    def source(row0, rows, slot):
+        r = row0 % P
+        return Xh[r:r + rows]
+
+    def fit(iters):
+        if wl.pool_rows:
+            return km.fit_source(source, wl.N, C0, iters, chunk)
+        return km.fit_host(Xh, C0, iters, chunk)
+
+    fit(args.warmup)
     torch.cuda.synchronize()
     with ClockSampler(0) as clk:
         l0 = km.launch_count()
         t0 = time.perf_counter()
-        r = km.fit_host(Xh, C0, args.steps, chunk)
+        r = fit(args.steps)
         Cout = r["C"].cpu()
         dt = time.perf_counter() - t0
         launches = km.launch_count() - l0
@@ -579,11 +604,11 @@ def run_host_resident(args, wl, km):
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": workload_config(wl, 1, "single"),
         "timed_region_s": round(dt, 3),
-        "roofline": {"bound": "h2d", "kernel": "km_fit_host stream", "achieved": round(achieved, 1),
+        "roofline": {"bound": "h2d", "kernel": "chunk stream", "achieved": round(achieved, 1),
                      "peak": round(link, 1), "unit": "GB/s", "frac": round(achieved / link, 4),
                      "peak_kind": "pinned host->device copy measured in this run (best of 5, 16M-row chunk)",
                      "traffic": None, "algorithmic_per_launch": xbytes},
-        "gpu_launches": int(launches) // max(args.steps, 1),
+        "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
@@ -630,8 +655,9 @@ def run_reference(args, world, rank):
     wl = WORKLOADS[args.workload]
     gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
     if wl.host_resident:
-        # rows are iid: the first rows of the host-resident set are a sample of it
-        base = wl.with_(N=min(wl.N, 1 << 22), host_resident=False)
+        # rows are iid: the first rows of the host-resident set (of its pool)
+        # are a sample of it
+        base = pool_workload(wl).with_(N=min(pool_workload(wl).N, 1 << 22), host_resident=False)
         X, C0 = make_inputs(base, args.seed, gen_dev)
     else:
         X, C0 = make_inputs(wl if wl.B == 1 else wl.with_(B=1), args.seed, gen_dev)

@@ -257,6 +257,32 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
                 double* objective_hist, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * A source of point rows for km_fit_source: returns a pointer to the rows
+ * [row0, row0 + rows) of the point set (rows x D elements of the fit's
+ * dtype, row-major) in page-locked host memory.  `slot` is 0 or 1: the
+ * memory returned for a slot must stay valid and unchanged until the library
+ * asks for the same slot again (by then the copy out of it has completed),
+ * so a source may fill two caller-owned staging buffers in turn, or point
+ * into a larger pinned pool.  Return NULL to abort the fit
+ * (KM_ERR_INVALID_ARG).  Called on the thread that called km_fit_source.
+ */
+typedef const void* (*km_chunk_source)(void* user, int64_t row0, int64_t rows, int slot);
+
+/*
+ * km_fit_host for point sets that are never held whole in host memory
+ * (Flash-KMeans §2.3 Chunked Stream Overlap; §4 Results runs one billion
+ * points, beyond the device's memory): the rows come chunk by chunk from
+ * `source`, every iteration, in order.  The host asks for chunk c+2 once the
+ * copy of chunk c has finished, so filling a staging buffer on the host
+ * overlaps the copy and the compute of the chunks before it.  Same
+ * arguments, results and workspace (KM_OP_FIT_HOST) as km_fit_host, with
+ * `source` and `user` in place of X_host; synchronous.
+ */
+int km_fit_source(km_chunk_source source, void* user, const void* C0, int64_t N, int D, int K, int dtype, int iters,
+                  int64_t chunk_rows, float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * km_assign for callers that cannot allocate device memory.  Some callers
  * own every byte of device memory: a host framework that serves memory only
  * from its own pool and forbids side allocations, or a latency-critical loop

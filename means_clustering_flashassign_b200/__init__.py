@@ -28,7 +28,7 @@ from . import build as _build
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
            "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static",
            "ablation_assign_materialized", "ablation_update_atomic", "plan", "update_accumulate",
-           "finalize_sums", "fit_data_parallel", "pack_layout", "exchange_packed", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "finalize_sums", "fit_data_parallel", "pack_layout", "exchange_packed", "fit_source", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -39,10 +39,14 @@ STATUS = {0: "KM_OK", 1: "KM_ERR_INVALID_ARG", 2: "KM_ERR_UNSUPPORTED", 3: "KM_E
 EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size", "km_workspace_status",
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_timed", "km_fit_host", "km_selftest_timeout",
            "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
-           "km_ablation_update_atomic", "km_plan_describe", "km_update_accumulate", "km_finalize_sums"]
+           "km_ablation_update_atomic", "km_plan_describe", "km_update_accumulate", "km_finalize_sums",
+           "km_fit_source"]
 
 _lock = threading.Lock()
 _lib = None
+
+# km_chunk_source: const void* (*)(void* user, int64_t row0, int64_t rows, int slot)
+CHUNK_SOURCE = ctypes.CFUNCTYPE(ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int)
 
 
 class KMError(RuntimeError):
@@ -92,6 +96,7 @@ def library() -> ctypes.CDLL:
             L.km_fit_timed.argtypes = [P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, P, P]
             L.km_launch_count.restype = ctypes.c_uint64
             L.km_assign_static.argtypes = [P, P, I, I64, I, I, I, P, P, P, P]
+            L.km_fit_source.argtypes = [CHUNK_SOURCE, P, P, I64, I, I, I, I, I64, P, P, P, P, P, SZ, P]
             for f in EXPORTS:
                 getattr(L, f).restype = getattr(L, f).restype or I
             _lib = L
@@ -576,6 +581,62 @@ def fit_host(X_host: torch.Tensor, C0: torch.Tensor, iters: int, chunk_rows: int
         _check(library().km_fit_host(_ptr(X_host), _ptr(C0), N, D, K, dt, iters, chunk_rows, _ptr(C_out),
                                      _ptr(idx_out), _ptr(counts_out), _ptr(obj), _ptr(ws), ws.numel(),
                                      _stream(stream)))
+    return dict(C=C_out, idx=idx_out, counts=counts_out, objective=obj)
+
+
+def fit_source(source, N: int, C0: torch.Tensor, iters: int, chunk_rows: int, *, dtype=torch.bfloat16,
+               C_out=None, idx_out=None, want_idx: bool = False, counts_out=None, workspace=None, stream=None):
+    """Out-of-core Lloyd over a point set that is never held whole: every
+    iteration, source(row0, rows, slot) returns a pinned CPU tensor holding
+    rows [row0, row0 + rows) (shape (rows, D), the given dtype).  The tensor
+    returned for a slot (0 or 1) is kept alive and unchanged until that slot
+    is asked for again.  Same results as fit_host on the concatenated rows.
+
+    Synchronous.  Returns dict(C, idx or None, counts, objective (CPU float64 [iters])).
+    """
+    _contig_cuda(C0, "C0")
+    if C0.dim() != 2 or C0.dtype != dtype:
+        raise ValueError("C0 must be [K, D] of the points' dtype")
+    K, D = C0.shape
+    dt = _dtype_code(C0)
+    dev = C0.device
+    _check_stream(stream, dev)
+    held = [None, None]      # the tensors behind the two slots
+    errors = []
+    es = C0.element_size()
+
+    def trampoline(_user, row0, rows, slot):
+        try:
+            t = source(int(row0), int(rows), int(slot))
+            if (t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != dtype
+                    or tuple(t.shape) != (rows, D)):
+                raise ValueError(f"the source must return a pinned contiguous {dtype} tensor of shape ({rows}, {D})")
+            held[slot] = t
+            return t.data_ptr()
+        except BaseException as e:  # the library sees NULL and stops
+            errors.append(e)
+            return None
+
+    cb = CHUNK_SOURCE(trampoline)
+    with torch.cuda.device(dev):
+        C_out = torch.empty((K, D), dtype=torch.float32, device=dev) if C_out is None else C_out
+        _check_tensor(C_out, "C_out", dev, torch.float32, (K, D))
+        if idx_out is None and want_idx:
+            idx_out = torch.empty(N, dtype=torch.int32, device=dev)
+        if idx_out is not None:
+            _check_tensor(idx_out, "idx_out", dev, torch.int32, (N,))
+        counts_out = torch.empty(K, dtype=torch.int32, device=dev) if counts_out is None else counts_out
+        _check_tensor(counts_out, "counts_out", dev, torch.int32, (K,))
+        obj = torch.empty(iters, dtype=torch.float64)
+        ws = _workspace(OP_FIT_HOST, 1, N, D, K, dt, dev, workspace, chunk_rows)
+        _check_tensor(ws, "workspace", dev, torch.uint8)
+        st = library().km_fit_source(cb, None, _ptr(C0), N, D, K, dt, iters, chunk_rows, _ptr(C_out),
+                                     _ptr(idx_out), _ptr(counts_out), _ptr(obj), _ptr(ws), ws.numel(),
+                                     _stream(stream))
+    if errors:
+        raise errors[0]
+    _check(st)
+    del es
     return dict(C=C_out, idx=idx_out, counts=counts_out, objective=obj)
 
 

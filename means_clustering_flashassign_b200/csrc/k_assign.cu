@@ -61,6 +61,8 @@ struct AssignK {
   uint32_t zero;    // always 0; keeps the epilogue's column constants in registers
   int32_t* hist0;   // may be null: sort pass-0 block digit counts, [row / hist_T][digit]
   int hist_T, hist_R;
+  int32_t* rk;      // may be null (with hist0): per point, the cluster id | rank << 20 | (count - 1) << 25
+  int32_t* kcnt;    // may be null (with hist0): members per cluster, accumulated
   unsigned int* status;
   uint64_t limit_ns;
 };
@@ -498,8 +500,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           // warp, not one per point)
           const int dig = valid ? (bk & (p.hist_R - 1)) : -1;
           const uint32_t peers = __match_any_sync(0xffffffffu, dig);
-          if (valid && lane == __ffs(peers) - 1)
-            atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + dig, __popc(peers));
+          const int rank_in = __popc(peers & ((1u << lane) - 1u));
+          if (valid && rank_in == 0) atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + dig, __popc(peers));
+          // The sort's first scatter ranks equal digits inside the same
+          // 32-point groups: hand it this group's rank and size with the key
+          if (p.rk && valid)
+            p.rk[static_cast<int64_t>(b) * p.rows + row] =
+                bk | (rank_in << 20) | ((__popc(peers) - 1) << 25);
+          // members per cluster (two-pass sorts take the cluster starts from these)
+          if (p.kcnt) {
+            const uint32_t same = __match_any_sync(0xffffffffu, valid ? bk : -1);
+            if (valid && lane == __ffs(same) - 1) atomicAdd(p.kcnt + bk, __popc(same));
+          }
         }
         double ds = static_cast<double>(md);
 #pragma unroll
@@ -585,6 +597,8 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.hist0 = a.B == 1 ? a.hist0 : nullptr;
   k.hist_T = a.hist_T;
   k.hist_R = a.hist_R;
+  k.rk = k.hist0 ? a.rk : nullptr;
+  k.kcnt = k.hist0 ? a.kcnt : nullptr;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN, PAIR>(k.natoms, k.XB, k.CS);

@@ -11,9 +11,15 @@
 //            digit's counts, plus the digit totals (digit-major order of the
 //            runs makes the concatenation the stable counting-sort offsets)
 //   scatter  each block ranks its keys stably with per-warp counters
-//            (ballots group equal digits inside a warp step), scans the
-//            digit totals and its own digit counts, and writes every element
-//            to its final position.
+//            (equal digits inside a warp step grouped by ballots -- or, on
+//            the first pass of a fit, by the assignment kernel, which hands
+//            each key over with its rank and count inside its 32-point
+//            group), scans the digit totals and its own digit counts, and
+//            writes every element to its final position.
+// Cluster starts: a one-pass sort's digit is the cluster id, so the scatter
+// writes start[]; a two-pass sort inside a fit takes them from the cluster
+// sizes the assignment kernel counted (one more column-scan block), else
+// from the sorted keys (k_bounds).
 // The sort is deterministic: equal keys keep point order, so the permutation
 // is unique and the later float sums always run in the same order.
 #include <cstdint>
@@ -60,11 +66,52 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
 // its part, the parts are scanned in shared memory, and each warp rewrites
 // its part as running prefixes.
 constexpr int kColscanWarps = 32;
+
+// start[0..K] of a two-pass sort from the cluster sizes the assignment kernel
+// counted: an exclusive scan over the clusters (each thread a contiguous run
+// of them, then a block scan of the run sums), start[K] = n; the sizes are
+// zeroed for the next accumulation.  One block of kColscanWarps warps.
+__device__ void starts_from_sizes(int32_t* __restrict__ kcnt, int K, int64_t n, int32_t* __restrict__ start,
+                                  int32_t (*part)[32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nt = kColscanWarps * 32;
+  const int per = (K + nt - 1) / nt;
+  const int k0 = static_cast<int>(threadIdx.x) * per;
+  const int k1 = k0 + per < K ? k0 + per : K;
+  int32_t own = 0;
+  for (int k = k0; k < k1; ++k) own += kcnt[k];
+  int32_t x = own;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) part[0][warp] = x;
+  __syncthreads();
+  int32_t run = x - own;
+  for (int w = 0; w < warp; ++w) run += part[0][w];
+  for (int k = k0; k < k1; ++k) {
+    const int32_t c = kcnt[k];
+    start[k] = run;
+    run += c;
+    kcnt[k] = 0;
+  }
+  if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
+}
+
+// With kcnt (two-pass sorts whose cluster sizes the assignment kernel
+// counted) the grid has one more block, which writes start[] from them.
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
-                                                                     int64_t nblk, int32_t* __restrict__ total) {
+                                                                     int64_t nblk, int32_t* __restrict__ total,
+                                                                     int32_t* __restrict__ kcnt, int K, int64_t n,
+                                                                     int32_t* __restrict__ start) {
   __shared__ int32_t part[kColscanWarps][32];
   pdl_trigger();
   pdl_wait();
+  if (kcnt && blockIdx.x == gridDim.x - 1) {
+    starts_from_sizes(kcnt, K, n, start, part);
+    return;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d = blockIdx.x * 32 + lane;
   const bool ok = d < R;
@@ -194,7 +241,7 @@ __device__ __forceinline__ void block_scan_pair(int32_t a, int32_t b, int32_t& e
 // the next accumulation.
 // Resident blocks per SM the register budget is sized for: what the shared
 // memory (2T + 9R ints) admits, 1 to 4.
-template <int IPT, int RPT, bool PAIRS>
+template <int IPT, int RPT, bool PAIRS, bool PRE>
 __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT < 8 ? 4 : 2)) k_sort_scatter(
     const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n, int shift, int R, int bits,
     int32_t* __restrict__ blkhist, const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
@@ -236,6 +283,10 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   auto valid = [&](int s) { return 32 * s < nw; };
   auto digit = [&](int32_t k) { return (k >> shift) & (R - 1); };
   int32_t key[IPT], val[PAIRS ? IPT : 1];
+  // PRE: the key word also holds the point's rank among the equal digits of
+  // its 32-point group (bits 20..24) and the group's count of that digit
+  // minus one (bits 25..29), as the assignment kernel found them
+  uint32_t pre[PRE ? IPT : 1];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {  // all loads first
     const int64_t i = w0 + s * 32 + lane;
@@ -243,6 +294,10 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
       const int2 pk = i < n ? pairs_in[i] : make_int2(0, 0);
       val[s] = pk.x;
       key[s] = pk.y;
+    } else if constexpr (PRE) {
+      const int32_t w = i < n ? keys_in[i] : 0;
+      key[s] = clamp_key(w & 0xFFFFF, K);
+      pre[s] = static_cast<uint32_t>(w) >> 20;
     } else {
       key[s] = i < n ? clamp_key(keys_in[i], K) : 0;
     }
@@ -255,21 +310,35 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   }
   // digit bits: R = 256 RPT exactly when RPT > 1; at most 8 when RPT == 1
   constexpr int NB = RPT == 1 ? 8 : RPT == 2 ? 9 : RPT == 4 ? 10 : RPT == 8 ? 11 : 12;
-  uint32_t peers[IPT];
+  // per step: this lane's rank among the step's lanes of equal digit, and
+  // (on the group's first lane) the group's size
+  uint32_t gr[IPT], gn[IPT];
+  if constexpr (PRE) {
 #pragma unroll
-  for (int s = 0; s < IPT; ++s) peers[s] = match_digit<NB>(digit(key[s]), bits, valid(s));
+    for (int s = 0; s < IPT; ++s) {
+      gr[s] = pre[s] & 31u;
+      gn[s] = ((pre[s] >> 5) & 31u) + 1u;
+    }
+  } else {
+    const uint32_t ltm = lanemask_lt();
+#pragma unroll
+    for (int s = 0; s < IPT; ++s) {
+      const uint32_t peers = match_digit<NB>(digit(key[s]), bits, valid(s));
+      gr[s] = __popc(peers & ltm);
+      gn[s] = __popc(peers);
+    }
+  }
   __syncthreads();  // counters zeroed
 
-  const uint32_t ltm = lanemask_lt();
   int32_t rank[IPT];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const bool v = valid(s);
     int32_t* cp = wcnt + warp * R + digit(key[s]);
     const int32_t before = v ? *cp : 0;
-    rank[s] = before + __popc(peers[s] & ltm);
+    rank[s] = before + static_cast<int32_t>(gr[s]);
     __syncwarp();
-    if (v && lane == __ffs(peers[s]) - 1) *cp = before + __popc(peers[s]);
+    if (v && gr[s] == 0) *cp = before + static_cast<int32_t>(gn[s]);
     __syncwarp();
   }
   __syncthreads();
@@ -326,7 +395,9 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int32_t pt = PAIRS ? val[PAIRS ? s : 0] : static_cast<int32_t>(w0 + s * 32 + lane);
-    if (rank[s] >= 0) stage[rank[s]] = make_int2(pt, key[s]);
+    // ranks are below T unless the counts came from an assignment kernel that
+    // gave up on a bounded wait: stay inside the stage then
+    if (rank[s] >= 0 && rank[s] < T) stage[rank[s]] = make_int2(pt, key[s]);
   }
   __syncthreads();
   const int64_t left = n - t0;
@@ -370,27 +441,27 @@ static size_t scatter_smem(int R, int T) {
   return (2 * static_cast<size_t>(T) + static_cast<size_t>(kSortWarps + 1) * R + 2 * kSortWarps) * 4;
 }
 
-template <int IPT, int RPT, bool PAIRS>
+template <int IPT, int RPT, bool PAIRS, bool PRE>
 static cudaError_t launch_scatter_t(int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys, const int2* pin,
                                     int64_t n, int shift, int R, int bits, int32_t* bh, const int32_t* total,
                                     int2* out, int32_t* perm, int32_t* st, int K) {
-  auto kern = k_sort_scatter<IPT, RPT, PAIRS>;
+  auto kern = k_sort_scatter<IPT, RPT, PAIRS, PRE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
   if (e != cudaSuccess) return e;
   return launch_chained(kern, dim3(static_cast<unsigned>(nblk)), dim3(kSortThreads), sm, s, keys, pin, n, shift, R,
                         bits, bh, total, out, perm, st, K);
 }
 
-template <int IPT, bool PAIRS>
+template <int IPT, bool PAIRS, bool PRE>
 static cudaError_t launch_scatter_r(int rpt, int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys,
                                     const int2* pin, int64_t n, int shift, int R, int bits, int32_t* bh,
                                     const int32_t* total, int2* out, int32_t* perm, int32_t* st, int K) {
   switch (rpt) {
-    case 1: return launch_scatter_t<IPT, 1, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 2: return launch_scatter_t<IPT, 2, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 4: return launch_scatter_t<IPT, 4, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 8: return launch_scatter_t<IPT, 8, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 16: return launch_scatter_t<IPT, 16, PAIRS>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 1: return launch_scatter_t<IPT, 1, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 2: return launch_scatter_t<IPT, 2, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 4: return launch_scatter_t<IPT, 4, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 8: return launch_scatter_t<IPT, 8, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 16: return launch_scatter_t<IPT, 16, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -418,7 +489,11 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     else
       e = cudaSuccess;
     if (e != cudaSuccess) return e;
-    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32), dim3(kColscanWarps * 32), 0, s, bh, R, nblk, a.total);
+    // a two-pass sort with counted cluster sizes takes start[] from them in
+    // the first column scan (one more block) and needs no bounds kernel
+    int32_t* kc = ps == 0 && c.passes > 1 ? a.kcnt : nullptr;
+    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 + (kc ? 1 : 0)), dim3(kColscanWarps * 32), 0, s, bh, R,
+                       nblk, a.total, kc, a.K, a.n, a.start);
     if (e != cudaSuccess) return e;
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
@@ -428,18 +503,23 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     int32_t* st = (last && c.passes == 1) ? a.start : nullptr;
     const int rpt = scatter_rpt(R);
     if (pairs_in)
-      e = c.IPT == 16 ? launch_scatter_r<16, true>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R, bits,
-                                                   bh, a.total, out, perm, st, a.K)
-                      : launch_scatter_r<8, true>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R, bits,
-                                                  bh, a.total, out, perm, st, a.K);
+      e = c.IPT == 16 ? launch_scatter_r<16, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
+                                                          bits, bh, a.total, out, perm, st, a.K)
+                      : launch_scatter_r<8, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
+                                                         bits, bh, a.total, out, perm, st, a.K);
+    else if (a.rk)
+      e = c.IPT == 16 ? launch_scatter_r<16, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
+                                                          bh, a.total, out, perm, st, a.K)
+                      : launch_scatter_r<8, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
+                                                         bh, a.total, out, perm, st, a.K);
     else
-      e = c.IPT == 16 ? launch_scatter_r<16, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R, bits, bh,
-                                                    a.total, out, perm, st, a.K)
-                      : launch_scatter_r<8, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R, bits, bh,
-                                                   a.total, out, perm, st, a.K);
+      e = c.IPT == 16 ? launch_scatter_r<16, false, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R,
+                                                           bits, bh, a.total, out, perm, st, a.K)
+                      : launch_scatter_r<8, false, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R,
+                                                          bits, bh, a.total, out, perm, st, a.K);
     if (e != cudaSuccess) return e;
   }
-  if (c.passes > 1) {
+  if (c.passes > 1 && !a.kcnt) {
     const int64_t cnt = a.n + 1;
     count_launch();
     e = launch_chained(k_bounds, dim3(static_cast<unsigned>((cnt + 255) / 256)), dim3(256), 0, s, a.pairs, a.n, a.K,

@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <atomic>
+#include <functional>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -366,6 +367,10 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     p.off_pl = take(sizeof(float) * gc.nchunks * D);
     p.off_pr = take(sizeof(float) * gc.nchunks * D);
   }
+  if ((op == KM_OP_FIT || op == KM_OP_FIT_HOST) && B == 1 && !p.small_update) {
+    p.off_rk = take(sizeof(int32_t) * static_cast<size_t>(p.rows));
+    if (sc.passes > 1) p.off_kcnt = take(sizeof(int32_t) * static_cast<size_t>(K));
+  }
   if (op == KM_OP_FIT_HOST) {
     p.off_dbuf0 = take(static_cast<size_t>(p.chunk_rows) * D * p.es);
     p.off_dbuf1 = take(static_cast<size_t>(p.chunk_rows) * D * p.es);
@@ -415,7 +420,8 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
-                    bool hist0_ready = false, double* acc_ext = nullptr, double* cnt_ext = nullptr) {
+                    bool hist0_ready = false, double* acc_ext = nullptr, double* cnt_ext = nullptr,
+                    const int32_t* rk = nullptr, int32_t* kcnt = nullptr) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
@@ -423,6 +429,8 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
               hist0_ready,
+              rk,
+              kcnt,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),
@@ -599,13 +607,19 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   // digit per block; the sort's scatter zeroes the counts again after use.
   const bool fused_hist = B == 1 && !p.small_update;
   int32_t* hist0 = fused_hist ? at<int32_t>(c.ws, p.off_blkhist) : nullptr;
+  // with the counts, the assignment kernel hands the sort each point's key
+  // with its rank inside its 32-point group, and (two passes) the cluster sizes
+  int32_t* rk = fused_hist ? at<int32_t>(c.ws, p.off_rk) : nullptr;
+  int32_t* kcnt = fused_hist && p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
   if (fused_hist)
     KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
+  chain_break();
+  if (kcnt) KM_CUDA(cudaMemsetAsync(kcnt, 0, sizeof(int32_t) * static_cast<size_t>(K), c.s));
   chain_break();
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
-                 &groups, hist0, p.sc.T, 1 << p.sc.bits[0]};
+                 &groups, hist0, p.sc.T, 1 << p.sc.bits[0], rk, kcnt};
     if (ev && (per_phase || t == 0)) {
       KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t : 0], c.s));
       chain_break();
@@ -626,7 +640,8 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
                             C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
                             caug + static_cast<int64_t>(b) * p.Kp * 32,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
-                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, fused_hist);
+                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, fused_hist, nullptr,
+                            nullptr, rk, kcnt);
         if (r != KM_OK) return r;
       }
     }
@@ -712,11 +727,25 @@ int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, 
   return r;
 }
 
-int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int dtype, int iters, int64_t chunk_rows,
-                float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
-                size_t workspace_bytes, void* stream) {
-  g_err.clear();
-  if (!X_host || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X_host, C0 and C_out are required");
+}  // extern "C"
+
+namespace {
+
+// Rows [r0, r0 + nr) of a streamed point set for staging slot `slot` (0 or
+// 1): a pointer to page-locked host memory, or null with *why set.
+using ChunkFn = std::function<const void*(int64_t r0, int64_t nr, int slot, const char** why)>;
+
+// The chunked out-of-core fit (Flash-KMeans §2.3 Chunked Stream Overlap):
+// each iteration streams the point set to the device in chunks of
+// chunk_rows rows through two device buffers, the copy of chunk c+1 on a
+// library-owned copy stream overlapping the assignment and update of chunk
+// c on `stream`; per-cluster sums accumulate across chunks in float64, in
+// chunk order.  With slot_reuse the host memory behind a slot may be
+// rewritten by the source: before asking for slot s again the host waits
+// until the previous copy out of slot s has completed.
+int fit_stream(const ChunkFn& chunk, bool slot_reuse, const void* C0, int64_t N, int D, int K, int dtype,
+               int iters, int64_t chunk_rows, float* C_out, int32_t* idx_out, int32_t* counts_out,
+               double* objective_hist, void* workspace, size_t workspace_bytes, void* stream) {
   if (iters < 0 || iters > kMaxHostIters) return fail(KM_ERR_INVALID_ARG, "iters must be in [0, %lld]",
                                                       static_cast<long long>(kMaxHostIters));
   if (!aligned16(C0) || !aligned16(C_out)) return fail(KM_ERR_INVALID_ARG, "C0 and C_out must be 16-byte aligned");
@@ -724,9 +753,6 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
   int r = prepare(c, KM_OP_FIT_HOST, 1, N, D, K, dtype, chunk_rows, workspace, workspace_bytes, stream);
   if (r != KM_OK) return r;
   const Plan& p = c.p;
-  cudaPointerAttributes pa;
-  KM_CUDA(cudaPointerGetAttributes(&pa, X_host));
-  if (pa.type != cudaMemoryTypeHost) return fail(KM_ERR_INVALID_ARG, "X_host must be page-locked host memory");
   void* xaug = at<void>(c.ws, p.off_xaug);
   void* caug = at<void>(c.ws, p.off_caug);
   void* clp = at<void>(c.ws, p.off_clp);
@@ -768,6 +794,12 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
     int32_t* hist0 = at<int32_t>(c.ws, p.off_blkhist);
     KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
     chain_break();
+    int32_t* rk = at<int32_t>(c.ws, p.off_rk);
+    int32_t* kcnt = p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
+    if (kcnt) {
+      KM_CUDA(cudaMemsetAsync(kcnt, 0, sizeof(int32_t) * static_cast<size_t>(K), c.s));
+      chain_break();
+    }
     for (int i = 0; i < 2; ++i) {
       KM_CUDA(cudaEventRecord(ev_free[i], c.s));
       chain_break();
@@ -785,11 +817,17 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         const int bi = static_cast<int>(g & 1);
         const int64_t r0 = ch * p.chunk_rows;
         const int64_t nr = N - r0 < p.chunk_rows ? N - r0 : p.chunk_rows;
+        // the slot's previous copy (chunk g - 2) must be done before the
+        // source may write that slot again
+        if (slot_reuse && g >= 2) KM_CUDA(cudaEventSynchronize(ev_copied[bi]));
+        const char* why = "";
+        const void* src = chunk(r0, nr, bi, &why);
+        if (!src) return fail(KM_ERR_INVALID_ARG, "rows %lld..%lld: %s", static_cast<long long>(r0),
+                              static_cast<long long>(r0 + nr), why);
         KM_CUDA(cudaStreamWaitEvent(cs, ev_free[bi], 0));
         chain_break();
         if (fault_hit(kFaultH2D)) return fail(KM_ERR_CUDA, "cudaMemcpyAsync of chunk %lld failed", (long long)ch);
-        KM_CUDA(cudaMemcpyAsync(dbuf[bi], static_cast<const uint8_t*>(X_host) + r0 * rowb, nr * rowb,
-                                cudaMemcpyHostToDevice, cs));
+        KM_CUDA(cudaMemcpyAsync(dbuf[bi], src, nr * rowb, cudaMemcpyHostToDevice, cs));
         chain_break();
         KM_CUDA(cudaEventRecord(ev_copied[bi], cs));
         chain_break();
@@ -808,12 +846,12 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
         int64_t groups = 0;
         AssignArgs a{&xmap, &xamap, &cmap, &camap, 1,       nr,      K,           p.Kp,
                      idxc,  nullptr, tobj,  c.status(), wait_limit_ns(), &groups, hist0, p.sc.T,
-                     1 << p.sc.bits[0]};
+                     1 << p.sc.bits[0], rk, kcnt};
         KM_CUDA(launch_assign(pc, a, c.s));
         Ctx cc = c;
         cc.p = pc;
         rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1,
-                             true);
+                             true, nullptr, nullptr, rk, kcnt);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
         chain_break();
@@ -831,6 +869,55 @@ int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int
   return r;
 }
 
+}  // namespace
+
+extern "C" {
+
+int km_fit_host(const void* X_host, const void* C0, int64_t N, int D, int K, int dtype, int iters, int64_t chunk_rows,
+                float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!X_host || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X_host, C0 and C_out are required");
+  cudaPointerAttributes pa;
+  const cudaError_t pe = cudaPointerGetAttributes(&pa, X_host);
+  if (pe != cudaSuccess || pa.type != cudaMemoryTypeHost) {
+    if (pe != cudaSuccess && pe != cudaErrorInvalidValue) {
+      const int rc = check_device();
+      if (rc != KM_OK) return rc;
+    }
+    return fail(KM_ERR_INVALID_ARG, "X_host must be page-locked host memory");
+  }
+  const size_t rowb = static_cast<size_t>(D) * (dtype == KM_BF16 ? 2 : 4);
+  const ChunkFn chunk = [&](int64_t r0, int64_t, int, const char**) -> const void* {
+    return static_cast<const uint8_t*>(X_host) + r0 * rowb;
+  };
+  return fit_stream(chunk, false, C0, N, D, K, dtype, iters, chunk_rows, C_out, idx_out, counts_out, objective_hist,
+                    workspace, workspace_bytes, stream);
+}
+
+int km_fit_source(km_chunk_source source, void* user, const void* C0, int64_t N, int D, int K, int dtype, int iters,
+                  int64_t chunk_rows, float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  if (!source || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "source, C0 and C_out are required");
+  const ChunkFn chunk = [&](int64_t r0, int64_t nr, int slot, const char** why) -> const void* {
+    const void* ptr = source(user, r0, nr, slot);
+    if (!ptr) {
+      *why = "the chunk source returned no rows";
+      return nullptr;
+    }
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, ptr) != cudaSuccess || pa.type != cudaMemoryTypeHost) {
+      cudaGetLastError();
+      *why = "the chunk source returned memory that is not page-locked host memory";
+      return nullptr;
+    }
+    return ptr;
+  };
+  return fit_stream(chunk, true, C0, N, D, K, dtype, iters, chunk_rows, C_out, idx_out, counts_out, objective_hist,
+                    workspace, workspace_bytes, stream);
+}
+
 int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* start, void* workspace,
                size_t workspace_bytes, void* stream) {
   g_err.clear();
@@ -845,6 +932,8 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
               false,
+              nullptr,
+              nullptr,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),

@@ -137,6 +137,7 @@ struct Plan {
   size_t off_blkhist = 0, off_blkhist1 = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0, off_objpart = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
+  size_t off_rk = 0, off_kcnt = 0;  // fused-sort inputs (single-instance fits)
   size_t total = 0;
 };
 
@@ -179,6 +180,8 @@ struct AssignArgs {
   int64_t* obj_groups;  // host out (may be null): 4-double groups of partials per instance
   int32_t* hist0;       // may be null: pass-0 block digit counts to accumulate (B == 1 only)
   int hist_T, hist_R;   // keys per sort block, pass-0 radix
+  int32_t* rk = nullptr;    // with hist0, may be null: packed keys for the sort's first scatter
+  int32_t* kcnt = nullptr;  // with hist0, may be null: cluster sizes to accumulate (zero on entry)
 };
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s);
 
@@ -196,6 +199,10 @@ struct SortArgs {
   int32_t* blkhist;     // [nblk][R0] pass-0 block digit counts (zeroed again by the pass-0 scatter)
   int32_t* blkhist1;    // [nblk][R1] pass-1 block digit counts (two-pass sorts only)
   bool hist0_ready;     // pass-0 counts were accumulated by the assignment kernel
+  const int32_t* rk;    // may be null: the keys with their 32-point group rank and size (from the
+                        // assignment kernel); the first scatter then needs no digit ballots
+  int32_t* kcnt;        // may be null: cluster sizes counted by the assignment kernel; a two-pass
+                        // sort then takes start[] from them (and zeroes them) instead of k_bounds
   int32_t* total;       // [Rmax]
   int2* pairs_tmp;      // [n] (two-pass sorts only)
   int2* pairs;          // [n] sorted (point index, cluster id)

@@ -12,5 +12,6 @@ from .mixtures import (  # noqa: F401
     make_points,
     make_problem,
     init_rows,
+    pool_workload,
     instance_seed,
 )

@@ -37,6 +37,8 @@ class Workload:
     weights: str = "equal"       # "equal" or "zipf1.2"
     iters: int = 10
     host_resident: bool = False  # X lives in pinned host memory and is streamed
+    pool_rows: int = 0           # > 0: the N rows are streamed from a pool of this many rows,
+                                 # row i being pool row i mod pool_rows (the set is never held whole)
 
     @property
     def torch_dtype(self):
@@ -61,6 +63,11 @@ WORKLOADS = {
     # N=268M, D=128, K=4096 bf16 in pinned host memory, streamed in 16M-row chunks
     "ooc_268m_k4096": Workload("ooc_268m_k4096", N=1 << 28, D=128, K=4096,
                                iters=5, host_resident=True),
+    # N=2^30 (one billion) rows, D=128, K=4096 bf16: 256 GiB, never held
+    # whole; streamed in 16M-row chunks from a 2^28-row pinned pool (the
+    # ooc_268m_k4096 points), row i = pool row i mod 2^28
+    "ooc_1b_k4096": Workload("ooc_1b_k4096", N=1 << 30, D=128, K=4096,
+                             iters=3, host_resident=True, pool_rows=1 << 28),
 }
 
 
@@ -126,9 +133,16 @@ def make_points(wl: Workload, seed: int = 0, device="cpu", rows: Optional[slice]
 
 
 def init_rows(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
-    """Indices of the K initial centroids: first K of a seeded permutation of N."""
+    """Indices of the K initial centroids: first K of a seeded permutation of N
+    (of the pool's rows for a pooled workload, so the K rows are distinct)."""
     g = _gen(instance_seed(seed, 999_999), device)
-    return torch.randperm(wl.N, generator=g, device=device)[: wl.K]
+    n = wl.pool_rows if wl.pool_rows else wl.N
+    return torch.randperm(n, generator=g, device=device)[: wl.K]
+
+
+def pool_workload(wl: Workload) -> Workload:
+    """The workload whose points form the pool of a pooled workload."""
+    return wl.with_(N=wl.pool_rows, pool_rows=0) if wl.pool_rows else wl
 
 
 def make_problem(wl: Workload, seed: int = 0, device="cpu"):

@@ -1,10 +1,9 @@
 """Bitwise reproducibility of whole fits on the two-pass sort path.
 
 K = 16,384 clusters need 14-bit keys, so the Sort-Inverse Update sorts in two
-radix passes (histogram, column scan, scatter, twice, then the bounds
-kernel), and the Zipf(1.2) weights put a fifth of the points in one cluster,
-whose sums cross every segmented-sum block and take the finaliser's
-whole-block path.  Every kernel of the iteration chains to the previous one
+radix passes, and a quarter of the points on one spot make one cluster whose
+sums cross every segmented-sum block and take the finaliser's whole-block
+path.  Every kernel of the iteration chains to the previous one
 by programmatic dependent launch.  Ten fits in one process must return the
 same centroids, assignment, counts and objective bit for bit; the objective
 is summed from per-tile partials in a fixed order, so it does not depend on
@@ -28,6 +27,11 @@ def _zipf_problem(N, K, seed):
 
 def test_two_pass_zipf_fits_are_bit_identical():
     X, C0 = _zipf_problem(1 << 20, 16384, seed=3)
+    # random-point centroids split the Zipf components' points among many
+    # clusters; a quarter of the points on one spot makes one hot cluster
+    # whose sums cross every segmented-sum block (the finaliser's
+    # whole-block path)
+    X[::4] = X[0]
     assert km.plan(km.OP_FIT, 1, X.shape[0], 128, 16384, km.BF16)["sort_passes"] == 2
     ref = None
     for _ in range(10):
@@ -42,7 +46,7 @@ def test_two_pass_zipf_fits_are_bit_identical():
         assert torch.equal(cur[2], ref[2])
         assert torch.equal(cur[3], ref[3])
     # the hot cluster crosses many segmented-sum blocks
-    assert int(ref[2].max()) > 0.1 * X.shape[0]
+    assert int(ref[2].max()) >= X.shape[0] // 4
 
 
 def test_fit_objective_equals_the_assign_objective_bitwise_up_to_order():
