@@ -8,7 +8,8 @@ so that the same (workload, seed, device) always yields the same tensors.
 Recipe per instance:
   * component centres: uniform in [-R, R]^D, or N(0, s^2 I);
   * component weights: equal, or Zipf(s) (w_k proportional to (k+1)^-s);
-  * labels: iid categorical draws from the weights;
+  * labels: iid categorical draws from the weights (inverse-CDF lookup of
+    uniform draws; the CDF is a float64 sum on the CPU);
   * points: centre[label] + sigma * N(0, I) in float32, then cast to the
     workload dtype (bfloat16 casts round to nearest even);
   * initial centroids: rows of X at the first K entries of a seeded random
@@ -83,6 +84,13 @@ def _gen(seed: int, device) -> torch.Generator:
 
 
 def _mixture(wl: Workload, seed: int, device):
+    """Generator, component centres and the cumulative component weights.
+
+    The cumulative weights are formed on the CPU in float64 (a fixed
+    sequential sum) and labels are drawn by inverse-CDF lookup of uniform
+    draws: a device cumulative sum (as inside a CUDA multinomial) may
+    associate its float additions differently from run to run, which moves
+    labels at bucket edges and makes the same seed give different points."""
     comps = wl.comps or wl.K
     g = _gen(seed, device)
     if wl.centers == "uniform10":
@@ -92,13 +100,15 @@ def _mixture(wl: Workload, seed: int, device):
     else:
         raise ValueError(wl.centers)
     if wl.weights == "equal":
-        w = torch.ones(comps, device=device)
+        w = torch.ones(comps, dtype=torch.float64)
     elif wl.weights.startswith("zipf"):
         s = float(wl.weights[4:])
-        w = torch.arange(1, comps + 1, device=device, dtype=torch.float64).pow(-s).float()
+        w = torch.arange(1, comps + 1, dtype=torch.float64).pow(-s)
     else:
         raise ValueError(wl.weights)
-    return g, mu.float(), w / w.sum()
+    cdf = torch.cumsum(w, 0)
+    cdf = (cdf / cdf[-1]).to(torch.float32).to(device)
+    return g, mu.float(), cdf
 
 
 def make_points(wl: Workload, seed: int = 0, device="cpu", rows: Optional[slice] = None,
@@ -111,7 +121,7 @@ def make_points(wl: Workload, seed: int = 0, device="cpu", rows: Optional[slice]
     Returns (X, labels) where labels are the generating components (int64),
     or (out, None) when ``out`` is given.
     """
-    g, mu, w = _mixture(wl, seed, device)
+    g, mu, cdf = _mixture(wl, seed, device)
     start = 0 if rows is None else rows.start
     stop = wl.N if rows is None else rows.stop
     n = stop - start
@@ -122,7 +132,8 @@ def make_points(wl: Workload, seed: int = 0, device="cpu", rows: Optional[slice]
     for c in range(c0, c1):
         lo, hi = c * chunk, min((c + 1) * chunk, wl.N)
         gc = _gen(instance_seed(seed, 1_000_000 + c), device)
-        lab = torch.multinomial(w, hi - lo, replacement=True, generator=gc)
+        u = torch.rand(hi - lo, generator=gc, device=device)
+        lab = torch.searchsorted(cdf, u, right=True).clamp_(max=cdf.numel() - 1)
         pts = mu[lab] + wl.sigma * torch.randn(hi - lo, wl.D, generator=gc, device=device)
         a, b_ = max(lo, start), min(hi, stop)
         piece = pts[a - lo:b_ - lo].to(wl.torch_dtype)

@@ -45,3 +45,40 @@ def test_zipf_weights_concentrate():
     _, lab = make_points(wl, seed=0)
     top = torch.bincount(lab, minlength=1000).max().item()
     assert top > 0.1 * wl.N
+
+
+def test_cdf_is_a_fixed_float64_sum():
+    """Labels come from a CPU float64 cumulative sum of the weights, so the
+    same seed gives the same labels on every run (a device cumulative sum may
+    associate its additions differently from run to run)."""
+    wl = WORKLOADS["4m_k16384_zipf"].with_(N=50_000)
+    _, lab1 = make_points(wl, seed=4)
+    _, lab2 = make_points(wl, seed=4)
+    assert torch.equal(lab1, lab2)
+    assert int(lab1.max()) < wl.K and int(lab1.min()) >= 0
+
+
+GEN_CHILD = r"""
+import hashlib, sys, torch
+from synth import WORKLOADS, make_problem
+X, C0, L = make_problem(WORKLOADS[sys.argv[1]], seed=0, device="cuda")
+h = hashlib.sha256()
+for t in (X, C0, L):
+    h.update(t.cpu().contiguous().view(torch.uint8).numpy().tobytes())
+print(h.hexdigest())
+"""
+
+
+import pytest  # noqa: E402
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["4m_k16384_zipf", "1m_k1024"])
+def test_device_generation_is_the_same_in_every_process(name):
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hashes = {subprocess.run([sys.executable, "-c", GEN_CHILD, name], cwd=root, capture_output=True, text=True,
+                             check=True, env=dict(os.environ, PYTHONPATH=root)).stdout.strip() for _ in range(3)}
+    assert len(hashes) == 1, hashes
