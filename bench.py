@@ -182,15 +182,19 @@ class ClockSampler:
                 "period_ms": self.period, "power_w_median": statistics.median(pw) if pw else None}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend: str = "nccl", same_device: bool = False):
+    """One process per GPU (rank r on cuda:LOCAL_RANK) over NCCL.  For a
+    single-GPU smoke run of the multi-rank path, `same_device` puts every
+    rank on cuda:0 and `backend` "gloo" exchanges through host copies (the
+    ranks' kernels never wait on one another)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    local = 0 if same_device else int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -203,6 +207,8 @@ def max_over_ranks(world, v: float, device="cuda") -> float:
     """The slowest rank's value: every rank contributes, every rank gets it."""
     if world == 1:
         return v
+    if torch.distributed.get_backend() == "gloo":
+        device = "cpu"
     t = torch.tensor([v], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
@@ -691,6 +697,10 @@ def main():
     ap.add_argument("--parallelism", default="dp", choices=["dp", "replicas"],
                     help="with several ranks: shard one problem by rows (dp) or run independent replicas")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--dist-backend", default="nccl", choices=["nccl", "gloo"],
+                    help="gloo only for a single-GPU smoke run of the multi-rank path (with --same-device)")
+    ap.add_argument("--same-device", action="store_true",
+                    help="every rank on cuda:0 (smoke run of the multi-rank path on one GPU)")
     ap.add_argument("--min-timed-s", type=float, default=1.0,
                     help="repeat the K-step fit until the timed region lasts this long")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="host work of the CPU-baseline sample")
@@ -719,7 +729,7 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         res = run_reference(args, world, rank)
     else:
-        world, rank, local = dist_setup(args.gpus)
+        world, rank, local = dist_setup(args.gpus, args.dist_backend, args.same_device)
         res = run_ours(args, world, rank, local)
         if world > 1:
             torch.distributed.destroy_process_group()
