@@ -15,14 +15,18 @@
 //     ||x||^2 + ||c||^2 - 2 x.c        (centroid operand holds -2c)
 // and the epilogue is a pure argmin.  Per score it forms a key -- the float
 // bits with the 5 low mantissa bits replaced by the column inside its
-// 32-column chunk -- and reduces keys with 3-input float minimum.  A score
-// below zero (a point on a centroid, where the expanded form rounds to a few
-// ulps either side of 0) is clamped to +0 first: among negative floats a
-// larger column would make a more negative key and win the tie.  So equal
-// distances resolve to the lowest column, and a chunk's winner is merged
-// into the running best only on a strictly smaller distance: the lowest
-// index wins exact ties.  (Distances closer than 2^-18 relative also compare
-// equal; that is far inside the parity rule's near-tie band.)
+// 32-column chunk -- and reduces keys with 3-input float minimum; a chunk's
+// winner is merged into the running best only on a strictly smaller
+// distance, so equal positive distances go to the lowest index.  A score at
+// or below zero is a zero distance up to rounding (a point on a centroid,
+// where the expanded form lands a few ulps either side of 0), and among
+// negative floats a larger column makes a more negative key.  So when a
+// tile leaves a point's best at or below zero, the warp reads that tile
+// again with every score raised to +0, takes the lowest such column, and
+// pins the best to -inf: no later centroid can then displace it, and the
+// reported distance is 0.  The lowest index wins exact ties.  (Distances
+// closer than 2^-18 relative also compare equal; that is far inside the
+// parity rule's near-tie band.)
 //
 // Structure: persistent CTAs (one per SM), warp-specialised:
 //   warp 0       TMA producer: point tile + its augmentation (resident for the
@@ -63,6 +67,8 @@ struct AssignK {
   int hist_T, hist_R;
   int32_t* rk;      // may be null (with hist0): per point, the cluster id | rank << 20 | (count - 1) << 25
   int32_t* kcnt;    // may be null (with hist0): members per cluster, accumulated
+  int dig_bits;     // log2(hist_R): bits of the sort's first digit
+  int key_bits;     // bits compared per point: dig_bits, or all key bits when kcnt is counted
   unsigned int* status;
   uint64_t limit_ns;
 };
@@ -162,19 +168,18 @@ __device__ __forceinline__ void tmem_ld_wait<16>(uint32_t (&r)[16]) {
                : "memory");
 }
 
-// Minimum key of CW scores: key = max(score, +0) bits with the low 5 bits
-// replaced by the column index i in [0, CW) (mask == ~31 in a register, i an
-// immediate): an integer maximum with 0 (a negative float is a negative
-// signed integer) and one three-input bitwise operation.  Clamping keeps the
-// key order of exact ties: for +0 and positive scores a lower column gives a
-// smaller key.  Reduced with 3-input minima.
-template <int CW>
+// Minimum key of CW scores: key = score bits with the low 5 bits replaced by
+// the column index i in [0, CW) (mask == ~31 in a register, i an
+// immediate), one three-input bitwise operation per score, reduced with
+// 3-input minima.  With CLAMP the score is first raised to +0 (an integer
+// maximum with 0: a negative float is a negative signed integer).
+template <int CW, bool CLAMP>
 __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint32_t mask) {
   float k[CW];
 #pragma unroll
   for (int i = 0; i < CW; ++i) {
-    const uint32_t nonneg = static_cast<uint32_t>(max(static_cast<int32_t>(v[i]), 0));
-    k[i] = __uint_as_float((nonneg & mask) | static_cast<uint32_t>(i));
+    const uint32_t s = CLAMP ? static_cast<uint32_t>(max(static_cast<int32_t>(v[i]), 0)) : v[i];
+    k[i] = __uint_as_float((s & mask) | static_cast<uint32_t>(i));
   }
   constexpr int L1 = CW / 3 + (CW % 3);  // CW=32: 10 triples + 2 singles; CW=16: 5 triples + 1 single
   float a[L1];
@@ -194,6 +199,30 @@ __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint3
   for (; i + 1 < L2; i += 2) m = fmin3(m, b[i], b[i + 1]);
   if (i < L2) m = fminf(m, b[i]);
   return __float_as_uint(m);
+}
+
+// Lowest column of one accumulator tile (`chunks` chunks of CW columns from
+// TMEM column col0 of this thread's lane) among the minimal scores, with
+// every score raised to +0 first (mask == ~31); columns are numbered from
+// base.  Kept out of line: it runs only for tiles that won with a zero
+// distance, and inlined it would hold registers across the common path.
+// All lanes of the warp call it (TMEM loads are warp-wide).
+template <int CW>
+__device__ __noinline__ int lowest_zero_column(uint32_t col0, int chunks, uint32_t mask, int base) {
+  uint32_t v[CW];
+  float tb = CUDART_INF_F;
+  int tk = base;
+  for (int c = 0; c < chunks; ++c) {
+    tmem_ld_issue<CW>(col0 + static_cast<uint32_t>(c * CW), v);
+    tmem_ld_wait<CW>(v);
+    const uint32_t m = chunk_min_key<CW, true>(v, mask);
+    const float mv = __uint_as_float(m & mask);
+    if (mv < tb) {
+      tb = mv;
+      tk = base + c * CW + static_cast<int>(m & ~mask);
+    }
+  }
+  return tk;
 }
 
 // ONE_CT: one centroid tile per point tile (K <= BN), kept resident per
@@ -467,13 +496,28 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           if (c + 1 < kChunks) tmem_ld_issue<CW>(col0 + static_cast<uint32_t>((c + 1) * CW), v[(c + 1) & 1]);
-          const uint32_t m = chunk_min_key<CW>(v[c & 1], kmask);
+          const uint32_t m = chunk_min_key<CW, false>(v[c & 1], kmask);
           const float mv = __uint_as_float(m & ~31u);
           if (mv < best) {
             best = mv;
             bk = j * BN + half * kHalf + c * CW + static_cast<int>(m & 31u);
           }
           if (c + 1 < kChunks) tmem_ld_wait<CW>(v[(c + 1) & 1]);
+        }
+        {
+          // A point whose best this tile just set at or below zero sits on a
+          // centroid: find this tile's lowest column at distance 0 and pin the
+          // best to -inf (reported as 0), so that no later tile displaces it.
+          // Rare (points that coincide with a centroid), hence out of line.
+          const int base = j * BN + half * kHalf;
+          const bool fix = best <= 0.f && bk >= base && bk < base + kHalf;
+          if (__any_sync(0xffffffffu, fix)) {
+            const int tk = lowest_zero_column<CW>(col0, kChunks, kmask, base);
+            if (fix) {
+              bk = tk;
+              best = -CUDART_INF_F;
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -498,8 +542,17 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           // (hist_T is a multiple of 32), so equal digits are added once per
           // warp, by their lowest lane (a hot cluster costs one atomic per
           // warp, not one per point)
-          const int dig = valid ? (bk & (p.hist_R - 1)) : -1;
-          const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+          // lanes of equal digit (and, for the cluster sizes, of equal key):
+          // one ballot per key bit, each lane keeping the lanes that agree
+          // with it (match.any measured several times slower here)
+          uint32_t same = __ballot_sync(0xffffffffu, valid), peers = same;
+          for (int bit = 0; bit < p.key_bits; ++bit) {
+            const bool set = (bk >> bit) & 1;
+            const uint32_t bb = __ballot_sync(0xffffffffu, set);
+            same &= set ? bb : ~bb;
+            if (bit + 1 == p.dig_bits) peers = same;
+          }
+          const int dig = bk & (p.hist_R - 1);
           const int rank_in = __popc(peers & ((1u << lane) - 1u));
           if (valid && rank_in == 0) atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + dig, __popc(peers));
           // The sort's first scatter ranks equal digits inside the same
@@ -508,10 +561,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             p.rk[static_cast<int64_t>(b) * p.rows + row] =
                 bk | (rank_in << 20) | ((__popc(peers) - 1) << 25);
           // members per cluster (two-pass sorts take the cluster starts from these)
-          if (p.kcnt) {
-            const uint32_t same = __match_any_sync(0xffffffffu, valid ? bk : -1);
-            if (valid && lane == __ffs(same) - 1) atomicAdd(p.kcnt + bk, __popc(same));
-          }
+          if (p.kcnt && valid && (same & ((1u << lane) - 1u)) == 0) atomicAdd(p.kcnt + bk, __popc(same));
         }
         double ds = static_cast<double>(md);
 #pragma unroll
@@ -599,6 +649,11 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.hist_R = a.hist_R;
   k.rk = k.hist0 ? a.rk : nullptr;
   k.kcnt = k.hist0 ? a.kcnt : nullptr;
+  k.dig_bits = 0;
+  while ((1 << k.dig_bits) < a.hist_R) ++k.dig_bits;
+  k.key_bits = k.dig_bits;
+  if (k.kcnt)
+    while ((1 << k.key_bits) < a.K) ++k.key_bits;
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN, PAIR>(k.natoms, k.XB, k.CS);

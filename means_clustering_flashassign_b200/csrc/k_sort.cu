@@ -60,11 +60,10 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
   for (int d = threadIdx.x; d < R; d += blockDim.x) out[d] = sh[d];
 }
 
-// In-place exclusive scan of blkhist[0..nblk)[d] over the blocks, and the
-// digit totals.  A block takes 32 digits (one per lane, so every load is
-// coalesced) and splits the block range among its 32 warps: each warp sums
-// its part, the parts are scanned in shared memory, and each warp rewrites
-// its part as running prefixes.
+// In-place exclusive scan of blkhist[0..nblk)[d] over the blocks (within
+// segments of blocks, see k_sort_colscan), and the digit totals of each
+// segment.  Each warp sums its part of the segment, the parts are scanned in
+// shared memory, and each warp rewrites its part as running prefixes.
 constexpr int kColscanWarps = 32;
 
 // start[0..K] of a two-pass sort from the cluster sizes the assignment kernel
@@ -99,10 +98,18 @@ __device__ void starts_from_sizes(int32_t* __restrict__ kcnt, int K, int64_t n, 
   if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
 }
 
-// With kcnt (two-pass sorts whose cluster sizes the assignment kernel
-// counted) the grid has one more block, which writes start[] from them.
+// The block counts are scanned in S segments of consecutive sort blocks, so
+// that few digits still spread over many CTAs: CTA (g, s) takes digits
+// [32 g, 32 g + 32) (one per lane, every load coalesced) and the blocks of
+// segment s, split among its 32 warps; it rewrites them in place as prefixes
+// within the segment and stores the segment's digit totals in segtot[s][d].
+// The scatter adds the totals of the earlier segments (and sums all of them
+// for the digit totals).  With kcnt (two-pass sorts whose cluster sizes the
+// assignment kernel counted) the grid has one more block, which writes
+// start[] from them.
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
-                                                                     int64_t nblk, int32_t* __restrict__ total,
+                                                                     int64_t nblk, int S,
+                                                                     int32_t* __restrict__ segtot,
                                                                      int32_t* __restrict__ kcnt, int K, int64_t n,
                                                                      int32_t* __restrict__ start) {
   __shared__ int32_t part[kColscanWarps][32];
@@ -113,11 +120,16 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
     return;
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int d = blockIdx.x * 32 + lane;
+  const int groups = (R + 31) / 32;
+  const int g = static_cast<int>(blockIdx.x) % groups, sg = static_cast<int>(blockIdx.x) / groups;
+  const int d = g * 32 + lane;
   const bool ok = d < R;
-  const int64_t seg = (nblk + kColscanWarps - 1) / kColscanWarps;
-  const int64_t b0 = warp * seg < nblk ? warp * seg : nblk;
-  const int64_t b1 = b0 + seg < nblk ? b0 + seg : nblk;
+  const int64_t L = (nblk + S - 1) / S;
+  const int64_t r0 = sg * L < nblk ? sg * L : nblk;
+  const int64_t r1 = r0 + L < nblk ? r0 + L : nblk;
+  const int64_t seg = (r1 - r0 + kColscanWarps - 1) / kColscanWarps;
+  const int64_t b0 = r0 + warp * seg < r1 ? r0 + warp * seg : r1;
+  const int64_t b1 = b0 + seg < r1 ? b0 + seg : r1;
   // The first KEEP rows of the warp's part stay in registers for the second
   // pass (all of it up to 512 blocks); rows beyond are read again.
   constexpr int KEEP = 16, CH = 8;
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
 #pragma unroll
   for (int w = 0; w < kColscanWarps; ++w)
     if (w < warp) run += part[w][lane];
-  if (warp == kColscanWarps - 1 && ok) total[d] = run + s;
+  if (warp == kColscanWarps - 1 && ok) segtot[static_cast<int64_t>(sg) * R + d] = run + s;
 #pragma unroll
   for (int u = 0; u < KEEP; ++u) {
     if (ok && b0 + u < b1) blkhist[(b0 + u) * R + d] = run;
@@ -244,8 +256,8 @@ __device__ __forceinline__ void block_scan_pair(int32_t a, int32_t b, int32_t& e
 template <int IPT, int RPT, bool PAIRS, bool PRE>
 __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT < 8 ? 4 : 2)) k_sort_scatter(
     const int32_t* __restrict__ keys_in, const int2* __restrict__ pairs_in, int64_t n, int shift, int R, int bits,
-    int32_t* __restrict__ blkhist, const int32_t* __restrict__ total, int2* __restrict__ pairs_out,
-    int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
+    int32_t* __restrict__ blkhist, const int32_t* __restrict__ segtot, int S, int64_t L,
+    int2* __restrict__ pairs_out, int32_t* __restrict__ perm_out, int32_t* __restrict__ start, int K) {
   constexpr int W = kSortWarps;
   constexpr int T = kSortThreads * IPT;
   extern __shared__ __align__(16) int32_t sh[];
@@ -303,10 +315,21 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
     }
   }
   int32_t* boff = blkhist + static_cast<int64_t>(blockIdx.x) * R;
+  // digit totals (all segments) and this block's offsets (its prefix inside
+  // its segment plus the totals of the earlier segments)
   int32_t tot[RPT] = {}, bo[RPT] = {};
   if (owner) {
-    ld_run<RPT>(total + d0, tot);
     ld_run<RPT>(boff + d0, bo);
+    const int sb = static_cast<int>(static_cast<int64_t>(blockIdx.x) / L);
+    for (int s2 = 0; s2 < S; ++s2) {
+      int32_t v[RPT];
+      ld_run<RPT>(segtot + static_cast<int64_t>(s2) * R + d0, v);
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        tot[j] += v[j];
+        if (s2 < sb) bo[j] += v[j];
+      }
+    }
   }
   // digit bits: R = 256 RPT exactly when RPT > 1; at most 8 when RPT == 1
   constexpr int NB = RPT == 1 ? 8 : RPT == 2 ? 9 : RPT == 4 ? 10 : RPT == 8 ? 11 : 12;
@@ -444,24 +467,25 @@ static size_t scatter_smem(int R, int T) {
 template <int IPT, int RPT, bool PAIRS, bool PRE>
 static cudaError_t launch_scatter_t(int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys, const int2* pin,
                                     int64_t n, int shift, int R, int bits, int32_t* bh, const int32_t* total,
-                                    int2* out, int32_t* perm, int32_t* st, int K) {
+                                    int S, int64_t L, int2* out, int32_t* perm, int32_t* st, int K) {
   auto kern = k_sort_scatter<IPT, RPT, PAIRS, PRE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
   if (e != cudaSuccess) return e;
   return launch_chained(kern, dim3(static_cast<unsigned>(nblk)), dim3(kSortThreads), sm, s, keys, pin, n, shift, R,
-                        bits, bh, total, out, perm, st, K);
+                        bits, bh, total, S, L, out, perm, st, K);
 }
 
 template <int IPT, bool PAIRS, bool PRE>
 static cudaError_t launch_scatter_r(int rpt, int64_t nblk, size_t sm, cudaStream_t s, const int32_t* keys,
                                     const int2* pin, int64_t n, int shift, int R, int bits, int32_t* bh,
-                                    const int32_t* total, int2* out, int32_t* perm, int32_t* st, int K) {
+                                    const int32_t* total, int S, int64_t L, int2* out, int32_t* perm, int32_t* st,
+                                    int K) {
   switch (rpt) {
-    case 1: return launch_scatter_t<IPT, 1, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 2: return launch_scatter_t<IPT, 2, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 4: return launch_scatter_t<IPT, 4, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 8: return launch_scatter_t<IPT, 8, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
-    case 16: return launch_scatter_t<IPT, 16, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, out, perm, st, K);
+    case 1: return launch_scatter_t<IPT, 1, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, S, L, out, perm, st, K);
+    case 2: return launch_scatter_t<IPT, 2, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, S, L, out, perm, st, K);
+    case 4: return launch_scatter_t<IPT, 4, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, S, L, out, perm, st, K);
+    case 8: return launch_scatter_t<IPT, 8, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, S, L, out, perm, st, K);
+    case 16: return launch_scatter_t<IPT, 16, PAIRS, PRE>(nblk, sm, s, keys, pin, n, shift, R, bits, bh, total, S, L, out, perm, st, K);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -492,8 +516,10 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     // a two-pass sort with counted cluster sizes takes start[] from them in
     // the first column scan (one more block) and needs no bounds kernel
     int32_t* kc = ps == 0 && c.passes > 1 ? a.kcnt : nullptr;
-    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 + (kc ? 1 : 0)), dim3(kColscanWarps * 32), 0, s, bh, R,
-                       nblk, a.total, kc, a.K, a.n, a.start);
+    const int S = c.segs[ps];
+    const int64_t L = (nblk + S - 1) / S;
+    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 * S + (kc ? 1 : 0)), dim3(kColscanWarps * 32), 0, s, bh,
+                       R, nblk, S, a.total, kc, a.K, a.n, a.start);
     if (e != cudaSuccess) return e;
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
@@ -504,19 +530,19 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     const int rpt = scatter_rpt(R);
     if (pairs_in)
       e = c.IPT == 16 ? launch_scatter_r<16, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
-                                                          bits, bh, a.total, out, perm, st, a.K)
+                                                          bits, bh, a.total, S, L, out, perm, st, a.K)
                       : launch_scatter_r<8, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
-                                                         bits, bh, a.total, out, perm, st, a.K);
+                                                         bits, bh, a.total, S, L, out, perm, st, a.K);
     else if (a.rk)
       e = c.IPT == 16 ? launch_scatter_r<16, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
-                                                          bh, a.total, out, perm, st, a.K)
+                                                          bh, a.total, S, L, out, perm, st, a.K)
                       : launch_scatter_r<8, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
-                                                         bh, a.total, out, perm, st, a.K);
+                                                         bh, a.total, S, L, out, perm, st, a.K);
     else
       e = c.IPT == 16 ? launch_scatter_r<16, false, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R,
-                                                           bits, bh, a.total, out, perm, st, a.K)
+                                                           bits, bh, a.total, S, L, out, perm, st, a.K)
                       : launch_scatter_r<8, false, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R,
-                                                          bits, bh, a.total, out, perm, st, a.K);
+                                                          bits, bh, a.total, S, L, out, perm, st, a.K);
     if (e != cudaSuccess) return e;
   }
   if (c.passes > 1 && !a.kcnt) {

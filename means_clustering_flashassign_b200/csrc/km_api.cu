@@ -324,6 +324,17 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   sc.T = sc.W * 32 * sc.IPT;
   sc.nblk = (p.rows + sc.T - 1) / sc.T;
   sc.Rmax = 1 << (sc.bits[0] > sc.bits[1] ? sc.bits[0] : sc.bits[1]);
+  // Column-scan segments: about 96 CTAs (32 digits each) when there are few
+  // digits and many blocks, at most 16 segments of at least 32 blocks.
+  for (int ps = 0; ps < sc.passes; ++ps) {
+    const int groups = ((1 << sc.bits[ps]) + 31) / 32;
+    int S = (96 + groups - 1) / groups;
+    const int64_t byrows = sc.nblk / 32;
+    if (S > byrows) S = static_cast<int>(byrows);
+    if (S > 16) S = 16;
+    sc.segs[ps] = S < 1 ? 1 : S;
+  }
+  const int segmax = sc.segs[0] > sc.segs[1] ? sc.segs[0] : sc.segs[1];
   SegCfg& gc = p.gc;
   gc.BNS = static_cast<int>(seg_block_positions(p.rows));
   gc.nchunks = (p.rows + gc.BNS - 1) / gc.BNS;
@@ -340,7 +351,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   if (op == KM_OP_ARGSORT) {
     p.off_blkhist = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[0]) * sc.nblk);
     if (sc.passes > 1) p.off_blkhist1 = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[1]) * sc.nblk);
-    p.off_total = take(sizeof(int32_t) * sc.Rmax);
+    p.off_total = take(sizeof(int32_t) * sc.Rmax * segmax);
     if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
     p.off_pairs = take(sizeof(int2) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));
@@ -359,7 +370,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   if (op != KM_OP_ASSIGN && !p.small_update) {
     p.off_blkhist = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[0]) * sc.nblk);
     if (sc.passes > 1) p.off_blkhist1 = take(sizeof(int32_t) * (static_cast<size_t>(1) << sc.bits[1]) * sc.nblk);
-    p.off_total = take(sizeof(int32_t) * sc.Rmax);
+    p.off_total = take(sizeof(int32_t) * sc.Rmax * segmax);
     if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
     p.off_pairs = take(sizeof(int2) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));

@@ -61,6 +61,7 @@ struct SortCfg {
   int T = 0;         // keys per block
   int64_t nblk = 0;  // blocks per pass
   int Rmax = 0;      // largest radix
+  int segs[2] = {1, 1};  // segments of blocks each pass's column scan splits the blocks into
 };
 
 struct SegCfg {
@@ -203,7 +204,7 @@ struct SortArgs {
                         // assignment kernel); the first scatter then needs no digit ballots
   int32_t* kcnt;        // may be null: cluster sizes counted by the assignment kernel; a two-pass
                         // sort then takes start[] from them (and zeroes them) instead of k_bounds
-  int32_t* total;       // [Rmax]
+  int32_t* total;       // [segs][Rmax]: digit totals of each column-scan segment
   int2* pairs_tmp;      // [n] (two-pass sorts only)
   int2* pairs;          // [n] sorted (point index, cluster id)
   int32_t* perm;        // [n] sorted point indices, or null
