@@ -17,16 +17,17 @@
 // bits with the 5 low mantissa bits replaced by the column inside its
 // 32-column chunk -- and reduces keys with 3-input float minimum; a chunk's
 // winner is merged into the running best only on a strictly smaller
-// distance, so equal positive distances go to the lowest index.  A score at
-// or below zero is a zero distance up to rounding (a point on a centroid,
-// where the expanded form lands a few ulps either side of 0), and among
-// negative floats a larger column makes a more negative key.  So when a
-// tile leaves a point's best at or below zero, the warp reads that tile
-// again with every score raised to +0, takes the lowest such column, and
-// pins the best to -inf: no later centroid can then displace it, and the
-// reported distance is 0.  The lowest index wins exact ties.  (Distances
-// closer than 2^-18 relative also compare equal; that is far inside the
-// parity rule's near-tie band.)
+// distance, and the column quarters of a tile merge lowest index first on
+// equal distances, so equal scores go to the lowest index -- except inside
+// one chunk when they are negative, where a larger column makes a more
+// negative key.  Equal negative scores mean a zero distance (a point on a
+// centroid; the expanded form lands a few ulps either side of 0) to two or
+// more identical centroid rows, which the tensor cores score bit for bit
+// alike.  So a point whose best ends at or below zero takes the lowest
+// centroid of its winning chunk whose operand row equals the winner's (a
+// rare, out-of-line scan of at most 31 rows).  The lowest index wins exact
+// ties.  (Distances closer than 2^-18 relative also compare equal; that is
+// far inside the parity rule's near-tie band.)
 //
 // Structure: persistent CTAs (one per SM), warp-specialised:
 //   warp 0       TMA producer: point tile + its augmentation (resident for the
@@ -63,12 +64,8 @@ struct AssignK {
   float* mindist;
   double* tobj;     // [B * tiles128_per_inst][4]: per 128-point tile, one sum per 32-row quarter
   uint32_t zero;    // always 0; keeps the epilogue's column constants in registers
-  int32_t* hist0;   // may be null: sort pass-0 block digit counts, [row / hist_T][digit]
-  int hist_T, hist_R;
-  int32_t* rk;      // may be null (with hist0): per point, the cluster id | rank << 20 | (count - 1) << 25
-  int32_t* kcnt;    // may be null (with hist0): members per cluster, accumulated
-  int dig_bits;     // log2(hist_R): bits of the sort's first digit
-  int key_bits;     // bits compared per point: dig_bits, or all key bits when kcnt is counted
+  const uint8_t* cop;  // centroid operand rows (-2c), K per instance, cop_rb bytes each
+  int64_t cop_rb;
   unsigned int* status;
   uint64_t limit_ns;
 };
@@ -201,28 +198,22 @@ __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint3
   return __float_as_uint(m);
 }
 
-// Lowest column of one accumulator tile (`chunks` chunks of CW columns from
-// TMEM column col0 of this thread's lane) among the minimal scores, with
-// every score raised to +0 first (mask == ~31); columns are numbered from
-// base.  Kept out of line: it runs only for tiles that won with a zero
-// distance, and inlined it would hold registers across the common path.
-// All lanes of the warp call it (TMEM loads are warp-wide).
-template <int CW>
-__device__ __noinline__ int lowest_zero_column(uint32_t col0, int chunks, uint32_t mask, int base) {
-  uint32_t v[CW];
-  float tb = CUDART_INF_F;
-  int tk = base;
-  for (int c = 0; c < chunks; ++c) {
-    tmem_ld_issue<CW>(col0 + static_cast<uint32_t>(c * CW), v);
-    tmem_ld_wait<CW>(v);
-    const uint32_t m = chunk_min_key<CW, true>(v, mask);
-    const float mv = __uint_as_float(m & mask);
-    if (mv < tb) {
-      tb = mv;
-      tk = base + c * CW + static_cast<int>(m & ~mask);
+// Lowest centroid index in k's 32-column chunk whose operand row (rb
+// bytes, a multiple of 16) equals row k's; rows holds the instance's rows.
+// Kept out of line: it runs only for points at distance 0.
+__device__ __forceinline__ int lowest_copy(const uint8_t* rows, int64_t rb, int k) {
+  const uint4* rk = reinterpret_cast<const uint4*>(rows + k * rb);
+  const int n16 = static_cast<int>(rb / 16);
+  for (int c = k & ~31; c < k; ++c) {
+    const uint4* rc = reinterpret_cast<const uint4*>(rows + c * rb);
+    int i = 0;
+    for (; i < n16; ++i) {
+      const uint4 u = rc[i], w = rk[i];
+      if (u.x != w.x || u.y != w.y || u.z != w.z || u.w != w.w) break;
     }
+    if (i == n16) return c;
   }
-  return tk;
+  return k;
 }
 
 // ONE_CT: one centroid tile per point tile (K <= BN), kept resident per
@@ -504,21 +495,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           }
           if (c + 1 < kChunks) tmem_ld_wait<CW>(v[(c + 1) & 1]);
         }
-        {
-          // A point whose best this tile just set at or below zero sits on a
-          // centroid: find this tile's lowest column at distance 0 and pin the
-          // best to -inf (reported as 0), so that no later tile displaces it.
-          // Rare (points that coincide with a centroid), hence out of line.
-          const int base = j * BN + half * kHalf;
-          const bool fix = best <= 0.f && bk >= base && bk < base + kHalf;
-          if (__any_sync(0xffffffffu, fix)) {
-            const int tk = lowest_zero_column<CW>(col0, kChunks, kmask, base);
-            if (fix) {
-              bk = tk;
-              best = -CUDART_INF_F;
-            }
-          }
-        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -534,34 +510,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (valid) {
           const int64_t o = static_cast<int64_t>(b) * p.rows + row;
           md = fmaxf(0.f, best);
+          if (best <= 0.f && p.cop) bk = lowest_copy(p.cop + static_cast<int64_t>(b) * p.K * p.cop_rb, p.cop_rb, bk);
           p.idx[o] = bk;
           if (p.mindist) p.mindist[o] = md;
-        }
-        if (p.hist0) {
-          // sort pass-0 digit counts: the warp's 32 rows share one sort block
-          // (hist_T is a multiple of 32), so equal digits are added once per
-          // warp, by their lowest lane (a hot cluster costs one atomic per
-          // warp, not one per point)
-          // lanes of equal digit (and, for the cluster sizes, of equal key):
-          // one ballot per key bit, each lane keeping the lanes that agree
-          // with it (match.any measured several times slower here)
-          uint32_t same = __ballot_sync(0xffffffffu, valid), peers = same;
-          for (int bit = 0; bit < p.key_bits; ++bit) {
-            const bool set = (bk >> bit) & 1;
-            const uint32_t bb = __ballot_sync(0xffffffffu, set);
-            same &= set ? bb : ~bb;
-            if (bit + 1 == p.dig_bits) peers = same;
-          }
-          const int dig = bk & (p.hist_R - 1);
-          const int rank_in = __popc(peers & ((1u << lane) - 1u));
-          if (valid && rank_in == 0) atomicAdd(p.hist0 + (row / p.hist_T) * p.hist_R + dig, __popc(peers));
-          // The sort's first scatter ranks equal digits inside the same
-          // 32-point groups: hand it this group's rank and size with the key
-          if (p.rk && valid)
-            p.rk[static_cast<int64_t>(b) * p.rows + row] =
-                bk | (rank_in << 20) | ((__popc(peers) - 1) << 25);
-          // members per cluster (two-pass sorts take the cluster starts from these)
-          if (p.kcnt && valid && (same & ((1u << lane) - 1u)) == 0) atomicAdd(p.kcnt + bk, __popc(same));
         }
         double ds = static_cast<double>(md);
 #pragma unroll
@@ -644,16 +595,8 @@ static cudaError_t launch_t(const Plan& pl, const AssignArgs& a, cudaStream_t s)
   k.mindist = a.mindist;
   k.tobj = a.tobj;
   k.zero = 0;
-  k.hist0 = a.B == 1 ? a.hist0 : nullptr;
-  k.hist_T = a.hist_T;
-  k.hist_R = a.hist_R;
-  k.rk = k.hist0 ? a.rk : nullptr;
-  k.kcnt = k.hist0 ? a.kcnt : nullptr;
-  k.dig_bits = 0;
-  while ((1 << k.dig_bits) < a.hist_R) ++k.dig_bits;
-  k.key_bits = k.dig_bits;
-  if (k.kcnt)
-    while ((1 << k.key_bits) < a.K) ++k.key_bits;
+  k.cop = static_cast<const uint8_t*>(a.cop);
+  k.cop_rb = static_cast<int64_t>(a.cop_row_bytes);
   k.status = a.status;
   k.limit_ns = a.limit_ns;
   const size_t smem = assign_smem_bytes<BN, PAIR>(k.natoms, k.XB, k.CS);

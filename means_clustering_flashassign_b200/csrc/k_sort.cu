@@ -5,21 +5,24 @@
 //
 // A stable least-significant-digit radix sort of (key = cluster id, value =
 // point index), one or two passes of at most 12 bits.  Per pass:
-//   hist     block b counts the digits of its T keys -> blkhist[b][digit]
-//            (on the first pass of a fit, the assignment kernel counts them)
+//   count    block b counts the digits of its T keys -> blkhist[b][digit],
+//            per 32-key group with ballots (one shared-memory add per
+//            distinct digit of a group, so a hot digit does not serialise);
+//            on the first pass of a fit it also stores each key with its
+//            rank and count among the equal digits of its group (for the
+//            scatter) and, for two-pass sorts, adds up the cluster sizes
 //   colscan  one lane per digit: exclusive scan over the blocks of each
 //            digit's counts, plus the digit totals (digit-major order of the
 //            runs makes the concatenation the stable counting-sort offsets)
 //   scatter  each block ranks its keys stably with per-warp counters
-//            (equal digits inside a warp step grouped by ballots -- or, on
-//            the first pass of a fit, by the assignment kernel, which hands
-//            each key over with its rank and count inside its 32-point
-//            group), scans the digit totals and its own digit counts, and
-//            writes every element to its final position.
+//            (equal digits inside a warp step grouped by ballots, or taken
+//            from the ranks the count kernel stored), scans the digit
+//            totals and its own digit counts, and writes every element to
+//            its final position.
 // Cluster starts: a one-pass sort's digit is the cluster id, so the scatter
 // writes start[]; a two-pass sort inside a fit takes them from the cluster
-// sizes the assignment kernel counted (one more column-scan block), else
-// from the sorted keys (k_bounds).
+// sizes the count kernel added up (one more column-scan block), else from
+// the sorted keys (k_bounds).
 // The sort is deterministic: equal keys keep point order, so the permutation
 // is unique and the later float sums always run in the same order.
 #include <cstdint>
@@ -37,27 +40,76 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 
 __device__ __forceinline__ int32_t clamp_key(int32_t k, int K) { return k < 0 ? 0 : (k >= K ? K - 1 : k); }
 
-// Digit counts of each block's T keys, block-major: blkhist[b][d].
-// Pass 0 reads the assignment vector, later passes the (point, key) pairs.
-template <bool PAIRS>
-__global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ keys, const int2* __restrict__ pairs,
-                                                   int64_t n, int T, int shift, int R, int32_t* __restrict__ blkhist,
-                                                   int K) {
+constexpr int kSortThreads = 256;
+constexpr int kSortWarps = kSortThreads / 32;
+
+// Digit counts of each block's T keys, block-major blkhist[b][d].  The
+// block's 32 warps take STEPS = T / 1024 steps of 32 consecutive keys each
+// (all loads issued first).  The lanes of a step with equal digits are found
+// with one ballot per bit of kv (the digit, or with rk / kcnt the whole key,
+// whose low bits are the pass-0 digit): each lane keeps the lanes whose bit
+// agrees with its own, the digit's bits first; the lowest of the lanes with
+// its digit adds their number to the block's count.  With rk (pass 0): rk[i] = key | rank << 20 |
+// (count - 1) << 25, the key's rank among the equal digits of its aligned
+// 32-key group and their number, as the scatter ranks them.  With kcnt: the
+// lowest lane of each distinct key adds the key's count in the group.
+constexpr int kCountThreads = 1024;
+template <int STEPS, bool PAIRS>
+__global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __restrict__ keys,
+                                                              const int2* __restrict__ pairs, int64_t n, int shift,
+                                                              int R, int dig_bits, int key_bits,
+                                                              int32_t* __restrict__ blkhist,
+                                                              int32_t* __restrict__ rk, int32_t* __restrict__ kcnt,
+                                                              int K) {
+  constexpr int T = kCountThreads * STEPS;
   extern __shared__ int32_t sh[];
   pdl_trigger();
-  for (int d = threadIdx.x; d < R; d += blockDim.x) sh[d] = 0;
+  for (int d = threadIdx.x; d < R; d += kCountThreads) sh[d] = 0;
   pdl_wait();
   __syncthreads();
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * T;
-  for (int j = threadIdx.x; j < T; j += blockDim.x) {
-    const int64_t i = t0 + j;
-    if (i >= n) break;
-    const int key = PAIRS ? pairs[i].y : clamp_key(keys[i], K);
-    atomicAdd(&sh[(key >> shift) & (R - 1)], 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * T + static_cast<int64_t>(warp) * (32 * STEPS);
+  int32_t key[STEPS];
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int64_t i = w0 + 32 * s + lane;
+    key[s] = i < n ? (PAIRS ? pairs[i].y : clamp_key(keys[i], K)) : 0;
+  }
+  const bool whole = !PAIRS && (rk || kcnt);  // pass 0 of a fit: group by the whole key
+  const int nb = whole ? key_bits : dig_bits;
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int64_t i = w0 + 32 * s + lane;
+    const bool valid = i < n;
+    const int dig = (key[s] >> shift) & (R - 1);
+    const uint32_t kv = whole ? static_cast<uint32_t>(key[s]) : static_cast<uint32_t>(dig);
+    const uint32_t kz = valid ? kv : 0u;
+    uint32_t same = __ballot_sync(0xffffffffu, valid);
+    auto narrow = [&](int bit) {
+      const uint32_t b = (kz >> bit) & 1u;
+      const uint32_t bb = __ballot_sync(0xffffffffu, b != 0u);
+      same &= ~(bb ^ (0u - b));
+    };
+    int bit = 0;
+    for (; bit + 4 <= dig_bits; bit += 4) {
+      narrow(bit);
+      narrow(bit + 1);
+      narrow(bit + 2);
+      narrow(bit + 3);
+    }
+    for (; bit < dig_bits; ++bit) narrow(bit);
+    const uint32_t peers = same;
+    for (; bit < nb; ++bit) narrow(bit);
+    if (!valid) continue;
+    const int rank = __popc(peers & lt), cnt = __popc(peers);
+    if (rank == 0) atomicAdd(&sh[dig], cnt);
+    if (!PAIRS && rk) rk[i] = key[s] | (rank << 20) | ((cnt - 1) << 25);
+    if (!PAIRS && kcnt && (same & lt) == 0) atomicAdd(kcnt + key[s], __popc(same));
   }
   __syncthreads();
   int32_t* out = blkhist + static_cast<int64_t>(blockIdx.x) * R;
-  for (int d = threadIdx.x; d < R; d += blockDim.x) out[d] = sh[d];
+  for (int d = threadIdx.x; d < R; d += kCountThreads) out[d] = sh[d];
 }
 
 // In-place exclusive scan of blkhist[0..nblk)[d] over the blocks (within
@@ -66,8 +118,8 @@ __global__ void __launch_bounds__(256) k_sort_hist(const int32_t* __restrict__ k
 // shared memory, and each warp rewrites its part as running prefixes.
 constexpr int kColscanWarps = 32;
 
-// start[0..K] of a two-pass sort from the cluster sizes the assignment kernel
-// counted: an exclusive scan over the clusters (each thread a contiguous run
+// start[0..K] of a two-pass sort from the cluster sizes the count kernel
+// added up: an exclusive scan over the clusters (each thread a contiguous run
 // of them, then a block scan of the run sums), start[K] = n; the sizes are
 // zeroed for the next accumulation.  One block of kColscanWarps warps.
 __device__ void starts_from_sizes(int32_t* __restrict__ kcnt, int K, int64_t n, int32_t* __restrict__ start,
@@ -105,8 +157,8 @@ __device__ void starts_from_sizes(int32_t* __restrict__ kcnt, int K, int64_t n, 
 // within the segment and stores the segment's digit totals in segtot[s][d].
 // The scatter adds the totals of the earlier segments (and sums all of them
 // for the digit totals).  With kcnt (two-pass sorts whose cluster sizes the
-// assignment kernel counted) the grid has one more block, which writes
-// start[] from them.
+// count kernel added up) the grid has one more block, which writes start[]
+// from them.
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
                                                                      int64_t nblk, int S,
                                                                      int32_t* __restrict__ segtot,
@@ -169,9 +221,6 @@ __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __
     }
   }
 }
-
-constexpr int kSortThreads = 256;
-constexpr int kSortWarps = kSortThreads / 32;
 
 // RPT consecutive ints (RPT = 1, 2 or a multiple of 4; p aligned to them).
 template <int RPT>
@@ -249,8 +298,7 @@ __device__ __forceinline__ void block_scan_pair(int32_t a, int32_t b, int32_t& e
 // digit order in shared memory and writes them out in that order, so the
 // elements of one digit leave as one contiguous run.  Writes one 8-byte
 // (point, key) pair per element, and optionally the bare point index
-// (perm_out) on the last pass; zeroes the block's counts (blkhist row) for
-// the next accumulation.
+// (perm_out) on the last pass.
 // Resident blocks per SM the register budget is sized for: what the shared
 // memory (2T + 9R ints) admits, 1 to 4.
 template <int IPT, int RPT, bool PAIRS, bool PRE>
@@ -275,9 +323,7 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
     for (int w = 0; w < W; ++w) st_run<RPT>(wcnt + w * R + d0, z);
   }
   {
-    // While the previous kernel drains: pull this block's keys into L2 (the
-    // assignment vector is written early in the assignment kernel and partly
-    // evicted by the point stream that follows).
+    // While the previous kernel drains: pull this block's keys into L2.
     const int64_t first = static_cast<int64_t>(blockIdx.x) * T;
     const int64_t line = first + static_cast<int64_t>(tid) * (PAIRS ? 16 : 32);
     if (tid < T / (PAIRS ? 16 : 32) && line < n) {
@@ -297,7 +343,7 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   int32_t key[IPT], val[PAIRS ? IPT : 1];
   // PRE: the key word also holds the point's rank among the equal digits of
   // its 32-point group (bits 20..24) and the group's count of that digit
-  // minus one (bits 25..29), as the assignment kernel found them
+  // minus one (bits 25..29), as the count kernel found them
   uint32_t pre[PRE ? IPT : 1];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {  // all loads first
@@ -407,8 +453,6 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
 #pragma unroll
       for (int j = 0; j < RPT; ++j) run[j] += c[j];
     }
-    const int32_t z[RPT] = {};
-    st_run<RPT>(boff + d0, z);  // leave the counts zeroed for the next accumulation
   }
   if (start && blockIdx.x == 0 && tid == 0) start[K] = static_cast<int32_t>(n);
   __syncthreads();
@@ -418,8 +462,7 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {
     const int32_t pt = PAIRS ? val[PAIRS ? s : 0] : static_cast<int32_t>(w0 + s * 32 + lane);
-    // ranks are below T unless the counts came from an assignment kernel that
-    // gave up on a bounded wait: stay inside the stage then
+    // ranks are below T; the check keeps the stage safe whatever the counts
     if (rank[s] >= 0 && rank[s] < T) stage[rank[s]] = make_int2(pt, key[s]);
   }
   __syncthreads();
@@ -436,8 +479,7 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   for (int s = 0; s < IPT; ++s) {
     const int i = s * kSortThreads + tid;
     const int64_t pos = static_cast<int64_t>(gp[s]) + i;
-    // Counts accumulated elsewhere (the assignment kernel) agree with these
-    // keys unless that kernel gave up on a bounded wait; stay in bounds then.
+    // positions lie in [0, n) when the counts match the keys; checked anyway
     if (i < nvalid && pos >= 0 && pos < n) {
       pairs_out[pos] = pk[s];
       if (perm_out) perm_out[pos] = pk[s].x;
@@ -502,20 +544,28 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     const bool last = ps == c.passes - 1;
     const bool pairs_in = ps > 0;
     int32_t* bh = ps == 0 ? a.blkhist : a.blkhist1;
-    count_launch(ps == 0 && a.hist0_ready ? 2 : 3);  // [hist,] colscan, scatter
+    count_launch(3);  // count, colscan, scatter
     const dim3 hgrid(static_cast<unsigned>(nblk));
-    if (pairs_in)
-      e = launch_chained(k_sort_hist<true>, hgrid, dim3(256), R * 4, s, nullptr, a.pairs_tmp, a.n, c.T, c.shift[ps],
-                         R, bh, a.K);
-    else if (!a.hist0_ready)
-      e = launch_chained(k_sort_hist<false>, hgrid, dim3(256), R * 4, s, a.keys, nullptr, a.n, c.T, c.shift[ps], R,
-                         bh, a.K);
+    int32_t* rk = pairs_in ? nullptr : a.rk;
+    int32_t* kc0 = pairs_in || c.passes == 1 ? nullptr : a.kcnt;
+    int key_bits = bits;
+    if (kc0)
+      while ((1 << key_bits) < a.K) ++key_bits;
+    // T = 4096 or 2048 keys per block: 4 or 2 steps per warp of 1024 threads
+    if (c.IPT == 16)
+      e = pairs_in ? launch_chained(k_sort_count<4, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bits, bh, nullptr, nullptr, a.K)
+                   : launch_chained(k_sort_count<4, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
+                                    a.n, c.shift[ps], R, bits, key_bits, bh, rk, kc0, a.K);
     else
-      e = cudaSuccess;
+      e = pairs_in ? launch_chained(k_sort_count<2, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bits, bh, nullptr, nullptr, a.K)
+                   : launch_chained(k_sort_count<2, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
+                                    a.n, c.shift[ps], R, bits, key_bits, bh, rk, kc0, a.K);
     if (e != cudaSuccess) return e;
     // a two-pass sort with counted cluster sizes takes start[] from them in
     // the first column scan (one more block) and needs no bounds kernel
-    int32_t* kc = ps == 0 && c.passes > 1 ? a.kcnt : nullptr;
+    int32_t* kc = kc0;
     const int S = c.segs[ps];
     const int64_t L = (nblk + S - 1) / S;
     e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 * S + (kc ? 1 : 0)), dim3(kColscanWarps * 32), 0, s, bh,
@@ -533,10 +583,10 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
                                                           bits, bh, a.total, S, L, out, perm, st, a.K)
                       : launch_scatter_r<8, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
                                                          bits, bh, a.total, S, L, out, perm, st, a.K);
-    else if (a.rk)
-      e = c.IPT == 16 ? launch_scatter_r<16, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
+    else if (rk)
+      e = c.IPT == 16 ? launch_scatter_r<16, false, true>(rpt, nblk, sm, s, rk, nullptr, a.n, c.shift[ps], R, bits,
                                                           bh, a.total, S, L, out, perm, st, a.K)
-                      : launch_scatter_r<8, false, true>(rpt, nblk, sm, s, a.rk, nullptr, a.n, c.shift[ps], R, bits,
+                      : launch_scatter_r<8, false, true>(rpt, nblk, sm, s, rk, nullptr, a.n, c.shift[ps], R, bits,
                                                          bh, a.total, S, L, out, perm, st, a.K);
     else
       e = c.IPT == 16 ? launch_scatter_r<16, false, false>(rpt, nblk, sm, s, a.keys, nullptr, a.n, c.shift[ps], R,

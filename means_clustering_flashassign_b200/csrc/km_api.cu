@@ -355,6 +355,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     if (sc.passes > 1) p.off_pairs_tmp = take(sizeof(int2) * p.rows);
     p.off_pairs = take(sizeof(int2) * p.rows);
     p.off_start = take(sizeof(int32_t) * (K + 1));
+    p.off_rk = take(sizeof(int32_t) * static_cast<size_t>(p.rows));
     p.total = off;
     return KM_OK;
   }
@@ -378,7 +379,7 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
     p.off_pl = take(sizeof(float) * gc.nchunks * D);
     p.off_pr = take(sizeof(float) * gc.nchunks * D);
   }
-  if ((op == KM_OP_FIT || op == KM_OP_FIT_HOST) && B == 1 && !p.small_update) {
+  if ((op == KM_OP_FIT || op == KM_OP_FIT_HOST) && !p.small_update) {
     p.off_rk = take(sizeof(int32_t) * static_cast<size_t>(p.rows));
     if (sc.passes > 1) p.off_kcnt = take(sizeof(int32_t) * static_cast<size_t>(K));
   }
@@ -431,15 +432,14 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
-                    bool hist0_ready = false, double* acc_ext = nullptr, double* cnt_ext = nullptr,
-                    const int32_t* rk = nullptr, int32_t* kcnt = nullptr) {
+                    double* acc_ext = nullptr, double* cnt_ext = nullptr, int32_t* rk = nullptr,
+                    int32_t* kcnt = nullptr) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
               p.K,
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
-              hist0_ready,
               rk,
               kcnt,
               at<int32_t>(c.ws, p.off_total),
@@ -555,6 +555,8 @@ int km_assign(const void* X, const void* C, int B, int64_t N, int D, int K, int 
   int64_t groups = 0;
   AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, mindist, tobj, c.status(), wait_limit_ns(),
                &groups};
+  a.cop = clp;
+  a.cop_row_bytes = op_row_bytes(p);
   KM_CUDA(launch_assign(p, a, c.s));
   if (objective) KM_CUDA(launch_objective(tobj, B, groups, objective, 1, c.s));
   return KM_OK;
@@ -614,23 +616,16 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   KM_CUDA(launch_cprep(C0, dtype, B, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
-  // Single-instance fits let the assignment kernel count the sort's first
-  // digit per block; the sort's scatter zeroes the counts again after use.
-  const bool fused_hist = B == 1 && !p.small_update;
-  int32_t* hist0 = fused_hist ? at<int32_t>(c.ws, p.off_blkhist) : nullptr;
-  // with the counts, the assignment kernel hands the sort each point's key
-  // with its rank inside its 32-point group, and (two passes) the cluster sizes
-  int32_t* rk = fused_hist ? at<int32_t>(c.ws, p.off_rk) : nullptr;
-  int32_t* kcnt = fused_hist && p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
-  if (fused_hist)
-    KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
-  chain_break();
+  // The sort's count kernel hands its scatter each point's key with its
+  // rank inside its 32-point group, and (two passes) counts the cluster sizes
+  int32_t* rk = p.small_update ? nullptr : at<int32_t>(c.ws, p.off_rk);
+  int32_t* kcnt = !p.small_update && p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
   if (kcnt) KM_CUDA(cudaMemsetAsync(kcnt, 0, sizeof(int32_t) * static_cast<size_t>(K), c.s));
   chain_break();
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
-                 &groups, hist0, p.sc.T, 1 << p.sc.bits[0], rk, kcnt};
+                 &groups, clp, op_row_bytes(p)};
     if (ev && (per_phase || t == 0)) {
       KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t : 0], c.s));
       chain_break();
@@ -651,8 +646,8 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
                             C_out + static_cast<int64_t>(b) * K * D, static_cast<uint8_t*>(clp) + b * opstride,
                             caug + static_cast<int64_t>(b) * p.Kp * 32,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
-                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, fused_hist, nullptr,
-                            nullptr, rk, kcnt);
+                            tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, nullptr, nullptr,
+                            rk, kcnt);
         if (r != KM_OK) return r;
       }
     }
@@ -802,9 +797,6 @@ int fit_stream(const ChunkFn& chunk, bool slot_reuse, const void* C0, int64_t N,
     KM_CUDA(cudaMemsetAsync(objacc, 0, sizeof(double), c.s));
     chain_break();
     KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
-    int32_t* hist0 = at<int32_t>(c.ws, p.off_blkhist);
-    KM_CUDA(cudaMemsetAsync(hist0, 0, sizeof(int32_t) * (static_cast<size_t>(1) << p.sc.bits[0]) * p.sc.nblk, c.s));
-    chain_break();
     int32_t* rk = at<int32_t>(c.ws, p.off_rk);
     int32_t* kcnt = p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
     if (kcnt) {
@@ -855,14 +847,14 @@ int fit_stream(const ChunkFn& chunk, bool slot_reuse, const void* C0, int64_t N,
         pc.tiles_per_inst = (nr + kTileM - 1) / kTileM;
         pc.ntiles = pc.tiles_per_inst;
         int64_t groups = 0;
-        AssignArgs a{&xmap, &xamap, &cmap, &camap, 1,       nr,      K,           p.Kp,
-                     idxc,  nullptr, tobj,  c.status(), wait_limit_ns(), &groups, hist0, p.sc.T,
-                     1 << p.sc.bits[0], rk, kcnt};
+        AssignArgs a{&xmap, &xamap, &cmap,      &camap,          1,       nr,  K,
+                     p.Kp,  idxc,   nullptr,    tobj,            c.status(), wait_limit_ns(), &groups,
+                     clp,   op_row_bytes(p)};
         KM_CUDA(launch_assign(pc, a, c.s));
         Ctx cc = c;
         cc.p = pc;
         rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1,
-                             true, nullptr, nullptr, rk, kcnt);
+                             nullptr, nullptr, rk, kcnt);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
         chain_break();
@@ -942,8 +934,7 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               K,
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
-              false,
-              nullptr,
+              at<int32_t>(c.ws, p.off_rk),
               nullptr,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
@@ -968,8 +959,7 @@ int km_update_accumulate(const void* X, const int32_t* idx, int64_t N, int D, in
     KM_CUDA(cudaMemsetAsync(counts, 0, sizeof(double) * K, c.s));
     chain_break();
   }
-  return update_instance(c, X, idx, N, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 1, false, sums,
-                         counts);
+  return update_instance(c, X, idx, N, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 1, sums, counts);
 }
 
 int km_finalize_sums(const double* sums, const double* counts, int K, int D, int dtype, float* C, void* C_lp,

@@ -179,10 +179,8 @@ struct AssignArgs {
   unsigned int* status;
   uint64_t limit_ns;
   int64_t* obj_groups;  // host out (may be null): 4-double groups of partials per instance
-  int32_t* hist0;       // may be null: pass-0 block digit counts to accumulate (B == 1 only)
-  int hist_T, hist_R;   // keys per sort block, pass-0 radix
-  int32_t* rk = nullptr;    // with hist0, may be null: packed keys for the sort's first scatter
-  int32_t* kcnt = nullptr;  // with hist0, may be null: cluster sizes to accumulate (zero on entry)
+  const void* cop = nullptr;  // the centroid operand rows the maps cover (ties at distance 0)
+  size_t cop_row_bytes = 0;
 };
 cudaError_t launch_assign(const Plan& p, const AssignArgs& a, cudaStream_t s);
 
@@ -197,13 +195,12 @@ struct SortArgs {
   const int32_t* keys;  // the assignment vector
   int64_t n;
   int K;
-  int32_t* blkhist;     // [nblk][R0] pass-0 block digit counts (zeroed again by the pass-0 scatter)
+  int32_t* blkhist;     // [nblk][R0] pass-0 block digit counts
   int32_t* blkhist1;    // [nblk][R1] pass-1 block digit counts (two-pass sorts only)
-  bool hist0_ready;     // pass-0 counts were accumulated by the assignment kernel
-  const int32_t* rk;    // may be null: the keys with their 32-point group rank and size (from the
-                        // assignment kernel); the first scatter then needs no digit ballots
-  int32_t* kcnt;        // may be null: cluster sizes counted by the assignment kernel; a two-pass
-                        // sort then takes start[] from them (and zeroes them) instead of k_bounds
+  int32_t* rk;          // [n] or null: the first pass stores each key with its 32-key group rank
+                        // and count there, and its scatter then needs no digit ballots
+  int32_t* kcnt;        // [K] or null (zero on entry): a two-pass sort adds up the cluster sizes
+                        // and takes start[] from them (zeroing them again) instead of k_bounds
   int32_t* total;       // [segs][Rmax]: digit totals of each column-scan segment
   int2* pairs_tmp;      // [n] (two-pass sorts only)
   int2* pairs;          // [n] sorted (point index, cluster id)

@@ -21,7 +21,7 @@ CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 # Kernels launched through launch_chained (or, for the assignment, with the
 # programmatic attribute set by hand).
-CHAINED = ["k_assign", "k_sort_hist", "k_sort_colscan", "k_sort_scatter", "k_bounds", "k_segsum",
+CHAINED = ["k_assign", "k_sort_count", "k_sort_colscan", "k_sort_scatter", "k_bounds", "k_segsum",
            "k_finalize", "k_small_update"]
 
 

@@ -11,6 +11,8 @@ of the ragged last tile) and across a chunk edge; the points lying exactly on
 them must be assigned to k, bit for bit equal to the oracle, under every
 centroid tile width and both kernel forms."""
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -36,7 +38,6 @@ def _tilings(dtype, D, K):
             for xb, cs in ((2, 4), (2, 3), (2, 2), (1, 2)):
                 t = f"{pair},{bn},{xb},{cs}"
                 try:
-                    import os
                     os.environ["KM_ASSIGN_TILE"] = t
                     km.plan(km.OP_ASSIGN, 1, 5000, D, K, dtype)
                 except km.KMError:
@@ -48,15 +49,18 @@ def _tilings(dtype, D, K):
     return out
 
 
-def _problem(dtype, D, K, pairs, seed):
-    wl = WORKLOADS["1m_k1024"].with_(N=5000, D=D, K=K, dtype=dtype,
+def _problem(dtype, D, K, pairs, seed, B=1):
+    wl = WORKLOADS["1m_k1024"].with_(N=5000, D=D, K=K, B=B, dtype=dtype,
                                      centers="normal2" if dtype == "bf16" else "uniform10")
     X, C, _ = make_problem(wl, seed=seed, device="cpu")
     C = C.clone()
     X = X.clone()
+    if B > 1:
+        return X, C, None
     on = []
-    for j, (k, k1) in enumerate(pairs):
-        C[k1] = C[k]
+    for j, (k, *copies) in enumerate(pairs):
+        for k1 in copies:
+            C[k1] = C[k]
         # eight points exactly on the pair, spread over point tiles
         rows = [j * 8 + r * 613 for r in range(8)]
         X[rows] = C[k]
@@ -83,5 +87,38 @@ def test_exact_ties_in_one_chunk_go_to_the_lowest_index(dtype, D, K, pairs, monk
         assert np.array_equal(got[rows], want), (t, got[rows][got[rows] != want], want[got[rows] != want])
         assert float(md.cpu()[rows].max()) >= 0.0
         # the duplicates (k+1) never win anywhere
-        assert not np.isin(got, [k1 for _, k1 in pairs]).any(), t
+        assert not np.isin(got, [k1 for _, *c in pairs for k1 in c]).any(), t
         check_assignment(X, C, idx, md, dtype)
+
+
+def test_three_copies_in_one_chunk_and_batched_instances():
+    """Three copies of a centroid in one chunk (the lowest is not the
+    chunk's first column), and duplicate pairs in each instance of a batch,
+    at other columns per instance: every point on a copy takes the lowest
+    copy of its own instance."""
+    groups = [(200, 204, 217), (40, 63), (3, 31)]
+    X, C, on = _problem("bf16", 128, 600, groups, seed=7)
+    rows = np.array([r for r, _ in on])
+    want = np.array([k for _, k in on])
+    for t in _tilings(km.BF16, 128, 600):
+        os.environ["KM_ASSIGN_TILE"] = t
+        try:
+            idx, _, _ = km.assign(X.cuda(), C.cuda())
+        finally:
+            os.environ.pop("KM_ASSIGN_TILE", None)
+        assert np.array_equal(idx.cpu().numpy()[rows], want), t
+    B, K = 3, 300
+    Xb, Cb, _ = _problem("bf16", 64, K, [], seed=9, B=B)
+    want_b = []
+    for b in range(B):
+        k = 10 + 37 * b
+        Cb[b, k + 5] = Cb[b, k]
+        Cb[b, k + 9] = Cb[b, k]
+        Xb[b, 100 + b] = Cb[b, k]
+        Xb[b, 2000 + b] = Cb[b, k]
+        want_b.append(k)
+    idx, _, _ = km.assign(Xb.cuda().contiguous(), Cb.cuda().contiguous())
+    got = idx.cpu().numpy()
+    for b in range(B):
+        assert got[b, 100 + b] == want_b[b] and got[b, 2000 + b] == want_b[b], (b, got[b, 100 + b], got[b, 2000 + b])
+        check_assignment(Xb[b], Cb[b], idx[b], None, "bf16")
