@@ -8,9 +8,8 @@
 //   count    block b counts the digits of its T keys -> blkhist[b][digit],
 //            per 32-key group with ballots (one shared-memory add per
 //            distinct digit of a group, so a hot digit does not serialise);
-//            on the first pass of a fit it also stores each key with its
-//            rank and count among the equal digits of its group (for the
-//            scatter) and, for two-pass sorts, adds up the cluster sizes
+//            on the first pass it also stores each key with its rank and
+//            count among the equal digits of its group, for the scatter
 //   colscan  one lane per digit: exclusive scan over the blocks of each
 //            digit's counts, plus the digit totals (digit-major order of the
 //            runs makes the concatenation the stable counting-sort offsets)
@@ -20,9 +19,7 @@
 //            totals and its own digit counts, and writes every element to
 //            its final position.
 // Cluster starts: a one-pass sort's digit is the cluster id, so the scatter
-// writes start[]; a two-pass sort inside a fit takes them from the cluster
-// sizes the count kernel added up (one more column-scan block), else from
-// the sorted keys (k_bounds).
+// writes start[]; a two-pass sort finds them in the sorted keys (k_bounds).
 // The sort is deterministic: equal keys keep point order, so the permutation
 // is unique and the later float sums always run in the same order.
 #include <cstdint>
@@ -46,21 +43,17 @@ constexpr int kSortWarps = kSortThreads / 32;
 // Digit counts of each block's T keys, block-major blkhist[b][d].  The
 // block's 32 warps take STEPS = T / 1024 steps of 32 consecutive keys each
 // (all loads issued first).  The lanes of a step with equal digits are found
-// with one ballot per bit of kv (the digit, or with rk / kcnt the whole key,
-// whose low bits are the pass-0 digit): each lane keeps the lanes whose bit
-// agrees with its own, the digit's bits first; the lowest of the lanes with
-// its digit adds their number to the block's count.  With rk (pass 0): rk[i] = key | rank << 20 |
-// (count - 1) << 25, the key's rank among the equal digits of its aligned
-// 32-key group and their number, as the scatter ranks them.  With kcnt: the
-// lowest lane of each distinct key adds the key's count in the group.
+// with one ballot per digit bit, each lane keeping the lanes whose bit agrees
+// with its own; the lowest of them adds their number to the block's count.
+// With rk (pass 0): rk[i] = key | rank << 20 | (count - 1) << 25, the key's
+// rank among the equal digits of its aligned 32-key group and their number,
+// as the scatter ranks them.
 constexpr int kCountThreads = 1024;
 template <int STEPS, bool PAIRS>
 __global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __restrict__ keys,
                                                               const int2* __restrict__ pairs, int64_t n, int shift,
-                                                              int R, int dig_bits, int key_bits,
-                                                              int32_t* __restrict__ blkhist,
-                                                              int32_t* __restrict__ rk, int32_t* __restrict__ kcnt,
-                                                              int K) {
+                                                              int R, int bits, int32_t* __restrict__ blkhist,
+                                                              int32_t* __restrict__ rk, int K) {
   constexpr int T = kCountThreads * STEPS;
   extern __shared__ int32_t sh[];
   pdl_trigger();
@@ -75,37 +68,31 @@ __global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __r
     const int64_t i = w0 + 32 * s + lane;
     key[s] = i < n ? (PAIRS ? pairs[i].y : clamp_key(keys[i], K)) : 0;
   }
-  const bool whole = !PAIRS && (rk || kcnt);  // pass 0 of a fit: group by the whole key
-  const int nb = whole ? key_bits : dig_bits;
   const uint32_t lt = lanemask_lt();
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     const int64_t i = w0 + 32 * s + lane;
     const bool valid = i < n;
     const int dig = (key[s] >> shift) & (R - 1);
-    const uint32_t kv = whole ? static_cast<uint32_t>(key[s]) : static_cast<uint32_t>(dig);
-    const uint32_t kz = valid ? kv : 0u;
-    uint32_t same = __ballot_sync(0xffffffffu, valid);
+    const uint32_t dz = valid ? static_cast<uint32_t>(dig) : 0u;
+    uint32_t peers = __ballot_sync(0xffffffffu, valid);
     auto narrow = [&](int bit) {
-      const uint32_t b = (kz >> bit) & 1u;
+      const uint32_t b = (dz >> bit) & 1u;
       const uint32_t bb = __ballot_sync(0xffffffffu, b != 0u);
-      same &= ~(bb ^ (0u - b));
+      peers &= ~(bb ^ (0u - b));
     };
     int bit = 0;
-    for (; bit + 4 <= dig_bits; bit += 4) {
+    for (; bit + 4 <= bits; bit += 4) {
       narrow(bit);
       narrow(bit + 1);
       narrow(bit + 2);
       narrow(bit + 3);
     }
-    for (; bit < dig_bits; ++bit) narrow(bit);
-    const uint32_t peers = same;
-    for (; bit < nb; ++bit) narrow(bit);
+    for (; bit < bits; ++bit) narrow(bit);
     if (!valid) continue;
     const int rank = __popc(peers & lt), cnt = __popc(peers);
     if (rank == 0) atomicAdd(&sh[dig], cnt);
     if (!PAIRS && rk) rk[i] = key[s] | (rank << 20) | ((cnt - 1) << 25);
-    if (!PAIRS && kcnt && (same & lt) == 0) atomicAdd(kcnt + key[s], __popc(same));
   }
   __syncthreads();
   int32_t* out = blkhist + static_cast<int64_t>(blockIdx.x) * R;
@@ -118,59 +105,19 @@ __global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __r
 // shared memory, and each warp rewrites its part as running prefixes.
 constexpr int kColscanWarps = 32;
 
-// start[0..K] of a two-pass sort from the cluster sizes the count kernel
-// added up: an exclusive scan over the clusters (each thread a contiguous run
-// of them, then a block scan of the run sums), start[K] = n; the sizes are
-// zeroed for the next accumulation.  One block of kColscanWarps warps.
-__device__ void starts_from_sizes(int32_t* __restrict__ kcnt, int K, int64_t n, int32_t* __restrict__ start,
-                                  int32_t (*part)[32]) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nt = kColscanWarps * 32;
-  const int per = (K + nt - 1) / nt;
-  const int k0 = static_cast<int>(threadIdx.x) * per;
-  const int k1 = k0 + per < K ? k0 + per : K;
-  int32_t own = 0;
-  for (int k = k0; k < k1; ++k) own += kcnt[k];
-  int32_t x = own;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) part[0][warp] = x;
-  __syncthreads();
-  int32_t run = x - own;
-  for (int w = 0; w < warp; ++w) run += part[0][w];
-  for (int k = k0; k < k1; ++k) {
-    const int32_t c = kcnt[k];
-    start[k] = run;
-    run += c;
-    kcnt[k] = 0;
-  }
-  if (threadIdx.x == 0) start[K] = static_cast<int32_t>(n);
-}
-
 // The block counts are scanned in S segments of consecutive sort blocks, so
 // that few digits still spread over many CTAs: CTA (g, s) takes digits
 // [32 g, 32 g + 32) (one per lane, every load coalesced) and the blocks of
 // segment s, split among its 32 warps; it rewrites them in place as prefixes
 // within the segment and stores the segment's digit totals in segtot[s][d].
 // The scatter adds the totals of the earlier segments (and sums all of them
-// for the digit totals).  With kcnt (two-pass sorts whose cluster sizes the
-// count kernel added up) the grid has one more block, which writes start[]
-// from them.
+// for the digit totals).
 __global__ void __launch_bounds__(kColscanWarps * 32) k_sort_colscan(int32_t* __restrict__ blkhist, int R,
                                                                      int64_t nblk, int S,
-                                                                     int32_t* __restrict__ segtot,
-                                                                     int32_t* __restrict__ kcnt, int K, int64_t n,
-                                                                     int32_t* __restrict__ start) {
+                                                                     int32_t* __restrict__ segtot) {
   __shared__ int32_t part[kColscanWarps][32];
   pdl_trigger();
   pdl_wait();
-  if (kcnt && blockIdx.x == gridDim.x - 1) {
-    starts_from_sizes(kcnt, K, n, start, part);
-    return;
-  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int groups = (R + 31) / 32;
   const int g = static_cast<int>(blockIdx.x) % groups, sg = static_cast<int>(blockIdx.x) / groups;
@@ -547,29 +494,22 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     count_launch(3);  // count, colscan, scatter
     const dim3 hgrid(static_cast<unsigned>(nblk));
     int32_t* rk = pairs_in ? nullptr : a.rk;
-    int32_t* kc0 = pairs_in || c.passes == 1 ? nullptr : a.kcnt;
-    int key_bits = bits;
-    if (kc0)
-      while ((1 << key_bits) < a.K) ++key_bits;
     // T = 4096 or 2048 keys per block: 4 or 2 steps per warp of 1024 threads
     if (c.IPT == 16)
       e = pairs_in ? launch_chained(k_sort_count<4, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
-                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bits, bh, nullptr, nullptr, a.K)
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, nullptr, a.K)
                    : launch_chained(k_sort_count<4, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
-                                    a.n, c.shift[ps], R, bits, key_bits, bh, rk, kc0, a.K);
+                                    a.n, c.shift[ps], R, bits, bh, rk, a.K);
     else
       e = pairs_in ? launch_chained(k_sort_count<2, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
-                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bits, bh, nullptr, nullptr, a.K)
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, nullptr, a.K)
                    : launch_chained(k_sort_count<2, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
-                                    a.n, c.shift[ps], R, bits, key_bits, bh, rk, kc0, a.K);
+                                    a.n, c.shift[ps], R, bits, bh, rk, a.K);
     if (e != cudaSuccess) return e;
-    // a two-pass sort with counted cluster sizes takes start[] from them in
-    // the first column scan (one more block) and needs no bounds kernel
-    int32_t* kc = kc0;
     const int S = c.segs[ps];
     const int64_t L = (nblk + S - 1) / S;
-    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 * S + (kc ? 1 : 0)), dim3(kColscanWarps * 32), 0, s, bh,
-                       R, nblk, S, a.total, kc, a.K, a.n, a.start);
+    e = launch_chained(k_sort_colscan, dim3((R + 31) / 32 * S), dim3(kColscanWarps * 32), 0, s, bh, R, nblk, S,
+                       a.total);
     if (e != cudaSuccess) return e;
     // pass 0 of two writes pairs_tmp; the last pass writes the sorted pairs
     // (and perm when asked for).
@@ -595,7 +535,7 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
                                                           bits, bh, a.total, S, L, out, perm, st, a.K);
     if (e != cudaSuccess) return e;
   }
-  if (c.passes > 1 && !a.kcnt) {
+  if (c.passes > 1) {
     const int64_t cnt = a.n + 1;
     count_launch();
     e = launch_chained(k_bounds, dim3(static_cast<unsigned>((cnt + 255) / 256)), dim3(256), 0, s, a.pairs, a.n, a.K,

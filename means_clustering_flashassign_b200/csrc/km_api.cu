@@ -381,7 +381,6 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   }
   if ((op == KM_OP_FIT || op == KM_OP_FIT_HOST) && !p.small_update) {
     p.off_rk = take(sizeof(int32_t) * static_cast<size_t>(p.rows));
-    if (sc.passes > 1) p.off_kcnt = take(sizeof(int32_t) * static_cast<size_t>(K));
   }
   if (op == KM_OP_FIT_HOST) {
     p.off_dbuf0 = take(static_cast<size_t>(p.chunk_rows) * D * p.es);
@@ -432,8 +431,7 @@ int prepare(Ctx& c, int op, int B, int64_t N, int D, int K, int dtype, int64_t c
 // Update of one instance through the multi-kernel path.
 int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n, float* Cb, void* c_opb, void* caugb,
                     int32_t* countsb, const double* tobjb, int64_t ntiles, double* obj, int mode,
-                    double* acc_ext = nullptr, double* cnt_ext = nullptr, int32_t* rk = nullptr,
-                    int32_t* kcnt = nullptr) {
+                    double* acc_ext = nullptr, double* cnt_ext = nullptr, int32_t* rk = nullptr) {
   const Plan& p = c.p;
   SortArgs sa{idxb,
               n,
@@ -441,7 +439,6 @@ int update_instance(const Ctx& c, const void* Xb, const int32_t* idxb, int64_t n
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
               rk,
-              kcnt,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),
@@ -617,11 +614,8 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
   const size_t xstride = static_cast<size_t>(N) * D * p.es;
   const size_t opstride = static_cast<size_t>(K) * op_row_bytes(p);
   // The sort's count kernel hands its scatter each point's key with its
-  // rank inside its 32-point group, and (two passes) counts the cluster sizes
+  // rank inside its 32-point group
   int32_t* rk = p.small_update ? nullptr : at<int32_t>(c.ws, p.off_rk);
-  int32_t* kcnt = !p.small_update && p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
-  if (kcnt) KM_CUDA(cudaMemsetAsync(kcnt, 0, sizeof(int32_t) * static_cast<size_t>(K), c.s));
-  chain_break();
   for (int t = 0; t < iters; ++t) {
     int64_t groups = 0;
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
@@ -647,7 +641,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
                             caug + static_cast<int64_t>(b) * p.Kp * 32,
                             counts_out ? counts_out + static_cast<int64_t>(b) * K : nullptr,
                             tobj + static_cast<int64_t>(b) * groups * 4, groups, ob, 0, nullptr, nullptr,
-                            rk, kcnt);
+                            rk);
         if (r != KM_OK) return r;
       }
     }
@@ -798,11 +792,6 @@ int fit_stream(const ChunkFn& chunk, bool slot_reuse, const void* C0, int64_t N,
     chain_break();
     KM_CUDA(launch_cprep(C0, dtype, 1, K, p.Kp, D, p.Dp, dtype, C_out, clp, caug, c.s));
     int32_t* rk = at<int32_t>(c.ws, p.off_rk);
-    int32_t* kcnt = p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_kcnt) : nullptr;
-    if (kcnt) {
-      KM_CUDA(cudaMemsetAsync(kcnt, 0, sizeof(int32_t) * static_cast<size_t>(K), c.s));
-      chain_break();
-    }
     for (int i = 0; i < 2; ++i) {
       KM_CUDA(cudaEventRecord(ev_free[i], c.s));
       chain_break();
@@ -854,7 +843,7 @@ int fit_stream(const ChunkFn& chunk, bool slot_reuse, const void* C0, int64_t N,
         Ctx cc = c;
         cc.p = pc;
         rr = update_instance(cc, dbuf[bi], idxc, nr, C_out, nullptr, nullptr, nullptr, tobj, groups, objacc, 1,
-                             nullptr, nullptr, rk, kcnt);
+                             nullptr, nullptr, rk);
         if (rr != KM_OK) return rr;
         KM_CUDA(cudaEventRecord(ev_free[bi], c.s));
         chain_break();
@@ -935,7 +924,6 @@ int km_argsort(const int32_t* idx, int64_t N, int K, int32_t* perm, int32_t* sta
               at<int32_t>(c.ws, p.off_blkhist),
               p.sc.passes > 1 ? at<int32_t>(c.ws, p.off_blkhist1) : nullptr,
               at<int32_t>(c.ws, p.off_rk),
-              nullptr,
               at<int32_t>(c.ws, p.off_total),
               p.sc.passes > 1 ? at<int2>(c.ws, p.off_pairs_tmp) : nullptr,
               at<int2>(c.ws, p.off_pairs),

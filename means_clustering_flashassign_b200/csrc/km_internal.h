@@ -138,7 +138,7 @@ struct Plan {
   size_t off_blkhist = 0, off_blkhist1 = 0, off_total = 0, off_pairs_tmp = 0, off_pairs = 0, off_start = 0;
   size_t off_sums = 0, off_pl = 0, off_pr = 0, off_obj = 0, off_objpart = 0;
   size_t off_dbuf0 = 0, off_dbuf1 = 0, off_acc64 = 0, off_cnt64 = 0, off_objacc = 0;
-  size_t off_rk = 0, off_kcnt = 0;  // fused-sort inputs (single-instance fits)
+  size_t off_rk = 0;  // the sort's packed first-pass keys
   size_t total = 0;
 };
 
@@ -199,8 +199,6 @@ struct SortArgs {
   int32_t* blkhist1;    // [nblk][R1] pass-1 block digit counts (two-pass sorts only)
   int32_t* rk;          // [n] or null: the first pass stores each key with its 32-key group rank
                         // and count there, and its scatter then needs no digit ballots
-  int32_t* kcnt;        // [K] or null (zero on entry): a two-pass sort adds up the cluster sizes
-                        // and takes start[] from them (zeroing them again) instead of k_bounds
   int32_t* total;       // [segs][Rmax]: digit totals of each column-scan segment
   int2* pairs_tmp;      // [n] (two-pass sorts only)
   int2* pairs;          // [n] sorted (point index, cluster id)
