@@ -246,13 +246,18 @@ int make_plan(Plan& p, int op, int B, int64_t N, int D, int K, int dtype, int64_
   ac.natoms = (p.Dop * p.es + 127) / 128;
   int bn0 = K <= 64 ? 64 : (K <= 128 ? 128 : 256);
   bool found = false;
-  // CTA pairs (cta_group::2) for centroid tiles of 128 or 256, else one CTA
-  // per 128-point tile; KM_ASSIGN_FORM=single|pair forces the form.  A sweep
-  // of every tiling that fits (bench.py --tile-sweep) measured pairs 1-2 %
-  // ahead on 1M x 1024 x 128 and level or ahead on the batched and Zipf
-  // shapes.
+  // CTA pairs (cta_group::2) for centroid tiles of 128 or 256 when a point
+  // tile meets several centroid tiles, else one CTA per 128-point tile;
+  // KM_ASSIGN_FORM=single|pair forces the form.  A sweep of every tiling
+  // that fits (bench.py --tile-sweep) measured pairs 1-2 % ahead on
+  // 1M x 1024 x 128 and level on 4M x 16384 x 128, and the single form 6 %
+  // ahead when K fits one centroid tile (512 x 4096 x 64, K = 256) and the
+  // single form keeps its full rings (4 point buffers, 3 centroid stages).
   const int form = assign_form();
-  for (int pair = form == 0 ? 0 : 1; pair >= 0 && !found; --pair) {
+  const bool single_one_ct =
+      K <= bn0 && assign_smem_for(bn0, ac.natoms, 4, 3, false) <= static_cast<size_t>(kSmemLimit);
+  const int pair_first = form == 0 ? 0 : (form == 1 ? 1 : (single_one_ct ? 0 : 1));
+  for (int pair = pair_first; pair >= 0 && !found; --pair) {
     if (form == 1 && !pair && bn0 >= 128) continue;
     for (int bn = bn0; bn >= 64 && !found; bn /= 2) {
       if (pair && bn < 128) continue;

@@ -110,12 +110,15 @@ def test_null_arguments_rejected_before_device_use():
 
 def test_plan_describes_the_chosen_tiling():
     # CTA pairs with 256-wide centroid tiles at D=128; two point buffers and
-    # four centroid stages for K > BN; a 4 x 3 ring when one tile covers K
+    # four centroid stages for K > BN; one CTA per point tile with a 4 x 3
+    # ring when one tile covers K and that ring fits, else pairs
     p = km.plan(km.OP_FIT, 1, 1 << 20, 128, 1024, km.BF16)
     assert (p["pair"], p["BN"], p["XB"], p["CS"], p["Kp"], p["sort_passes"]) == (1, 256, 2, 4, 1024, 1)
     assert p["smem"] <= 232448
     q = km.plan(km.OP_FIT, 512, 4096, 64, 256, km.BF16)
-    assert (q["pair"], q["BN"], q["XB"], q["CS"], q["Kp"]) == (1, 256, 4, 3, 256)
+    assert (q["pair"], q["BN"], q["XB"], q["CS"], q["Kp"]) == (0, 256, 4, 3, 256)
+    q2 = km.plan(km.OP_FIT, 1, 100000, 128, 200, km.BF16)
+    assert (q2["pair"], q2["BN"], q2["Kp"]) == (1, 256, 256)
     r = km.plan(km.OP_FIT, 1, 16384, 32, 64, km.F32)
     assert (r["pair"], r["BN"]) == (0, 64)  # pairs need 128-wide tiles
     assert km.plan(km.OP_FIT, 1, 1 << 22, 128, 16384, km.BF16)["sort_passes"] == 2
