@@ -91,7 +91,7 @@ extern "C" {
 typedef enum km_status {
   KM_OK = 0,
   KM_ERR_INVALID_ARG = 1, /* null required pointer, bad size, misaligned pointer */
-  KM_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve (shape, device) */
+  KM_ERR_UNSUPPORTED = 2, /* valid request the library cannot serve (shape, device) */
   KM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
   KM_ERR_WORKSPACE = 4,   /* workspace null or smaller than km_workspace_size() */
   KM_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait ran out */
