@@ -200,7 +200,7 @@ __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint3
 
 // Lowest centroid index in k's 32-column chunk whose operand row (rb
 // bytes, a multiple of 16) equals row k's; rows holds the instance's rows.
-// Kept out of line: it runs only for points at distance 0.
+// Runs only for points at distance 0, once per point, outside the tile loop.
 __device__ __forceinline__ int lowest_copy(const uint8_t* rows, int64_t rb, int k) {
   const uint4* rk = reinterpret_cast<const uint4*>(rows + k * rb);
   const int n16 = static_cast<int>(rb / 16);
