@@ -736,11 +736,13 @@ __device__ __forceinline__ float emit_operand_lpr(const float (&q)[8], int row_b
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(q[2 * i]), h1 = __float2bfloat16_rn(q[2 * i + 1]);
-      const float f0 = __bfloat162float(h0), f1 = __bfloat162float(h1);
-      if (active) s = fmaf(f1, f1, fmaf(f0, f0, s));
-      const __nv_bfloat16 o0 = __float2bfloat16_rn(-2.f * f0), o1 = __float2bfloat16_rn(-2.f * f1);
-      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o1)) << 16);
+      // two columns per instruction: round the pair to bf16, square the
+      // rounded values, scale by -2 in bf16 (exact: a power of two)
+      const __nv_bfloat162 h = __floats2bfloat162_rn(q[2 * i], q[2 * i + 1]);
+      const float2 f = __bfloat1622float2(h);
+      if (active) s = fmaf(f.y, f.y, fmaf(f.x, f.x, s));
+      const __nv_bfloat162 o = __hmul2(h, __float2bfloat162_rn(-2.f));
+      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o.x)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o.y)) << 16);
     }
     if (writer) reinterpret_cast<uint4*>(static_cast<uint8_t*>(row) + cl * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
@@ -863,11 +865,13 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   const int q1 = q0 + L < N ? q0 + L : N;
   warp_range_sums_keyed<LPR, BF16>(X, p.row_bytes, D, K, pairs, N, q0, q1, lane, slot_k + 2 * warp,
                                    slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
-                                     const float cntf = static_cast<float>(start[k + 1] - start[k]);
-                                     // divide (not multiply by a reciprocal) to match sum / count
+                                     // mean = sum x (1 / count): one division per cluster
+                                     // instead of eight (within 1.5 ulp of sum / count; this
+                                     // tail is the kernel's issue bottleneck)
+                                     const float inv = 1.f / static_cast<float>(start[k + 1] - start[k]);
                                      float q[8];
 #pragma unroll
-                                     for (int i = 0; i < 8; ++i) q[i] = acc[i] / cntf;
+                                     for (int i = 0; i < 8; ++i) q[i] = acc[i] * inv;
                                      store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q,
                                                           1.f);
                                      // operand row and norm row straight from the registers
