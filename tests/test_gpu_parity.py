@@ -86,7 +86,7 @@ def test_assign_batched_instances():
 @pytest.mark.parametrize("N,K,kind", [(100000, 1024, "uniform"), (50000, 16384, "zipf"), (7777, 5000, "uniform"),
                                       (4096, 1, "uniform"), (12345, 300, "empty"), (3, 2, "uniform"),
                                       (300000, 4096, "hot"), (65536, 300, "hot"), (65537, 300, "hot"),
-                                      (65536, 8192, "zipf")])
+                                      (65536, 8192, "zipf"), (700001, 1024, "zipf"), (700001, 9000, "hot")])
 def test_argsort_is_the_stable_inverse_map(N, K, kind):
     rng = np.random.default_rng(N + K)
     if kind == "zipf":
