@@ -31,9 +31,11 @@
  *    (float32 inputs; dot products use a three-term TF32 split, hi*hi + hi*lo
  *    + lo*hi, on the tensor cores, which keeps float32-level accuracy).
  *  - Centroid outputs are float32.  Assignments are int32 in [0, K).
- *  - Ties: the lowest centroid index wins an exact tie.  A cluster with no
- *    member keeps its previous centroid (the pages fix neither rule; these are
- *    the plain readings).
+ *  - Ties: the lowest centroid index wins an exact tie.  The device compares
+ *    distances with the column in their 5 lowest mantissa bits, so distances
+ *    within 2^-18 relative also count as tied; identical centroid rows tie
+ *    exactly, at distance 0 too.  A cluster with no member keeps its previous
+ *    centroid (the pages fix neither rule; these are the plain readings).
  *  - Supported shapes: D % 8 == 0; bf16: 8 <= D <= 256; f32: 8 <= D <= 64;
  *    1 <= K <= min(N, 1 << 20); N < 2^31.  Others return KM_ERR_UNSUPPORTED
  *    or KM_ERR_INVALID_ARG before anything is launched.
