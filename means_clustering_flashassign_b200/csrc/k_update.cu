@@ -105,7 +105,7 @@ __device__ __forceinline__ int clamp_id(int v, int64_t hi) {
   return v < 0 ? 0 : (v >= hi ? static_cast<int>(hi - 1) : v);
 }
 
-template <int LPR, bool BF16, class FinalStore>
+template <int LPR, bool BF16, bool RS, class FinalStore>
 __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D, int K,
                                                       const int2* __restrict__ pairs, int64_t n, int64_t q0,
                                                       int64_t q1, int lane, int* slot_k, float* slot_v,
@@ -126,17 +126,54 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   int open_k = kfirst;
   bool open_left = left_cont;
+  // RS (reduce-scatter): the row groups' partial sums are halved across
+  // lanes each round instead of all-reduced, so every lane ends with its own
+  // NV of the VPL columns and the per-cluster tail runs on all 32 lanes.
+  constexpr int VPL = BF16 ? 8 : 4;  // columns per lane's 16 bytes
+  constexpr bool kRS = RS && (32 / LPR) <= VPL;
   auto flush = [&](bool right) {
+    if constexpr (kRS) {
+      constexpr int NV = VPL / (32 / LPR);
+      int off = 0;
+      int len = VPL;
 #pragma unroll
-    for (int o = LPR; o < 32; o <<= 1)
+      for (int o = LPR; o < 32; o <<= 1) {
+        const int half = len >> 1;
+        const bool up = (lane & o) != 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-    if (!open_left && !right) {
-      final_store(open_k, acc);
+        for (int i = 0; i < VPL / 2; ++i) {
+          if (i < half) {
+            const float a = acc[i], b = acc[half + i];
+            const float keep = up ? b : a;
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, up ? a : b, o);
+          }
+        }
+        if (up) off += half;
+        len = half;
+      }
+      const int col0 = cl * VPL + off;  // this lane's NV columns start here
+      if (!open_left && !right) {
+        final_store(open_k, acc, col0, NV, active);
+      } else {
+        const int slot = open_left ? 0 : 1;
+        if (active)
+#pragma unroll
+          for (int i = 0; i < NV; ++i) slot_v[slot * D + col0 + i] = acc[i];
+        if (lane == 0) slot_k[slot] = open_k;
+      }
     } else {
-      const int slot = open_left ? 0 : 1;
-      store_row<LPR, BF16>(slot_v + slot * D, row_bytes, lane, acc, 1.f);
-      if (lane == 0) slot_k[slot] = open_k;
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      if (!open_left && !right) {
+        if constexpr (RS) final_store(open_k, acc, cl * VPL, VPL, active && lane < LPR);
+        else final_store(open_k, acc);
+      } else {
+        const int slot = open_left ? 0 : 1;
+        store_row<LPR, BF16>(slot_v + slot * D, row_bytes, lane, acc, 1.f);
+        if (lane == 0) slot_k[slot] = open_k;
+      }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -215,7 +252,7 @@ __global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X
   const int64_t Lw = P / W;
   const int64_t q0 = p0 + warp * Lw < p1 ? p0 + warp * Lw : p1;
   const int64_t q1 = q0 + Lw < p1 ? q0 + Lw : p1;
-  warp_range_sums_keyed<LPR, BF16>(X, row_bytes, D, K, pairs, n, q0, q1, lane, slot_k + 2 * warp,
+  warp_range_sums_keyed<LPR, BF16, false>(X, row_bytes, D, K, pairs, n, q0, q1, lane, slot_k + 2 * warp,
                                    slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
                                      store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc,
                                                           1.f);
@@ -721,52 +758,6 @@ __device__ __forceinline__ void scan256_exclusive(int32_t* v, int32_t* wsum) {
 
 static_assert(kSmallMaxN <= 65536 && kSmallMaxK <= 65536, "key and rank are packed in 16 bits each");
 
-// Operand row of a centroid held in the row-gather register layout (lane
-// cl = lane % LPR holds the 16-byte column group cl: 8 bf16 or 4 float
-// columns of the mean), and ||c||^2 of the operand values, on every lane.
-// bf16: -2 * bf16(mean); f32: the TF32 split -2 * [hi | lo | hi] of row
-// length 3 * Dp.  Lanes with lane >= LPR only help reduce.
-template <int LPR, bool BF16>
-__device__ __forceinline__ float emit_operand_lpr(const float (&q)[8], int row_bytes, int Dp, void* row, int lane) {
-  const int cl = lane % LPR;
-  const bool active = cl * 16 < row_bytes;
-  const bool writer = active && lane < LPR && row != nullptr;
-  float s = 0.f;
-  if constexpr (BF16) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      // two columns per instruction: round the pair to bf16, square the
-      // rounded values, scale by -2 in bf16 (exact: a power of two)
-      const __nv_bfloat162 h = __floats2bfloat162_rn(q[2 * i], q[2 * i + 1]);
-      const float2 f = __bfloat1622float2(h);
-      if (active) s = fmaf(f.y, f.y, fmaf(f.x, f.x, s));
-      const __nv_bfloat162 o = __hmul2(h, __float2bfloat162_rn(-2.f));
-      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o.x)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o.y)) << 16);
-    }
-    if (writer) reinterpret_cast<uint4*>(static_cast<uint8_t*>(row) + cl * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-    float hi[4], lo[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (active) s = fmaf(q[i], q[i], s);
-      hi[i] = tf32_round(q[i]);
-      lo[i] = tf32_round(q[i] - hi[i]);
-    }
-    if (writer) {
-      float* o = static_cast<float*>(row) + cl * 4;
-      reinterpret_cast<float4*>(o)[0] = make_float4(-2.f * hi[0], -2.f * hi[1], -2.f * hi[2], -2.f * hi[3]);
-      reinterpret_cast<float4*>(o + Dp)[0] = make_float4(-2.f * lo[0], -2.f * lo[1], -2.f * lo[2], -2.f * lo[3]);
-      reinterpret_cast<float4*>(o + 2 * Dp)[0] = make_float4(-2.f * hi[0], -2.f * hi[1], -2.f * hi[2], -2.f * hi[3]);
-    }
-  }
-  // the LPR lanes of one row hold its column groups; lanes of other rows
-  // (sub > 0) hold copies: reduce inside groups of LPR lanes
-#pragma unroll
-  for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  return s;
-}
-
 template <int LPR, bool BF16>
 __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   extern __shared__ __align__(16) int32_t ssm[];
@@ -863,25 +854,65 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   const int L = (N + W - 1) / W;
   const int q0 = warp * L < N ? warp * L : N;
   const int q1 = q0 + L < N ? q0 + L : N;
-  warp_range_sums_keyed<LPR, BF16>(X, p.row_bytes, D, K, pairs, N, q0, q1, lane, slot_k + 2 * warp,
-                                   slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
-                                     // mean = sum x (1 / count): one division per cluster
-                                     // instead of eight (within 1.5 ulp of sum / count; this
-                                     // tail is the kernel's issue bottleneck)
-                                     const float inv = 1.f / static_cast<float>(start[k + 1] - start[k]);
-                                     float q[8];
+  warp_range_sums_keyed<LPR, BF16, true>(
+      X, p.row_bytes, D, K, pairs, N, q0, q1, lane, slot_k + 2 * warp, slot_v + 2 * warp * D,
+      [&](int k, const float (&v)[8], int col0, int nv, bool writer) {
+        // mean = sum x (1 / count): one division per cluster (within 1.5 ulp of
+        // sum / count; this tail is the kernel's issue bottleneck).  Each lane
+        // holds nv columns from col0 (all lanes distinct when reduce-scattered).
+        const float inv = 1.f / static_cast<float>(start[k + 1] - start[k]);
+        const int64_t grow = static_cast<int64_t>(b) * K + k;
+        void* orow = op_row_of(p, grow);
+        float* crow = C + static_cast<int64_t>(k) * D;
+        float s = 0.f;
+        if constexpr (BF16) {
+          if (nv == 1) {  // 8 row groups (16-column rows): one column per lane, any offset
+            if (writer) {
+              const float q = v[0] * inv;
+              crow[col0] = q;
+              const __nv_bfloat16 h = __float2bfloat16_rn(q);
+              const float f = __bfloat162float(h);
+              s = f * f;
+              if (orow) static_cast<__nv_bfloat16*>(orow)[col0] = __float2bfloat16_rn(-2.f * f);
+            }
+          } else {
 #pragma unroll
-                                     for (int i = 0; i < 8; ++i) q[i] = acc[i] * inv;
-                                     store_row<LPR, BF16>(C + static_cast<int64_t>(k) * D, p.row_bytes, lane, q,
-                                                          1.f);
-                                     // operand row and norm row straight from the registers
-                                     const int64_t grow = static_cast<int64_t>(b) * K + k;
-                                     void* orow = op_row_of(p, grow);
-                                     const float sq = emit_operand_lpr<LPR, BF16>(q, p.row_bytes, p.Dp, orow, lane);
-                                     if (lane == 0 && p.caug)
-                                       write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes,
-                                                     p.dtype, sq, 1);
-                                   });
+          for (int i = 0; i < 8; i += 2) {
+            // nv is even here and so is col0: the pair stores are aligned
+            if (i < nv && writer) {
+              const float q0v = v[i] * inv, q1v = v[i + 1] * inv;
+              *reinterpret_cast<float2*>(crow + col0 + i) = make_float2(q0v, q1v);
+              // round the pair to bf16, square the rounded values, scale by -2 in
+              // bf16 (exact: a power of two)
+              const __nv_bfloat162 h = __floats2bfloat162_rn(q0v, q1v);
+              const float2 f = __bfloat1622float2(h);
+              s = fmaf(f.y, f.y, fmaf(f.x, f.x, s));
+              if (orow)
+                *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(orow) + col0 + i) =
+                    __hmul2(h, __float2bfloat162_rn(-2.f));
+            }
+          }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i < nv && writer) {
+              const float q = v[i] * inv;
+              crow[col0 + i] = q;
+              s = fmaf(q, q, s);
+              if (orow) {
+                float* o = static_cast<float*>(orow);
+                const float hi = tf32_round(q), lo = tf32_round(q - hi);
+                o[col0 + i] = -2.f * hi;
+                o[p.Dp + col0 + i] = -2.f * lo;
+                o[2 * p.Dp + col0 + i] = -2.f * hi;
+              }
+            }
+          }
+        }
+        s = warp_sum_f(s);
+        if (lane == 0 && p.caug) write_aug_row(p.caug + (static_cast<int64_t>(b) * p.Kp + k) * kAugBytes, p.dtype, s, 1);
+      });
   __syncthreads();
   int* cut_list = tmp;  // clusters finished by the combine below (at most 2W)
   if (threadIdx.x == 0) tmp[255] = 0;
