@@ -229,9 +229,9 @@ def shard_rows(n_per_rank: int, world: int, rank: int) -> slice:
 
 def repeats_for(min_timed_s: float, est_ms: float) -> int:
     """Repetitions of the K-step fit that make the timed region last at least
-    min_timed_s, given one repetition's estimated milliseconds (from the
-    warm-up, which runs before the clock settles under the power cap, hence
-    a 15 % margin)."""
+    min_timed_s, given one repetition's estimated milliseconds (from an
+    untimed fit that runs before the clock settles under the power cap,
+    hence a 15 % margin)."""
     return max(1, int(math.ceil(min_timed_s * 1.15e3 / max(est_ms, 1e-3))))
 
 
@@ -377,8 +377,11 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         return r["iters_ms"], c0.elapsed_time(c1)
 
-    warm_ms, _ = one_fit(args.warmup)
-    est = warm_ms / max(args.warmup, 1) * args.steps
+    one_fit(args.warmup)
+    # One more untimed K-step fit sizes the repeats: the warm-up call also
+    # carries the first call's module loading and workspace set-up, which
+    # would inflate the estimate and shorten the timed region.
+    _, est = one_fit(args.steps)
     reps = int(max_over_ranks(world, float(repeats_for(args.min_timed_s, est)), device=dev))
     barrier(world)
     rep_ms, call_ms = [], []
