@@ -25,8 +25,8 @@
 // more identical centroid rows, which the tensor cores score bit for bit
 // alike.  So a point whose best ends at or below zero takes the lowest
 // centroid of its winning chunk whose operand row equals the winner's (a
-// rare, out-of-line scan of at most 31 rows).  The lowest index wins exact
-// ties.  (Distances closer than 2^-18 relative also compare equal; that is
+// rare pass in which the warp compares up to 31 rows at once).  The lowest
+// index wins exact ties.  (Distances closer than 2^-18 relative also compare equal; that is
 // far inside the parity rule's near-tie band.)
 //
 // Structure: persistent CTAs (one per SM), warp-specialised:
@@ -200,20 +200,48 @@ __device__ __forceinline__ uint32_t chunk_min_key(const uint32_t (&v)[CW], uint3
 
 // Lowest centroid index in k's 32-column chunk whose operand row (rb
 // bytes, a multiple of 16) equals row k's; rows holds the instance's rows.
-// Runs only for points at distance 0, once per point, outside the tile loop.
-__device__ __forceinline__ int lowest_copy(const uint8_t* rows, int64_t rb, int k) {
-  const uint4* rk = reinterpret_cast<const uint4*>(rows + k * rb);
-  const int n16 = static_cast<int>(rb / 16);
-  for (int c = k & ~31; c < k; ++c) {
-    const uint4* rc = reinterpret_cast<const uint4*>(rows + c * rb);
-    int i = 0;
-    for (; i < n16; ++i) {
+// The whole warp takes part: lane c compares row (k & ~31) + c for the
+// columns below k, so the candidates are read in one parallel round rather
+// than one after another.  Runs only for points at distance 0.
+__device__ __forceinline__ int lowest_copy(const uint8_t* rows, int64_t rb, int k, int lane) {
+  const int c0 = k & ~31;
+  bool eq = lane < (k & 31);
+  if (eq) {
+    const uint4* rk = reinterpret_cast<const uint4*>(rows + k * rb);
+    const uint4* rc = reinterpret_cast<const uint4*>(rows + (c0 + lane) * rb);
+    const int n16 = static_cast<int>(rb / 16);
+    for (int i = 0; i < n16; ++i) {
       const uint4 u = rc[i], w = rk[i];
-      if (u.x != w.x || u.y != w.y || u.z != w.z || u.w != w.w) break;
+      if (u.x != w.x || u.y != w.y || u.z != w.z || u.w != w.w) {
+        eq = false;
+        break;
+      }
     }
-    if (i == n16) return c;
   }
-  return k;
+  const unsigned m = __ballot_sync(0xffffffffu, eq);
+  return m ? c0 + __ffs(m) - 1 : k;
+}
+
+// The warp's points at distance 0 (the zero set) take the lowest identical
+// centroid row, one warp-wide comparison each.  This runs rarely.  The
+// CTA-pair kernels call it out of line (inlined, it costs their hot loop
+// two registers); the single-CTA kernels inline it (out of line, they
+// spill).
+__device__ __forceinline__ int zero_distance_ties_body(const uint8_t* rows, int64_t rb, int bk, bool zero, int lane) {
+  for (unsigned need = __ballot_sync(0xffffffffu, zero); need; need &= need - 1) {
+    const int src = __ffs(need) - 1;
+    const int kk = lowest_copy(rows, rb, __shfl_sync(0xffffffffu, bk, src), lane);
+    if (lane == src) bk = kk;
+  }
+  return bk;
+}
+__device__ __noinline__ int zero_distance_ties_call(const uint8_t* rows, int64_t rb, int bk, bool zero, int lane) {
+  return zero_distance_ties_body(rows, rb, bk, zero, lane);
+}
+template <bool OUT_OF_LINE>
+__device__ __forceinline__ int zero_distance_ties(const uint8_t* rows, int64_t rb, int bk, bool zero, int lane) {
+  if constexpr (OUT_OF_LINE) return zero_distance_ties_call(rows, rb, bk, zero, lane);
+  else return zero_distance_ties_body(rows, rb, bk, zero, lane);
 }
 
 // ONE_CT: one centroid tile per point tile (K <= BN), kept resident per
@@ -507,10 +535,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       // the point tile's result: argmin index, distance, sort counts, objective
       auto emit = [&]() {
         float md = 0.f;
+        if (p.cop && __any_sync(0xffffffffu, valid && best <= 0.f))
+          bk = zero_distance_ties<PAIR>(p.cop + static_cast<int64_t>(b) * p.K * p.cop_rb, p.cop_rb, bk,
+                                        valid && best <= 0.f, lane);
         if (valid) {
           const int64_t o = static_cast<int64_t>(b) * p.rows + row;
           md = fmaxf(0.f, best);
-          if (best <= 0.f && p.cop) bk = lowest_copy(p.cop + static_cast<int64_t>(b) * p.K * p.cop_rb, p.cop_rb, bk);
           p.idx[o] = bk;
           if (p.mindist) p.mindist[o] = md;
         }
