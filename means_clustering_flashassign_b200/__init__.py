@@ -399,9 +399,9 @@ def fit_data_parallel(X: torch.Tensor, C0: torch.Tensor, iters: int, *, group=No
 
 def plan(op: int, B: int, N: int, D: int, K: int, dtype: int, chunk_rows: int = 0) -> dict:
     """The tiling the library would use for this shape (host-only query)."""
-    out = (ctypes.c_int64 * 8)()
+    out = (ctypes.c_int64 * 9)()
     _check(library().km_plan_describe(op, B, N, D, K, dtype, chunk_rows, ctypes.cast(out, ctypes.c_void_p)))
-    keys = ("pair", "BN", "XB", "CS", "smem", "Kp", "sort_passes", "sort_block")
+    keys = ("pair", "BN", "XB", "CS", "smem", "Kp", "sort_passes", "sort_block", "small_update")
     return {k: int(v) for k, v in zip(keys, out)}
 
 

@@ -984,6 +984,7 @@ int km_plan_describe(int op, int B, int64_t N, int D, int K, int dtype, int64_t 
   out[5] = p.Kp;
   out[6] = p.sc.passes;
   out[7] = p.sc.T;
+  out[8] = p.small_update ? 1 : 0;
   return KM_OK;
 }
 

@@ -131,19 +131,28 @@ def test_update_matches_member_means(N, D, K, dtype, weights):
     assert torch.equal(C[torch.from_numpy(empty).to(DEV)], Cprev[torch.from_numpy(empty).to(DEV)])
 
 
-@pytest.mark.parametrize("B,N,D,K", [(5, 4096, 64, 256), (3, 1000, 128, 37), (4, 8192, 32, 1024)])
-def test_update_batched_fused_path(B, N, D, K):
-    X, _ = _mixture(N, D, K, "bf16", B=B, seed=B)
+# The fused one-CTA-per-instance update: row sizes of 16 to 512 bytes (one
+# to four 128-byte word groups per lane), row stages of one to 32 rows,
+# clusters longer than a warp range and single-row clusters.
+FUSED = [(5, 4096, 64, 256, "bf16"), (3, 1000, 128, 37, "bf16"), (4, 8192, 32, 1024, "bf16"),
+         (2, 3000, 256, 100, "bf16"), (3, 2500, 192, 300, "bf16"), (2, 777, 8, 5, "bf16"),
+         (3, 16, 256, 4, "bf16"), (2, 4096, 64, 256, "f32"), (3, 1500, 24, 700, "f32"), (2, 8192, 64, 1024, "f32")]
+
+
+@pytest.mark.parametrize("B,N,D,K,dtype", FUSED)
+def test_update_batched_fused_path(B, N, D, K, dtype):
+    X, _ = _mixture(N, D, K, dtype, B=B, seed=B)
     rng = np.random.default_rng(B)
     idx = rng.integers(0, K, (B, N)).astype(np.int32)
     idx[:, : N // 5] = K - 1
     Cprev = torch.randn(B, K, D, device=DEV)
+    assert km.plan(km.OP_UPDATE, B, N, D, K, km.BF16 if dtype == "bf16" else km.F32)["small_update"]
     C, counts = km.update(X, torch.from_numpy(idx).to(DEV), Cprev.clone())
     torch.cuda.synchronize()
     for b in range(B):
         Cref, cref = oracle.update(X[b], idx[b], Cprev[b])
         assert np.array_equal(counts[b].cpu().numpy(), cref)
-        assert centroid_rel_err(C[b], Cref) <= CTOL["bf16"]
+        assert centroid_rel_err(C[b], Cref) <= CTOL[dtype]
 
 
 def _stepwise(X, C0, iters, kind):
