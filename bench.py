@@ -407,6 +407,9 @@ def run_ours(args, world, rank, local):
     # assignment and the update stop those kernels from overlapping their
     # launches, so it is kept apart from `value`.
     phase = km.fit_profile(X, C0, args.steps)["phase_ms"] if not dp else None
+    # The same fit replayed as a CUDA graph (km_fit_graph_*): device time of
+    # the whole call, comparable with value_call.
+    graph_ms = graph_call_ms(km, X, C0, args.steps) if not dp and rank == 0 else None
     if rank == 0:
         pk, pk_kind = peaks()
         value = job_rate(args.steps, world, ms_max)
@@ -418,6 +421,7 @@ def run_ours(args, world, rank, local):
             "repeats": reps, "timed_region_s": round(timed_s, 3),
             "ms_per_step_each_repeat": [round(v / args.steps, 4) for v in rep_ms[:64]],
             "value_call": round(job_rate(args.steps, world, ms_call_max), 3),
+            "value_graph_call": round(job_rate(args.steps, 1, graph_ms), 3) if graph_ms else None,
             "ms_call": round(ms_call_max, 4),
             "gpu_launches": int(launches),
             "gpu_launches_per_repeat": int(launches) // reps,
@@ -465,6 +469,21 @@ def run_ours(args, world, rank, local):
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl, X, C0, args.cpu_seconds)
     return res
+
+
+def graph_call_ms(km, X, C0, steps, budget_s=0.3):
+    """Median device time of one launch of the fit captured as a CUDA graph
+    (events around each launch), over launches worth about budget_s."""
+    g = km.FitGraph(X, C0, steps, want_idx=False)
+    try:
+        for _ in range(3):
+            g.launch()
+        torch.cuda.synchronize()
+        first = _event_ms(g.launch, reps=1)
+        n = max(5, min(200, int(budget_s * 1e3 / max(first, 1e-3))))
+        return _event_ms(g.launch, reps=n)
+    finally:
+        g.close()
 
 
 def _event_ms(fn, reps=3):

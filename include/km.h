@@ -235,6 +235,39 @@ int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, 
                  void* workspace, size_t workspace_bytes, void* stream, float* iters_ms);
 
 /*
+ * A fit captured once as a CUDA graph and then replayed.  For shapes whose
+ * kernels run for microseconds, launching them one by one from the host
+ * costs about as much as running them; a graph launch enqueues the whole
+ * fit at once.
+ *   km_fit_graph_create records what km_fit would enqueue with these
+ *     arguments (stream capture on a private stream: nothing runs, no
+ *     caller stream is used) on the current device.  With timed != 0 (and
+ *     iters > 0) the graph also records two events around its iterations,
+ *     as km_fit_timed does.  *graph receives the handle (NULL on failure).
+ *   km_fit_graph_launch enqueues one complete fit on `stream` (any stream of
+ *     the creating device, which must be current): every launch starts again
+ *     from C0 and writes the same outputs km_fit would.  The graph holds the
+ *     argument pointers, not the data: the buffers must stay allocated until
+ *     km_fit_graph_destroy, and their contents may change between launches.
+ *     Asynchronous; launches of one graph run one after another.
+ *   km_fit_graph_elapsed waits for the last launch and writes the
+ *     milliseconds of its iterations (timed graphs only).
+ *   km_fit_graph_destroy releases the graph (after its launches complete;
+ *     NULL is accepted).
+ * Switches read at launch time by km_fit (KM_PDL, KM_ASSIGN_FORM,
+ * KM_ASSIGN_TILE, KM_FAULT) are read once, at creation.  Arguments and
+ * errors of create as km_fit; km_launch_count counts the graph's kernels at
+ * every launch, not at creation.
+ */
+typedef struct km_fit_graph_t* km_fit_graph;
+int km_fit_graph_create(km_fit_graph* graph, const void* X, const void* C0, int B, int64_t N, int D, int K,
+                        int dtype, int iters, float* C_out, int32_t* idx_out, int32_t* counts_out,
+                        double* objective_hist, void* workspace, size_t workspace_bytes, int timed);
+int km_fit_graph_launch(km_fit_graph graph, void* stream);
+int km_fit_graph_elapsed(km_fit_graph graph, float* iters_ms);
+int km_fit_graph_destroy(km_fit_graph graph);
+
+/*
  * Number of kernels this library has enqueued in this process since it was
  * loaded (all entry points, all threads).  For accounting in benchmarks.
  */

@@ -28,7 +28,8 @@ from . import build as _build
 __all__ = ["KMError", "library", "library_path", "workspace_size", "assign", "update", "fit", "fit_host",
            "workspace_status", "selftest_timeout", "argsort", "fit_profile", "launch_count", "assign_static",
            "ablation_assign_materialized", "ablation_update_atomic", "plan", "update_accumulate",
-           "finalize_sums", "fit_data_parallel", "pack_layout", "exchange_packed", "fit_source", "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
+           "finalize_sums", "fit_data_parallel", "pack_layout", "exchange_packed", "fit_source", "FitGraph",
+           "OP_ASSIGN", "OP_UPDATE", "OP_FIT", "OP_FIT_HOST",
            "OP_ARGSORT",
            "F32", "BF16", "EXPORTS"]
 
@@ -40,7 +41,8 @@ EXPORTS = ["km_version", "km_status_string", "km_last_error", "km_workspace_size
            "km_assign", "km_update", "km_argsort", "km_fit", "km_fit_profile", "km_fit_timed", "km_fit_host", "km_selftest_timeout",
            "km_launch_count", "km_assign_static", "km_ablation_workspace_size", "km_ablation_assign_materialized",
            "km_ablation_update_atomic", "km_plan_describe", "km_update_accumulate", "km_finalize_sums",
-           "km_fit_source"]
+           "km_fit_source", "km_fit_graph_create", "km_fit_graph_launch", "km_fit_graph_elapsed",
+           "km_fit_graph_destroy"]
 
 _lock = threading.Lock()
 _lib = None
@@ -97,6 +99,10 @@ def library() -> ctypes.CDLL:
             L.km_launch_count.restype = ctypes.c_uint64
             L.km_assign_static.argtypes = [P, P, I, I64, I, I, I, P, P, P, P]
             L.km_fit_source.argtypes = [CHUNK_SOURCE, P, P, I64, I, I, I, I, I64, P, P, P, P, P, SZ, P]
+            L.km_fit_graph_create.argtypes = [P, P, P, I, I64, I, I, I, I, P, P, P, P, P, SZ, I]
+            L.km_fit_graph_launch.argtypes = [P, P]
+            L.km_fit_graph_elapsed.argtypes = [P, P]
+            L.km_fit_graph_destroy.argtypes = [P]
             for f in EXPORTS:
                 getattr(L, f).restype = getattr(L, f).restype or I
             _lib = L
@@ -541,6 +547,62 @@ def fit_timed(X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_
                                       _ptr(counts_out), _ptr(objective), _ptr(ws), ws.numel(), _stream(stream),
                                       ctypes.byref(ms)))
     return dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective, iters_ms=float(ms.value))
+
+
+class FitGraph:
+    """fit() captured once as a CUDA graph (km_fit_graph_create); every
+    launch() enqueues one complete fit from C0 into the same output tensors.
+
+    The graph holds pointers: this object keeps X, C0, the outputs and the
+    workspace alive, and the caller may refill X / C0 in place between
+    launches.  With timed=True, iters_ms() gives the device time of the last
+    launch's iterations.  close() (or garbage collection) releases it.
+    """
+
+    def __init__(self, X: torch.Tensor, C0: torch.Tensor, iters: int, *, C_out=None, idx_out=None,
+                 counts_out=None, objective=None, want_idx: bool = True, workspace=None, timed: bool = False):
+        self._h = None
+        _contig_cuda(X, "X")
+        with torch.cuda.device(X.device):
+            B, N, D, K, dt, C_out, idx_out, counts_out, objective = _fit_outputs(
+                X, C0, iters, C_out, idx_out, counts_out, objective, want_idx, None)
+            ws = _workspace(OP_FIT, B, N, D, K, dt, X.device, workspace)
+            _check_tensor(ws, "workspace", X.device, torch.uint8)
+            h = ctypes.c_void_p()
+            _check(library().km_fit_graph_create(ctypes.byref(h), _ptr(X), _ptr(C0), B, N, D, K, dt, iters,
+                                                 _ptr(C_out), _ptr(idx_out), _ptr(counts_out), _ptr(objective),
+                                                 _ptr(ws), ws.numel(), 1 if timed else 0))
+        self._h = h
+        self.device = X.device
+        self.X, self.C0, self.workspace = X, C0, ws
+        self.result = dict(C=C_out, idx=idx_out, counts=counts_out, objective=objective)
+
+    def launch(self, stream=None) -> dict:
+        """Enqueue one fit (asynchronous); returns the output tensors."""
+        if self._h is None:
+            raise RuntimeError("the graph was closed")
+        _check_stream(stream, self.device)
+        with torch.cuda.device(self.device):
+            _check(library().km_fit_graph_launch(self._h, _stream(stream)))
+        return self.result
+
+    def iters_ms(self) -> float:
+        """Waits for the last launch; milliseconds of its iterations."""
+        ms = ctypes.c_float(0.0)
+        _check(library().km_fit_graph_elapsed(self._h, ctypes.byref(ms)))
+        return float(ms.value)
+
+    def close(self) -> None:
+        if self._h is not None:
+            torch.cuda.synchronize(self.device)
+            library().km_fit_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def launch_count() -> int:

@@ -588,9 +588,13 @@ int km_update(const void* X, const int32_t* idx, int B, int64_t N, int D, int K,
   return KM_OK;
 }
 
+// ev: events recorded around every phase (per_phase) or around the whole
+// loop; ext_events: as event-record nodes of a graph being captured.
 static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int K, int dtype, int iters,
                     float* C_out, int32_t* idx_out, int32_t* counts_out, double* objective_hist, void* workspace,
-                    size_t workspace_bytes, void* stream, cudaEvent_t* ev, bool per_phase = true) {
+                    size_t workspace_bytes, void* stream, cudaEvent_t* ev, bool per_phase = true,
+                    bool ext_events = false) {
+  const unsigned rec_flags = ext_events ? cudaEventRecordExternal : cudaEventRecordDefault;
   if (!X || !C0 || !C_out) return fail(KM_ERR_INVALID_ARG, "X, C0 and C_out are required");
   if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
   if (!aligned16(X) || !aligned16(C0) || !aligned16(C_out))
@@ -626,12 +630,12 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
     AssignArgs a{&xmap, &xamap, &cmap, &camap, B, N, K, p.Kp, idx, nullptr, tobj, c.status(), wait_limit_ns(),
                  &groups, clp, op_row_bytes(p)};
     if (ev && (per_phase || t == 0)) {
-      KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t : 0], c.s));
+      KM_CUDA(cudaEventRecordWithFlags(ev[per_phase ? 3 * t : 0], c.s, rec_flags));
       chain_break();
     }
     KM_CUDA(launch_assign(p, a, c.s));
     if (ev && per_phase) {
-      KM_CUDA(cudaEventRecord(ev[3 * t + 1], c.s));
+      KM_CUDA(cudaEventRecordWithFlags(ev[3 * t + 1], c.s, rec_flags));
       chain_break();
     }
     if (p.small_update) {
@@ -651,7 +655,7 @@ static int fit_impl(const void* X, const void* C0, int B, int64_t N, int D, int 
       }
     }
     if (ev && (per_phase || t == iters - 1)) {
-      KM_CUDA(cudaEventRecord(ev[per_phase ? 3 * t + 2 : 1], c.s));
+      KM_CUDA(cudaEventRecordWithFlags(ev[per_phase ? 3 * t + 2 : 1], c.s, rec_flags));
       chain_break();
     }
   }
@@ -730,6 +734,99 @@ int km_fit_timed(const void* X, const void* C0, int B, int64_t N, int D, int K, 
     r = fail(KM_ERR_CUDA, "cudaEventElapsedTime failed");
   for (auto e : ev) cudaEventDestroy(e);
   return r;
+}
+
+}  // extern "C"
+
+struct km_fit_graph_t {
+  cudaGraphExec_t exec = nullptr;
+  cudaEvent_t ev[2] = {nullptr, nullptr};
+  bool timed = false;
+  bool launched = false;
+  uint64_t kernels = 0;  // kernels per launch
+  int device = -1;
+};
+
+extern "C" {
+
+int km_fit_graph_create(km_fit_graph* graph, const void* X, const void* C0, int B, int64_t N, int D, int K,
+                        int dtype, int iters, float* C_out, int32_t* idx_out, int32_t* counts_out,
+                        double* objective_hist, void* workspace, size_t workspace_bytes, int timed) {
+  g_err.clear();
+  if (!graph) return fail(KM_ERR_INVALID_ARG, "graph is required");
+  *graph = nullptr;
+  if (iters < 0) return fail(KM_ERR_INVALID_ARG, "iters must be >= 0");
+  fault_arm_from_env();
+  auto* g = new km_fit_graph_t();
+  g->timed = timed != 0 && iters > 0;
+  cudaStream_t cs = nullptr;
+  cudaGraph_t gr = nullptr;
+  auto cleanup = [&](int code) {
+    if (gr) cudaGraphDestroy(gr);
+    if (cs) cudaStreamDestroy(cs);
+    km_fit_graph_destroy(g);
+    return code;
+  };
+  if (cudaGetDevice(&g->device) != cudaSuccess) return cleanup(fail(KM_ERR_CUDA, "no CUDA device"));
+  if (g->timed)
+    for (auto& e : g->ev)
+      if (fault_hit(kFaultAlloc) || cudaEventCreate(&e) != cudaSuccess)
+        return cleanup(fail(KM_ERR_CUDA, "cudaEventCreate failed"));
+  // Capture on a private stream: nothing is executed, and no caller stream
+  // is involved until a launch.
+  if (fault_hit(kFaultAlloc) || cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess)
+    return cleanup(fail(KM_ERR_CUDA, "cudaStreamCreate failed"));
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return cleanup(fail(KM_ERR_CUDA, "cudaStreamBeginCapture failed"));
+  t_fault_keep = true;
+  t_capture_count = &g->kernels;
+  int r = fit_impl(X, C0, B, N, D, K, dtype, iters, C_out, idx_out, counts_out, objective_hist, workspace,
+                   workspace_bytes, cs, g->timed ? g->ev : nullptr, false, true);
+  t_capture_count = nullptr;
+  t_fault_keep = false;
+  const cudaError_t ec = cudaStreamEndCapture(cs, &gr);
+  if (r != KM_OK) return cleanup(r);
+  if (ec != cudaSuccess || !gr) return cleanup(fail(KM_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ec)));
+  if (cudaGraphInstantiate(&g->exec, gr, 0) != cudaSuccess)
+    return cleanup(fail(KM_ERR_CUDA, "cudaGraphInstantiate failed"));
+  cudaGraphDestroy(gr);
+  gr = nullptr;
+  cudaStreamDestroy(cs);
+  *graph = g;
+  return KM_OK;
+}
+
+int km_fit_graph_launch(km_fit_graph graph, void* stream) {
+  g_err.clear();
+  if (!graph || !graph->exec) return fail(KM_ERR_INVALID_ARG, "graph is NULL or was not created");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != graph->device)
+    return fail(KM_ERR_INVALID_ARG, "the current device is not the one the graph was created on");
+  if (cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(KM_ERR_CUDA, "cudaGraphLaunch failed");
+  count_launch(graph->kernels);
+  graph->launched = true;
+  return KM_OK;
+}
+
+int km_fit_graph_elapsed(km_fit_graph graph, float* iters_ms) {
+  g_err.clear();
+  if (!graph || !iters_ms) return fail(KM_ERR_INVALID_ARG, "graph and iters_ms are required");
+  if (!graph->timed) return fail(KM_ERR_INVALID_ARG, "the graph was created without timing (or with iters = 0)");
+  if (!graph->launched) return fail(KM_ERR_INVALID_ARG, "the graph has not been launched");
+  if (cudaEventSynchronize(graph->ev[1]) != cudaSuccess ||
+      cudaEventElapsedTime(iters_ms, graph->ev[0], graph->ev[1]) != cudaSuccess)
+    return fail(KM_ERR_CUDA, "reading the graph's events failed");
+  return KM_OK;
+}
+
+int km_fit_graph_destroy(km_fit_graph graph) {
+  if (!graph) return KM_OK;
+  if (graph->exec) cudaGraphExecDestroy(graph->exec);
+  for (auto e : graph->ev)
+    if (e) cudaEventDestroy(e);
+  delete graph;
+  return KM_OK;
 }
 
 }  // extern "C"

@@ -23,11 +23,17 @@ constexpr int kSmallMaxN = 8192;
 constexpr int kSmallMaxK = 1024;
 
 // Process-wide count of kernels enqueued by this library (km_launch_count).
+// While this thread captures a CUDA graph, its launches are only recorded,
+// so they go to the graph's own count (added at every graph launch).
 inline std::atomic<uint64_t>& launch_counter() {
   static std::atomic<uint64_t> c{0};
   return c;
 }
-inline void count_launch(uint64_t n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
+inline thread_local uint64_t* t_capture_count = nullptr;
+inline void count_launch(uint64_t n = 1) {
+  if (t_capture_count) *t_capture_count += n;
+  else launch_counter().fetch_add(n, std::memory_order_relaxed);
+}
 
 // Host-side fault injection, for testing the error paths without faulting a
 // GPU.  KM_FAULT=<point>[:<n>] in the environment (read at the entry of every

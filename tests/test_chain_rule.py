@@ -76,7 +76,7 @@ def test_assignment_kernel_does_not_release_dependents_early():
 
 def test_abi_layer_breaks_the_chain_after_every_stream_operation():
     text = _src("km_api.cu")
-    ops = list(re.finditer(r"\b(cudaMemsetAsync|cudaMemcpyAsync|cudaEventRecord|cudaStreamWaitEvent)\(", text))
+    ops = list(re.finditer(r"\b(cudaMemsetAsync|cudaMemcpyAsync|cudaEventRecord|cudaEventRecordWithFlags|cudaStreamWaitEvent)\(", text))
     assert len(ops) >= 10
     for m in ops:
         end = text.index(";", m.end())  # end of the statement holding the call
