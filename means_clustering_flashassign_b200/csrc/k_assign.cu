@@ -244,6 +244,32 @@ __device__ __forceinline__ int zero_distance_ties(const uint8_t* rows, int64_t r
   else return zero_distance_ties_body(rows, rb, bk, zero, lane);
 }
 
+// Point-tile position (instance b, tile rt inside it) of the one-tile
+// kernels, advanced by counting: they take contiguous runs of tiles per CTA
+// (or a single instance), and a 64-bit division per point tile, with only
+// the few K-steps of one centroid tile behind it, was a large share of
+// their instructions.  The other kernels divide once per point tile,
+// amortised over its centroid tiles.
+struct TileCount {
+  int b;
+  int64_t rt;
+  __device__ __forceinline__ TileCount(int64_t t0, int64_t tpi, int B) : b(0), rt(t0) {
+    if (B > 1) {
+      b = static_cast<int>(t0 / tpi);
+      rt = t0 - static_cast<int64_t>(b) * tpi;
+    }
+  }
+  // to the next tile of this CTA (B > 1 implies step 1 in these kernels)
+  __device__ __forceinline__ void advance(int64_t step, int64_t tpi, int B) {
+    if (B == 1) {
+      rt += step;
+    } else if (++rt == tpi) {
+      rt = 0;
+      ++b;
+    }
+  }
+};
+
 // ONE_CT: one centroid tile per point tile (K <= BN), kept resident per
 // instance (see the producer and the MMA issuer).
 template <int BN, bool TF32, bool PAIR, bool ONE_CT>
@@ -366,9 +392,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if constexpr (PAIR) tma_load_3d_pair(dst, map, x, y, z, mapa_shared(smem_addr(bar), 0));
         else tma_load_3d(dst, map, x, y, z, bar);
       };
+      TileCount tcn(t_first, p.tiles_per_inst, p.B);
       for (int64_t t = t_first; ok && t < t_end; t += t_step) {
-        const int b = static_cast<int>(t / p.tiles_per_inst);
-        const int rt = static_cast<int>(t - static_cast<int64_t>(b) * p.tiles_per_inst);
+        const int b = ONE_CT ? tcn.b : static_cast<int>(t / p.tiles_per_inst);
+        const int rt = ONE_CT ? static_cast<int>(tcn.rt) : static_cast<int>(t - static_cast<int64_t>(b) * p.tiles_per_inst);
+        if constexpr (ONE_CT) tcn.advance(t_step, p.tiles_per_inst, p.B);
         const int row0 = rt * TM + static_cast<int>(rank) * kTileM;
         if (!mbar_wait(&x_empty[xb], xph ^ 1u, g)) { ok = false; break; }
         uint8_t* xdst = xs + xb * xbb;
@@ -430,12 +458,14 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       uint32_t xph = 0, cph = 0, aph = 0;
       bool ok = true;
       int64_t b_cur = -1;
+      TileCount tcn(t_first, p.tiles_per_inst, p.B);
       for (int64_t t = t_first; ok && t < t_end; t += t_step) {
         if (!mbar_wait(&x_full[xb], xph, g)) { ok = false; break; }
         const uint32_t xaddr = smem_addr(xs + xb * xbb);
         bool keep = false;  // stage cst already holds this instance's tile
         if constexpr (ONE_CT) {
-          const int64_t b = t / p.tiles_per_inst;
+          const int64_t b = tcn.b;
+          tcn.advance(t_step, p.tiles_per_inst, p.B);
           keep = b == b_cur;
           if (!keep && b_cur >= 0) {  // leave the previous instance's stage
             commit(&c_empty[cst]);
@@ -497,9 +527,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const uint32_t kmask = ~31u + p.zero;
     const uint32_t a_empty_lead = PAIR ? mapa_shared(smem_addr(&a_empty[grp]), 0) : 0u;
     int64_t ct0 = 0;  // centroid tiles this CTA processed before the current point tile
+    TileCount tcn(t_first, p.tiles_per_inst, p.B);
     for (int64_t t = t_first; ok && t < t_end; t += t_step, ct0 += nct) {
-      const int b = static_cast<int>(t / p.tiles_per_inst);
-      const int64_t rt = t - static_cast<int64_t>(b) * p.tiles_per_inst;
+      const int b = ONE_CT ? tcn.b : static_cast<int>(t / p.tiles_per_inst);
+      const int64_t rt = ONE_CT ? tcn.rt : t - static_cast<int64_t>(b) * p.tiles_per_inst;
+      if constexpr (ONE_CT) tcn.advance(t_step, p.tiles_per_inst, p.B);
       const int64_t row = rt * TM + static_cast<int64_t>(rank) * kTileM + r_local;
       const bool valid = row < p.rows;
       float best = CUDART_INF_F;
