@@ -105,7 +105,7 @@ __device__ __forceinline__ int clamp_id(int v, int64_t hi) {
   return v < 0 ? 0 : (v >= hi ? static_cast<int>(hi - 1) : v);
 }
 
-template <int LPR, bool BF16, bool RS, class FinalStore>
+template <int LPR, bool BF16, bool RS, bool PF, class FinalStore>
 __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict__ X, int row_bytes, int D, int K,
                                                       const int2* __restrict__ pairs, int64_t n, int64_t q0,
                                                       int64_t q1, int lane, int* slot_k, float* slot_v,
@@ -201,6 +201,15 @@ __device__ __forceinline__ void warp_range_sums_keyed(const uint8_t* __restrict_
       else
         buf[s] = make_uint4(0u, 0u, 0u, 0u);
     }
+    // PF: the next batch's rows are pulled into L2 (hints, one per 128-byte
+    // line, each lane its own next position) while this batch is summed,
+    // so its loads wait on L2 rather than on DRAM
+    if constexpr (PF) {
+      if (in_batch && pn + lane < q1) {
+        const uint8_t* nrow = X + static_cast<int64_t>(clamp_id(pv.x, n)) * row_bytes;
+        for (int off = 0; off < row_bytes; off += 128) prefetch_l2(nrow + off);
+      }
+    }
     // ... then the runs inside it are split from registers
     if (starts == 0u) {
 #pragma unroll
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(256, 4) k_segsum(const uint8_t* __restrict__ X
   const int64_t Lw = P / W;
   const int64_t q0 = p0 + warp * Lw < p1 ? p0 + warp * Lw : p1;
   const int64_t q1 = q0 + Lw < p1 ? q0 + Lw : p1;
-  warp_range_sums_keyed<LPR, BF16, false>(X, row_bytes, D, K, pairs, n, q0, q1, lane, slot_k + 2 * warp,
+  warp_range_sums_keyed<LPR, BF16, false, false>(X, row_bytes, D, K, pairs, n, q0, q1, lane, slot_k + 2 * warp,
                                    slot_v + 2 * warp * D, [&](int k, const float (&acc)[8]) {
                                      store_row<LPR, BF16>(sums + static_cast<int64_t>(k) * D, row_bytes, lane, acc,
                                                           1.f);
@@ -854,7 +863,7 @@ __global__ void __launch_bounds__(256) k_small_update(const SmallK p) {
   const int L = (N + W - 1) / W;
   const int q0 = warp * L < N ? warp * L : N;
   const int q1 = q0 + L < N ? q0 + L : N;
-  warp_range_sums_keyed<LPR, BF16, true>(
+  warp_range_sums_keyed<LPR, BF16, true, true>(
       X, p.row_bytes, D, K, pairs, N, q0, q1, lane, slot_k + 2 * warp, slot_v + 2 * warp * D,
       [&](int k, const float (&v)[8], int col0, int nv, bool writer) {
         // mean = sum x (1 / count): one division per cluster (within 1.5 ulp of
