@@ -384,9 +384,10 @@ int km_finalize_sums(const double* sums, const double* counts, int K, int D, int
  * The tiling the library chooses for a shape (no device needed): out[0..9) =
  * assignment form (0 one CTA per 128-point tile, 1 CTA pairs), centroid tile
  * width BN, point-tile buffers, centroid stages, shared memory bytes of the
- * assignment kernel, K padded to BN, sort passes, sort block size, and 1
- * when the update runs as the fused kernel with one CTA per instance
- * (batched problems of at most 8192 points and 1024 clusters), else 0.  The
+ * assignment kernel, K padded to BN, sort passes, sort block size, and the
+ * update's form: 0 the sort chain (count, column scan, scatter, segmented
+ * sum, finalise), 1 the fused kernel with one CTA per instance (batched
+ * problems of at most 8192 points and 1024 clusters).  The
  * choice is a static function of the shape and the shared-memory limit
  * (KM_ASSIGN_FORM and KM_ASSIGN_TILE=pair,BN,XB,CS override it; an override
  * that does not fit is refused).

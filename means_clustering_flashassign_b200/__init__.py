@@ -407,7 +407,7 @@ def plan(op: int, B: int, N: int, D: int, K: int, dtype: int, chunk_rows: int = 
     """The tiling the library would use for this shape (host-only query)."""
     out = (ctypes.c_int64 * 9)()
     _check(library().km_plan_describe(op, B, N, D, K, dtype, chunk_rows, ctypes.cast(out, ctypes.c_void_p)))
-    keys = ("pair", "BN", "XB", "CS", "smem", "Kp", "sort_passes", "sort_block", "small_update")
+    keys = ("pair", "BN", "XB", "CS", "smem", "Kp", "sort_passes", "sort_block", "update_form")
     return {k: int(v) for k, v in zip(keys, out)}
 
 

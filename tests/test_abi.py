@@ -122,12 +122,13 @@ def test_plan_describes_the_chosen_tiling():
     r = km.plan(km.OP_FIT, 1, 16384, 32, 64, km.F32)
     assert (r["pair"], r["BN"]) == (0, 64)  # pairs need 128-wide tiles
     assert km.plan(km.OP_FIT, 1, 1 << 22, 128, 16384, km.BF16)["sort_passes"] == 2
-    # the fused one-CTA-per-instance update: batched, N <= 8192, K <= 1024,
-    # not for the host-streamed fit
-    assert q["small_update"] == 1 and p["small_update"] == 0
-    assert km.plan(km.OP_UPDATE, 2, 8192, 256, 1024, km.BF16)["small_update"] == 1
-    assert km.plan(km.OP_UPDATE, 2, 8193, 64, 256, km.BF16)["small_update"] == 0
-    assert km.plan(km.OP_UPDATE, 2, 4096, 64, 1025, km.BF16)["small_update"] == 0
+    # the update's form: the fused one-CTA-per-instance kernel for batched
+    # problems (N <= 8192, K <= 1024), else the sort chain
+    assert q["update_form"] == 1 and p["update_form"] == 0 and r["update_form"] == 0
+    assert km.plan(km.OP_UPDATE, 2, 8192, 256, 1024, km.BF16)["update_form"] == 1
+    assert km.plan(km.OP_UPDATE, 2, 8193, 64, 256, km.BF16)["update_form"] == 0
+    assert km.plan(km.OP_UPDATE, 2, 4096, 64, 1025, km.BF16)["update_form"] == 0
+    assert km.plan(km.OP_UPDATE, 1, 4096, 64, 256, km.BF16)["update_form"] == 0
 
 
 @pytest.mark.parametrize("N,block", [(16384, 2048), (147 * 4096, 2048), (147 * 4096 + 1, 4096), (1 << 20, 4096),

@@ -146,7 +146,7 @@ def test_update_batched_fused_path(B, N, D, K, dtype):
     idx = rng.integers(0, K, (B, N)).astype(np.int32)
     idx[:, : N // 5] = K - 1
     Cprev = torch.randn(B, K, D, device=DEV)
-    assert km.plan(km.OP_UPDATE, B, N, D, K, km.BF16 if dtype == "bf16" else km.F32)["small_update"]
+    assert km.plan(km.OP_UPDATE, B, N, D, K, km.BF16 if dtype == "bf16" else km.F32)["update_form"] == 1
     C, counts = km.update(X, torch.from_numpy(idx).to(DEV), Cprev.clone())
     torch.cuda.synchronize()
     for b in range(B):
