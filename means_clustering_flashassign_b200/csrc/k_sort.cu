@@ -436,14 +436,34 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
 
 // start[k] for every k in [0, K] from the sorted pairs: each change point i
 // (or the ends) writes the starts of all clusters between the two keys.
+// A thread covers kBoundsPer consecutive positions (two 16-byte loads).
+constexpr int kBoundsPer = 4;
 __global__ void k_bounds(const int2* __restrict__ sorted, int64_t n, int K, int32_t* __restrict__ start) {
   pdl_trigger();
   pdl_wait();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i > n) return;
-  const int a = i == 0 ? -1 : clamp_key(sorted[i - 1].y, K);
-  const int c = i == n ? K : clamp_key(sorted[i].y, K);
-  for (int k = a + 1; k <= c; ++k) start[k] = static_cast<int32_t>(i);
+  const int64_t i0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * kBoundsPer;
+  if (i0 > n) return;
+  int key[kBoundsPer];
+  if (i0 + kBoundsPer <= n) {
+    const int4* q = reinterpret_cast<const int4*>(sorted + i0);  // 32-byte aligned: i0 is a multiple of 4
+    const int4 u = q[0], w = q[1];
+    key[0] = u.y;
+    key[1] = u.w;
+    key[2] = w.y;
+    key[3] = w.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kBoundsPer; ++j) key[j] = i0 + j < n ? sorted[i0 + j].y : K;
+  }
+  int a = i0 == 0 ? -1 : clamp_key(sorted[i0 - 1].y, K);
+#pragma unroll
+  for (int j = 0; j < kBoundsPer; ++j) {
+    const int64_t i = i0 + j;
+    if (i > n) break;
+    const int c = i == n ? K : clamp_key(key[j], K);
+    for (int k = a + 1; k <= c; ++k) start[k] = static_cast<int32_t>(i);
+    a = c;
+  }
 }
 
 // Digits per scatter thread for radix R: R / 256, at least 1.
@@ -536,7 +556,7 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   if (c.passes > 1) {
-    const int64_t cnt = a.n + 1;
+    const int64_t cnt = (a.n + 1 + kBoundsPer - 1) / kBoundsPer;  // threads
     count_launch();
     e = launch_chained(k_bounds, dim3(static_cast<unsigned>((cnt + 255) / 256)), dim3(256), 0, s, a.pairs, a.n, a.K,
                        a.start);
