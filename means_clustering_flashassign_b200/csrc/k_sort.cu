@@ -45,9 +45,10 @@ constexpr int kSortWarps = kSortThreads / 32;
 // (all loads issued first).  The lanes of a step with equal digits are found
 // with one ballot per digit bit, each lane keeping the lanes whose bit agrees
 // with its own; the lowest of them adds their number to the block's count.
-// With rk (pass 0): rk[i] = key | rank << 20 | (count - 1) << 25, the key's
-// rank among the equal digits of its aligned 32-key group and their number,
-// as the scatter ranks them.
+// With rk: rk[i] = key | rank << 20 | (count - 1) << 25, the key's rank
+// among the equal digits of its aligned 32-key group and their number, as
+// the scatter ranks them (on a pass over pairs the key bits are 0: that
+// scatter reads the key from the pair).
 constexpr int kCountThreads = 1024;
 template <int STEPS, bool PAIRS>
 __global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __restrict__ keys,
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(kCountThreads) k_sort_count(const int32_t* __r
     if (!valid) continue;
     const int rank = __popc(peers & lt), cnt = __popc(peers);
     if (rank == 0) atomicAdd(&sh[dig], cnt);
-    if (!PAIRS && rk) rk[i] = key[s] | (rank << 20) | ((cnt - 1) << 25);
+    if (rk) rk[i] = (PAIRS ? 0 : key[s]) | (rank << 20) | ((cnt - 1) << 25);
   }
   __syncthreads();
   int32_t* out = blkhist + static_cast<int64_t>(blockIdx.x) * R;
@@ -187,6 +188,29 @@ __device__ __forceinline__ void ld_run(const int32_t* p, int32_t (&v)[RPT]) {
     v[1] = x.y;
   } else {
     v[0] = p[0];
+  }
+}
+
+// ld_run from device memory through L2 only (ld.global.cg): for arrays an
+// earlier kernel of the same chained sequence may have read into this SM's
+// L1 before a later kernel rewrote them (see k_sort_scatter).
+template <int RPT>
+__device__ __forceinline__ void ld_run_l2(const int32_t* p, int32_t (&v)[RPT]) {
+  if constexpr (RPT % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < RPT / 4; ++q) {
+      const int4 x = __ldcg(reinterpret_cast<const int4*>(p) + q);
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+    }
+  } else if constexpr (RPT == 2) {
+    const int2 x = __ldcg(reinterpret_cast<const int2*>(p));
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+    v[0] = __ldcg(p);
   }
 }
 
@@ -288,9 +312,15 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   auto valid = [&](int s) { return 32 * s < nw; };
   auto digit = [&](int32_t k) { return (k >> shift) & (R - 1); };
   int32_t key[IPT], val[PAIRS ? IPT : 1];
-  // PRE: the key word also holds the point's rank among the equal digits of
-  // its 32-point group (bits 20..24) and the group's count of that digit
-  // minus one (bits 25..29), as the count kernel found them
+  // PRE: the key word (keys_in) also holds the point's rank among the equal
+  // digits of its 32-point group (bits 20..24) and the group's count of that
+  // digit minus one (bits 25..29), as the count kernel found them; over
+  // pairs only those bits are used.  The rank array, like the digit totals,
+  // is rewritten by the second pass after the first pass's scatter read it,
+  // and a chained kernel can become resident while its predecessors still
+  // run: reading such arrays through the non-coherent L1 path returned the
+  // first pass's lines in the second pass (repeated fits stopped being
+  // bit-identical), so they are read through L2 (ld.global.cg).
   uint32_t pre[PRE ? IPT : 1];
 #pragma unroll
   for (int s = 0; s < IPT; ++s) {  // all loads first
@@ -299,8 +329,9 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
       const int2 pk = i < n ? pairs_in[i] : make_int2(0, 0);
       val[s] = pk.x;
       key[s] = pk.y;
+      if constexpr (PRE) pre[s] = i < n ? static_cast<uint32_t>(__ldcg(keys_in + i)) >> 20 : 0u;
     } else if constexpr (PRE) {
-      const int32_t w = i < n ? keys_in[i] : 0;
+      const int32_t w = i < n ? __ldcg(keys_in + i) : 0;
       key[s] = clamp_key(w & 0xFFFFF, K);
       pre[s] = static_cast<uint32_t>(w) >> 20;
     } else {
@@ -312,11 +343,11 @@ __global__ void __launch_bounds__(kSortThreads, RPT >= 16 ? 1 : (IPT <= 8 && RPT
   // its segment plus the totals of the earlier segments)
   int32_t tot[RPT] = {}, bo[RPT] = {};
   if (owner) {
-    ld_run<RPT>(boff + d0, bo);
+    ld_run_l2<RPT>(boff + d0, bo);
     const int sb = static_cast<int>(static_cast<int64_t>(blockIdx.x) / L);
     for (int s2 = 0; s2 < S; ++s2) {
       int32_t v[RPT];
-      ld_run<RPT>(segtot + static_cast<int64_t>(s2) * R + d0, v);
+      ld_run_l2<RPT>(segtot + static_cast<int64_t>(s2) * R + d0, v);
 #pragma unroll
       for (int j = 0; j < RPT; ++j) {
         tot[j] += v[j];
@@ -513,16 +544,16 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     int32_t* bh = ps == 0 ? a.blkhist : a.blkhist1;
     count_launch(3);  // count, colscan, scatter
     const dim3 hgrid(static_cast<unsigned>(nblk));
-    int32_t* rk = pairs_in ? nullptr : a.rk;
+    int32_t* rk = a.rk;
     // T = 4096 or 2048 keys per block: 4 or 2 steps per warp of 1024 threads
     if (c.IPT == 16)
       e = pairs_in ? launch_chained(k_sort_count<4, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
-                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, nullptr, a.K)
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, rk, a.K)
                    : launch_chained(k_sort_count<4, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
                                     a.n, c.shift[ps], R, bits, bh, rk, a.K);
     else
       e = pairs_in ? launch_chained(k_sort_count<2, true>, hgrid, dim3(kCountThreads), R * 4, s, nullptr,
-                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, nullptr, a.K)
+                                    a.pairs_tmp, a.n, c.shift[ps], R, bits, bh, rk, a.K)
                    : launch_chained(k_sort_count<2, false>, hgrid, dim3(kCountThreads), R * 4, s, a.keys, nullptr,
                                     a.n, c.shift[ps], R, bits, bh, rk, a.K);
     if (e != cudaSuccess) return e;
@@ -538,7 +569,12 @@ cudaError_t launch_sort(const Plan& p, const SortArgs& a, cudaStream_t s) {
     const size_t sm = scatter_smem(R, c.T);
     int32_t* st = (last && c.passes == 1) ? a.start : nullptr;
     const int rpt = scatter_rpt(R);
-    if (pairs_in)
+    if (pairs_in && rk)
+      e = c.IPT == 16 ? launch_scatter_r<16, true, true>(rpt, nblk, sm, s, rk, a.pairs_tmp, a.n, c.shift[ps], R,
+                                                         bits, bh, a.total, S, L, out, perm, st, a.K)
+                      : launch_scatter_r<8, true, true>(rpt, nblk, sm, s, rk, a.pairs_tmp, a.n, c.shift[ps], R,
+                                                        bits, bh, a.total, S, L, out, perm, st, a.K);
+    else if (pairs_in)
       e = c.IPT == 16 ? launch_scatter_r<16, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
                                                           bits, bh, a.total, S, L, out, perm, st, a.K)
                       : launch_scatter_r<8, true, false>(rpt, nblk, sm, s, nullptr, a.pairs_tmp, a.n, c.shift[ps], R,
