@@ -118,3 +118,21 @@ def test_chained_launch_helper_arms_and_breaks():
     m = re.search(r"launch_chained\s*\(", text)
     body = _body(text, m.end())
     assert "chain_armed()" in body and "chain_arm();" in body and "chain_break();" in body
+
+
+def test_scatter_reads_the_arrays_both_sort_passes_rewrite_through_l2():
+    # The rank buffer and the digit totals are read by the first pass's
+    # scatter and rewritten by the second pass before its scatter reads them;
+    # chained kernels become resident early, so those reads must bypass the
+    # non-coherent L1 path (a stale first-pass line broke repeated two-pass
+    # fits' bit-identity on the GPU).
+    text = _src("k_sort.cu")
+    start = text.index("k_sort_scatter(")
+    body = _body(text, start)
+    # the ranks (both passes) through L2; the plain key read is the
+    # unranked first pass's, whose keys (the assignment) no kernel of the
+    # iteration rewrites
+    assert body.count("__ldcg(keys_in + i)") == 2
+    assert re.search(r"ld_run_l2<RPT>\(segtot", body)
+    assert re.search(r"ld_run_l2<RPT>\(boff", body)
+    assert not re.search(r"ld_run<RPT>\(segtot", body)
