@@ -46,39 +46,6 @@ __device__ __forceinline__ void add16(float (&acc)[8], const uint4 v) {
   }
 }
 
-// Sum rows perm[lo..hi) into this lane's column chunk; every lane of the warp
-// must call it with the same lo/hi.  Afterwards lanes < LPR hold the column
-// sums of their 16-byte chunk (reduced across the row slots in a fixed order).
-template <int LPR, bool BF16>
-__device__ __forceinline__ void seg_rows_sum(const uint8_t* __restrict__ X, int row_bytes,
-                                             const int32_t* perm, int64_t lo, int64_t hi, int lane,
-                                             float (&acc)[8]) {
-  using G = RowGeom<LPR>;
-  const int sub = lane / LPR;
-  const int cl = lane % LPR;
-  const bool active = cl * 16 < row_bytes;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int64_t b0 = lo; b0 < hi; b0 += G::BATCH) {
-    const int myr = (lane < G::BATCH && b0 + lane < hi) ? perm[b0 + lane] : -1;
-    uint4 buf[G::STEPS];
-#pragma unroll
-    for (int s = 0; s < G::STEPS; ++s) {
-      const int r = __shfl_sync(0xffffffffu, myr, s * G::RPS + sub);
-      if (r >= 0 && active)
-        buf[s] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(r) * row_bytes + cl * 16));
-      else
-        buf[s] = make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int s = 0; s < G::STEPS; ++s) add16<BF16>(acc, buf[s]);
-  }
-#pragma unroll
-  for (int o = LPR; o < 32; o <<= 1)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-}
-
 // Store a lane's column sums (lanes < LPR) to dst[0..D) floats, scaled.
 template <int LPR, bool BF16>
 __device__ __forceinline__ void store_row(float* dst, int row_bytes, int lane, const float (&acc)[8], float scale) {
